@@ -1,0 +1,189 @@
+"""fp64 CPU oracle for tiled GQA prefill attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never touches it and shares no code with it.
+
+The arithmetic lives in ``tfa_oracle.c`` (plain C, fp64, OpenMP over rows);
+this module only builds it with gcc, marshals arrays through ctypes and
+returns numpy float64 results.  See the C file's header for the definition
+and the passages of the pages it follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tfa_oracle.c")
+_LIB = os.path.join(_HERE, "libtfa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# Planted mistakes understood by attention_mutant(); see tfa_oracle.c.
+MUTATIONS = {
+    "causal_sees_next": 1,
+    "window_one_wider": 2,
+    "head_modulo": 3,
+    "no_prefix_offset": 4,
+    "drop_scale": 5,
+    "keymask_inverted": 6,
+    "empty_row_uniform": 7,
+}
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (portable flags: no -march=native, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O3", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.oracle_attention.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
+                                             i32, i32, P, P, i64, i32]
+            lib.oracle_attention.restype = i32
+            lib.oracle_attention_mutant.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                                    f64, i32, i32, P, i32]
+            lib.oracle_attention_mutant.restype = i32
+            lib.oracle_softmax_weights.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64,
+                                                   i32, i32, P, i32, i32, i32]
+            lib.oracle_softmax_weights.restype = i32
+            lib.oracle_count_pairs.argtypes = [i32, i32, i32, i32, i32, i32, P]
+            lib.oracle_count_pairs.restype = i64
+            lib.oracle_allowed.argtypes = [ctypes.c_long] * 4 + [i32, ctypes.c_long, P]
+            lib.oracle_allowed.restype = i32
+            lib.oracle_attention_blockwise.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32,
+                                                       f64, i32, i32, P, i32, i32, i32, P]
+            lib.oracle_attention_blockwise.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 tensor (torch) or uint16 array -> contiguous uint16 numpy bit patterns."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("numpy inputs must be uint16 bf16 bit patterns")
+        return np.ascontiguousarray(x)
+    import torch
+
+    if x.dtype != torch.bfloat16:
+        raise TypeError("torch inputs must be bfloat16")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _mask(m):
+    if m is None:
+        return None
+    if not isinstance(m, np.ndarray):
+        m = m.detach().cpu().float().numpy()
+    return np.ascontiguousarray(m, dtype=np.float32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _shape(q, k):
+    B, Hq, L, D = q.shape
+    Bk, Hkv, S, Dk = k.shape
+    if Bk != B or Dk != D:
+        raise ValueError("q/k shapes disagree")
+    return B, Hq, Hkv, L, S, D
+
+
+def attention(q, k, v, *, scale, causal, window=0, key_mask=None, rows=None, threads=0):
+    """Plain fp64 definition.  rows: optional flattened (b*Hq+h)*L+i indices."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    km = _mask(key_mask)
+    if rows is None:
+        out = np.empty((B, Hq, L, D), dtype=np.float64)
+        r_ptr, nr = None, 0
+    else:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        out = np.empty((r.size, D), dtype=np.float64)
+        r_ptr, nr = r.ctypes.data_as(ctypes.c_void_p), r.size
+    rc = _load().oracle_attention(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L, S, D,
+                                  float(scale), int(bool(causal)), int(window), _ptr(km),
+                                  r_ptr, nr, int(threads))
+    if rc:
+        raise ValueError(f"oracle_attention rejected its arguments (code {rc})")
+    return out
+
+
+def attention_mutant(q, k, v, *, scale, causal, window=0, key_mask=None, mutation):
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    km = _mask(key_mask)
+    out = np.empty((B, Hq, L, D), dtype=np.float64)
+    code = MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
+    rc = _load().oracle_attention_mutant(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L,
+                                         S, D, float(scale), int(bool(causal)), int(window),
+                                         _ptr(km), code)
+    if rc:
+        raise ValueError(f"oracle_attention_mutant rejected its arguments (code {rc})")
+    return out
+
+
+def attention_blockwise(q, k, v, *, scale, causal, window=0, key_mask=None, bq=128, bk=128,
+                        skip_empty=True):
+    """Tiled online-softmax variant; returns (output, key tiles visited per row block sum)."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    km = _mask(key_mask)
+    out = np.empty((B, Hq, L, D), dtype=np.float64)
+    visited = ctypes.c_int64(0)
+    rc = _load().oracle_attention_blockwise(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv,
+                                            L, S, D, float(scale), int(bool(causal)), int(window),
+                                            _ptr(km), int(bq), int(bk), int(bool(skip_empty)),
+                                            ctypes.byref(visited))
+    if rc:
+        raise ValueError(f"oracle_attention_blockwise rejected its arguments (code {rc})")
+    return out, int(visited.value)
+
+
+def softmax_weights(q, k, *, b, h, scale, causal, window=0, key_mask=None, mutation=0):
+    """L x S softmax weights of one (batch, query head)."""
+    qb, kb = _bits(q), _bits(k)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    km = _mask(key_mask)
+    W = np.empty((L, S), dtype=np.float64)
+    code = MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
+    rc = _load().oracle_softmax_weights(_ptr(qb), _ptr(kb), _ptr(W), B, Hq, Hkv, L, S, D,
+                                        float(scale), int(bool(causal)), int(window), _ptr(km),
+                                        int(b), int(h), code)
+    if rc:
+        raise ValueError(f"oracle_softmax_weights rejected its arguments (code {rc})")
+    return W
+
+
+def allowed(L, S, i, j, *, causal, window=0, key_mask_row=None) -> bool:
+    km = _mask(key_mask_row)
+    return bool(_load().oracle_allowed(L, S, i, j, int(bool(causal)), int(window), _ptr(km)))
+
+
+def visibility(L, S, *, causal, window=0, key_mask_row=None) -> np.ndarray:
+    """L x S boolean matrix of allowed (row, key) pairs."""
+    return np.array([[allowed(L, S, i, j, causal=causal, window=window, key_mask_row=key_mask_row)
+                      for j in range(S)] for i in range(L)], dtype=bool)
+
+
+def count_pairs(B, Hq, L, S, *, causal, window=0, key_mask=None) -> int:
+    km = _mask(key_mask)
+    return int(_load().oracle_count_pairs(B, Hq, L, S, int(bool(causal)), int(window), _ptr(km)))

@@ -1,0 +1,372 @@
+/*
+ * tfa_oracle.c -- plain, slow, fp64 CPU oracle for tiled GQA prefill attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or helper with the
+ * CUDA library; the only thing the two sides have in common is the seeded
+ * input generator, which holds none of the attention arithmetic.
+ *
+ * What it computes (every function below restates it, with its source):
+ *
+ *   For batch b, query head h and new query row i (0 <= i < L), with
+ *   prefix P = S - L, absolute position p = P + i and KV head
+ *   g = floor(h / (Hq / Hkv)):
+ *     key j (0 <= j < S) is ALLOWED iff
+ *       (causal  => j <= p)                      causal mask aligned to the
+ *                                                end of the cached prefix
+ *       (causal && window > 0 => j > p - window) sliding window [p-W+1, p]
+ *       (key_mask == NULL || key_mask[b,j] > 0.5) length-S key mask
+ *     s_j = scale * sum_d q[b,h,i,d] * k[b,g,j,d]       (fp64, exact bf16 upcast)
+ *     no allowed key  -> o[b,h,i,:] = 0
+ *     otherwise       -> m = max s_j, w_j = exp(s_j - m),
+ *                        o[b,h,i,:] = sum_j w_j v[b,g,j,:] / sum_j w_j
+ *
+ * Sources (page title, section):
+ *   tiny-llm "Week 2 Day 5: Tiled Dense Prefill Attention", Task 1 (layout
+ *     Q [B,Hq,L,128], K/V [B,Hkv,S,128]; KV head floor(h/(Hq/Hkv)); the
+ *     online-softmax merge equations m', l', a'), Task 2 (causality aligned to
+ *     the end of the cached prefix: row i sees positions through S-L+i; a
+ *     fully masked row is finite and all zero).
+ *   brotensor "include/brotensor/ops/flash_attention.h" coverage page,
+ *     flash_attention_windowed_forward and flash_attention_decode comments
+ *     (window keeps keys [max(0, p-window+1), p], window <= 0 = unbounded;
+ *     FP32 key mask 1 valid / 0 invalid, positions with mask <= 0.5 dropped,
+ *     combined multiplicatively with the causal/window mask).
+ *   tinygrad "symbolic llm with prefill" compare view, apps/llm.py
+ *     (_attention_inner: scaled_dot_product_attention(..., enable_gqa=True)
+ *     with the causal mask full(-inf).triu(start_pos+1)).
+ *
+ * Inputs are bf16 bit patterns (uint16), upcast exactly to double.  Outputs
+ * are double.  Layouts: q/o [B,Hq,L,D], k/v [B,Hkv,S,D], key_mask [B,S] fp32,
+ * all contiguous row-major.
+ *
+ * The "mutant" entry point exists only so that tests can plant plausible
+ * mistakes in the oracle and show that the pins catch them.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* Mutations a test may plant (0 = the correct oracle). */
+enum {
+    MUT_NONE = 0,
+    MUT_CAUSAL_SEES_NEXT = 1,    /* j <= p + 1 instead of j <= p            */
+    MUT_WINDOW_ONE_WIDER = 2,    /* j >= p - window instead of j > p - W     */
+    MUT_HEAD_MODULO = 3,         /* g = h mod Hkv instead of floor(h / G)    */
+    MUT_NO_PREFIX_OFFSET = 4,    /* causal triangle as if S were L (P = 0)   */
+    MUT_DROP_SCALE = 5,          /* s_j without the scale factor             */
+    MUT_KEYMASK_INVERTED = 6,    /* keep mask <= 0.5 instead of > 0.5        */
+    MUT_EMPTY_ROW_UNIFORM = 7,   /* fully masked row averages all V rows     */
+};
+
+static double bf16_bits_to_f64(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Visibility of key j for new query row i.  tiny-llm Week 2 Day 5, Task 2
+ * (causal offset by the prefix); brotensor flash_attention.h, decode comment
+ * (window [p-window+1, p], window <= 0 unbounded) and forward comment
+ * (key mask <= 0.5 dropped, combined multiplicatively). */
+static int allowed_impl(long L, long S, long i, long j, int causal, long window,
+                        const float *key_mask_row, int mutation)
+{
+    long P = (mutation == MUT_NO_PREFIX_OFFSET) ? 0 : S - L;
+    long p = P + i;
+    if (j < 0 || j >= S) return 0;
+    if (causal) {
+        long last = (mutation == MUT_CAUSAL_SEES_NEXT) ? p + 1 : p;
+        if (j > last) return 0;
+        if (window > 0) {
+            long first = (mutation == MUT_WINDOW_ONE_WIDER) ? p - window : p - window + 1;
+            if (j < first) return 0;
+        }
+    }
+    if (key_mask_row) {
+        int keep = (mutation == MUT_KEYMASK_INVERTED) ? (key_mask_row[j] <= 0.5f)
+                                                      : (key_mask_row[j] > 0.5f);
+        if (!keep) return 0;
+    }
+    return 1;
+}
+
+int oracle_allowed(long L, long S, long i, long j, int causal, long window,
+                   const float *key_mask_row)
+{
+    return allowed_impl(L, S, i, j, causal, window, key_mask_row, MUT_NONE);
+}
+
+/* GQA head mapping: query head h reads KV head floor(h / (Hq / Hkv)).
+ * tiny-llm Week 2 Day 5, Task 1; brotensor flash_attention_decode comment
+ * (each KV head serves Hq/Hkv consecutive query heads). */
+static int kv_head_impl(int h, int Hq, int Hkv, int mutation)
+{
+    if (mutation == MUT_HEAD_MODULO) return h % Hkv;
+    return h / (Hq / Hkv);
+}
+
+static int check_args(const void *q, const void *k, const void *v, const void *o,
+                      int B, int Hq, int Hkv, int L, int S, int D)
+{
+    if (!q || !k || !v || !o) return 1;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || S < L || D < 1) return 2;
+    if (Hq % Hkv != 0) return 3;
+    return 0;
+}
+
+/* One output row, two passes, exact softmax, no tiling. */
+static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
+                    int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                    int causal, int window, const float *key_mask, int mutation,
+                    long row, double *s_buf)
+{
+    long i = row % L;
+    long bh = row / L;
+    int h = (int)(bh % Hq);
+    int b = (int)(bh / Hq);
+    int g = kv_head_impl(h, Hq, Hkv, mutation);
+    (void)B;
+    const uint16_t *qr = q + ((size_t)bh * L + i) * D;
+    const uint16_t *kb = k + ((size_t)b * Hkv + g) * (size_t)S * D;
+    const uint16_t *vb = v + ((size_t)b * Hkv + g) * (size_t)S * D;
+    const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+    double sc = (mutation == MUT_DROP_SCALE) ? 1.0 : scale;
+
+    double m = -INFINITY;
+    int any = 0;
+    for (long j = 0; j < S; ++j) {
+        if (!allowed_impl(L, S, i, j, causal, window, mrow, mutation)) {
+            s_buf[j] = -INFINITY;
+            continue;
+        }
+        double acc = 0.0;
+        const uint16_t *kr = kb + (size_t)j * D;
+        for (int d = 0; d < D; ++d) acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kr[d]);
+        s_buf[j] = sc * acc;
+        if (s_buf[j] > m) m = s_buf[j];
+        any = 1;
+    }
+    for (int d = 0; d < D; ++d) out[d] = 0.0;
+    if (!any) {
+        /* tiny-llm Week 2 Day 5, Task 2: no probability mass -> finite zeros. */
+        if (mutation == MUT_EMPTY_ROW_UNIFORM) {
+            for (long j = 0; j < S; ++j)
+                for (int d = 0; d < D; ++d) out[d] += bf16_bits_to_f64(vb[(size_t)j * D + d]) / (double)S;
+        }
+        return;
+    }
+    double denom = 0.0;
+    for (long j = 0; j < S; ++j) {
+        if (s_buf[j] == -INFINITY) continue;
+        double w = exp(s_buf[j] - m);
+        denom += w;
+        const uint16_t *vr = vb + (size_t)j * D;
+        for (int d = 0; d < D; ++d) out[d] += w * bf16_bits_to_f64(vr[d]);
+    }
+    for (int d = 0; d < D; ++d) out[d] /= denom;
+}
+
+static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                          int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                          int causal, int window, const float *key_mask,
+                          const int64_t *rows, int64_t nrows, int nthreads, int mutation)
+{
+    int rc = check_args(q, k, v, o, B, Hq, Hkv, L, S, D);
+    if (rc) return rc;
+    int64_t total = rows ? nrows : (int64_t)B * Hq * L;
+    if (rows) {
+        for (int64_t r = 0; r < nrows; ++r)
+            if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq * L) return 4;
+    }
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)S);
+        if (!s_buf) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (int64_t r = 0; r < total; ++r) {
+            if (!s_buf) continue;
+            long row = rows ? (long)rows[r] : (long)r;
+            one_row(q, k, v, o + (size_t)r * D, B, Hq, Hkv, L, S, D, scale, causal, window,
+                    key_mask, mutation, row, s_buf);
+        }
+        free(s_buf);
+    }
+    return failed ? 5 : 0;
+}
+
+/* Plain definition.  rows: optional list of flattened (b*Hq + h)*L + i row
+ * indices; o then holds nrows x D values in that order.  rows == NULL computes
+ * every row and o is [B,Hq,L,D].  Returns 0 on success. */
+int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                     int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                     int causal, int window, const float *key_mask,
+                     const int64_t *rows, int64_t nrows, int nthreads)
+{
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                          rows, nrows, nthreads, MUT_NONE);
+}
+
+/* The same definition with one planted mistake; for mutation tests only. */
+int oracle_attention_mutant(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                            int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                            int causal, int window, const float *key_mask, int mutation)
+{
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                          NULL, 0, 1, mutation);
+}
+
+/* Row-normalised softmax weights of one (b, h): W is L x S, zero where the
+ * key is not allowed, rows of a fully masked query all zero.  Same
+ * definition as oracle_attention, stopped before the weighted sum of V. */
+int oracle_softmax_weights(const uint16_t *q, const uint16_t *k, double *W,
+                           int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                           int causal, int window, const float *key_mask, int b, int h,
+                           int mutation)
+{
+    if (!q || !k || !W) return 1;
+    if (B < 1 || Hq < 1 || Hkv < 1 || L < 1 || S < L || D < 1 || Hq % Hkv) return 2;
+    if (b < 0 || b >= B || h < 0 || h >= Hq) return 4;
+    int g = kv_head_impl(h, Hq, Hkv, mutation);
+    const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+    double sc = (mutation == MUT_DROP_SCALE) ? 1.0 : scale;
+    for (long i = 0; i < L; ++i) {
+        double *wr = W + (size_t)i * S;
+        const uint16_t *qr = q + (((size_t)b * Hq + h) * L + i) * D;
+        double m = -INFINITY;
+        for (long j = 0; j < S; ++j) {
+            wr[j] = -INFINITY;
+            if (!allowed_impl(L, S, i, j, causal, window, mrow, mutation)) continue;
+            const uint16_t *kr = k + (((size_t)b * Hkv + g) * S + j) * D;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kr[d]);
+            wr[j] = sc * acc;
+            if (wr[j] > m) m = wr[j];
+        }
+        double denom = 0.0;
+        for (long j = 0; j < S; ++j) {
+            wr[j] = (wr[j] == -INFINITY) ? 0.0 : exp(wr[j] - m);
+            denom += wr[j];
+        }
+        if (denom > 0.0)
+            for (long j = 0; j < S; ++j) wr[j] /= denom;
+    }
+    return 0;
+}
+
+/* Brute-force count of allowed (b, h, i, j) quadruples: the "unmasked pairs"
+ * whose 4*D flops the throughput metric counts. */
+int64_t oracle_count_pairs(int B, int Hq, int L, int S, int causal, int window,
+                           const float *key_mask)
+{
+    int64_t n = 0;
+    for (int b = 0; b < B; ++b) {
+        const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+        int64_t nb = 0;
+        for (long i = 0; i < L; ++i)
+            for (long j = 0; j < S; ++j) nb += allowed_impl(L, S, i, j, causal, window, mrow, MUT_NONE);
+        n += nb * Hq;
+    }
+    return n;
+}
+
+/* Tiled online-softmax variant, following the merge of tiny-llm Week 2 Day 5,
+ * Task 1: per row keep FP-accumulated running max m, sum l and weighted value
+ * accumulator a; for each key tile with tile maximum m_b, tile sum l_b and
+ * tile accumulator a_b:
+ *     m' = max(m, m_b)
+ *     l' = e^(m - m') l + e^(m_b - m') l_b
+ *     a' = e^(m - m') a + e^(m_b - m') a_b
+ * and finally out = a' / l'.  Key tiles are BK wide; rows are grouped in
+ * blocks of BQ, and when skip_empty is set a key tile that has no allowed
+ * (row, key) pair for ANY row of the block is skipped without reading K/V
+ * (the masked-tile skipping of mlx-lm PR "Skip fully masked key tiles in Flint
+ * sliding-window prefill").  A tile with no allowed key for one row contributes
+ * nothing to that row ("padded score cells contribute no probability mass").
+ * Exists so tests can show that tiling, merging and skipping leave the plain
+ * definition's result unchanged. */
+int oracle_attention_blockwise(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                               int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                               int causal, int window, const float *key_mask,
+                               int BQ, int BK, int skip_empty, int64_t *tiles_visited)
+{
+    int rc = check_args(q, k, v, o, B, Hq, Hkv, L, S, D);
+    if (rc) return rc;
+    if (BQ < 1 || BK < 1) return 2;
+    int64_t visited = 0;
+    double *a = (double *)malloc(sizeof(double) * (size_t)D);
+    double *ab = (double *)malloc(sizeof(double) * (size_t)D);
+    double *sb = (double *)malloc(sizeof(double) * (size_t)BK);
+    if (!a || !ab || !sb) { free(a); free(ab); free(sb); return 5; }
+    for (int b = 0; b < B; ++b)
+    for (int h = 0; h < Hq; ++h) {
+        int g = kv_head_impl(h, Hq, Hkv, MUT_NONE);
+        const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+        for (long i0 = 0; i0 < L; i0 += BQ) {
+            long i1 = (i0 + BQ < L) ? i0 + BQ : L;
+            for (long i = i0; i < i1; ++i) {
+                const uint16_t *qr = q + (((size_t)b * Hq + h) * L + i) * D;
+                double m = -INFINITY, l = 0.0;
+                for (int d = 0; d < D; ++d) a[d] = 0.0;
+                for (long j0 = 0; j0 < S; j0 += BK) {
+                    long j1 = (j0 + BK < S) ? j0 + BK : S;
+                    if (skip_empty) {
+                        int live = 0;
+                        for (long ii = i0; ii < i1 && !live; ++ii)
+                            for (long j = j0; j < j1 && !live; ++j)
+                                live = allowed_impl(L, S, ii, j, causal, window, mrow, MUT_NONE);
+                        if (!live) continue;
+                    }
+                    if (i == i0) ++visited;
+                    double mb = -INFINITY;
+                    for (long j = j0; j < j1; ++j) {
+                        sb[j - j0] = -INFINITY;
+                        if (!allowed_impl(L, S, i, j, causal, window, mrow, MUT_NONE)) continue;
+                        const uint16_t *kr = k + (((size_t)b * Hkv + g) * S + j) * D;
+                        double acc = 0.0;
+                        for (int d = 0; d < D; ++d) acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kr[d]);
+                        sb[j - j0] = scale * acc;
+                        if (sb[j - j0] > mb) mb = sb[j - j0];
+                    }
+                    if (mb == -INFINITY) continue; /* no mass in this tile for this row */
+                    double lb = 0.0;
+                    for (int d = 0; d < D; ++d) ab[d] = 0.0;
+                    for (long j = j0; j < j1; ++j) {
+                        if (sb[j - j0] == -INFINITY) continue;
+                        double w = exp(sb[j - j0] - mb);
+                        lb += w;
+                        const uint16_t *vr = v + (((size_t)b * Hkv + g) * S + j) * D;
+                        for (int d = 0; d < D; ++d) ab[d] += w * bf16_bits_to_f64(vr[d]);
+                    }
+                    double mn = (m > mb) ? m : mb;
+                    double fo = (m == -INFINITY) ? 0.0 : exp(m - mn);
+                    double fb = exp(mb - mn);
+                    l = fo * l + fb * lb;
+                    for (int d = 0; d < D; ++d) a[d] = fo * a[d] + fb * ab[d];
+                    m = mn;
+                }
+                double *out = o + (((size_t)b * Hq + h) * L + i) * D;
+                for (int d = 0; d < D; ++d) out[d] = (l > 0.0) ? a[d] / l : 0.0;
+            }
+        }
+    }
+    free(a); free(ab); free(sb);
+    if (tiles_visited) *tiles_visited = visited;
+    return 0;
+}

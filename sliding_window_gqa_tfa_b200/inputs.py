@@ -1,0 +1,94 @@
+"""Seeded synthetic inputs for tiled GQA prefill attention.
+
+This module is the ONE piece shared by the CUDA path's harness and the CPU
+oracle's tests: it draws the arrays both sides consume and holds none of the
+attention arithmetic.
+
+Recipe: a CPU ``torch.Generator`` seeded with ``seed``; fp32 ``randn`` drawn in
+the order Q, K, V (K multiplied by ``k_scale`` before the cast), then, when the
+workload has a key mask, ``rand(B, S) >= 1 - keep`` as the 1/0 fp32 key mask;
+Q/K/V are cast to bf16 (round to nearest even).  The shapes are the model
+shapes the pages use: Qwen3-0.6B (16 query heads, 8 KV heads, head dim 128,
+tiny-llm "Week 2 Day 5"), the Llama geometry of TensorFold PR 3269 (56 query
+heads, 8 KV heads, group 7, head dim 128), the 1024-key sliding window of the
+same PR and of mlx-lm PR 2006 (rotating cache: window - 1 + L keys per chunk),
+and the 2048-token prefill chunks of mlx-lm PR 2006's benchmark.  No public
+dataset is involved.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, replace
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    L: int
+    S: int
+    D: int
+    causal: bool = True
+    window: int = 0
+    key_mask_keep: float | None = None  # None: no key mask; else Bernoulli keep prob
+    k_scale: float = 1.0
+    scale: float | None = None  # None: 1/sqrt(D)
+
+    @property
+    def softmax_scale(self) -> float:
+        return self.scale if self.scale is not None else 1.0 / math.sqrt(self.D)
+
+    @property
+    def prefix(self) -> int:
+        return self.S - self.L
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+WORKLOADS: dict[str, Workload] = {w.name: w for w in [
+    # 33 query rows over 47 keys (prefix 14): crosses both tile tails.
+    Workload("witness_33x47", B=1, Hq=8, Hkv=2, L=33, S=47, D=128),
+    # Qwen3-0.6B attention geometry, batch 4, 2048-token prompt, no prefix.
+    Workload("qwen3_prefill_b4_2048", B=4, Hq=16, Hkv=8, L=2048, S=2048, D=128),
+    # Llama GQA chunk: 2048 new rows over 8192 keys (prefix 6144), group 7.
+    Workload("llama_gqa_chunk_2048x8192", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128),
+    Workload("llama_gqa_chunk_2048x8192_keymask", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
+             key_mask_keep=0.9),
+    # Rotating-cache sliding window: 1024-key window, chunk 2048, S = 1023 + 2048.
+    Workload("swa_rotating_w1024_2048", B=1, Hq=32, Hkv=8, L=2048, S=3071, D=128, window=1024),
+    # Long-context chunk at 32K keys, K scaled x4 to sharpen the softmax.
+    Workload("long_chunk_2048x32768", B=1, Hq=32, Hkv=8, L=2048, S=32768, D=128, k_scale=4.0),
+    Workload("long_chunk_2048x32768_d64", B=1, Hq=32, Hkv=8, L=2048, S=32768, D=64, k_scale=4.0),
+    Workload("bidirectional_4096", B=1, Hq=32, Hkv=8, L=4096, S=4096, D=128, causal=False,
+             k_scale=4.0),
+]}
+
+# The workload the throughput figure is quoted on.
+HEADLINE = "llama_gqa_chunk_2048x8192"
+
+
+def make_inputs(w: Workload, seed: int = 0):
+    """Return (q, k, v, key_mask) as CPU tensors: bf16 [B,Hq,L,D], bf16 [B,Hkv,S,D] x2,
+    and fp32 [B,S] (or None)."""
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(w.B, w.Hq, w.L, w.D, generator=g, dtype=torch.float32)
+    k = torch.randn(w.B, w.Hkv, w.S, w.D, generator=g, dtype=torch.float32)
+    v = torch.randn(w.B, w.Hkv, w.S, w.D, generator=g, dtype=torch.float32)
+    if w.k_scale != 1.0:
+        k = k * w.k_scale
+    key_mask = None
+    if w.key_mask_keep is not None:
+        key_mask = (torch.rand(w.B, w.S, generator=g) >= (1.0 - w.key_mask_keep)).float()
+    return q.bfloat16(), k.bfloat16(), v.bfloat16(), key_mask
+
+
+def shaped(B, Hq, Hkv, L, S, D, *, causal=True, window=0, key_mask_keep=None, k_scale=1.0,
+           name="custom") -> Workload:
+    """A workload of arbitrary shape drawn by the same recipe (for edge-case tests)."""
+    return Workload(name, B=B, Hq=Hq, Hkv=Hkv, L=L, S=S, D=D, causal=causal, window=window,
+                    key_mask_keep=key_mask_keep, k_scale=k_scale)
