@@ -1,0 +1,140 @@
+/*
+ * tfa.h -- C ABI of the B200 (sm_100a) tiled GQA prefill attention library.
+ *
+ * One operation: dense prefill attention for grouped-query attention, where
+ * L new query rows attend to S = prefix + L keys, under a causal mask offset by
+ * the prefix, an optional sliding window and an optional length-S key mask.
+ *
+ * Definition (for batch b, query head h, new row i, P = S - L, p = P + i,
+ * G = Hq / Hkv, g = floor(h / G)):
+ *   key j is allowed iff (!causal || j <= p)
+ *                     && (!causal || window <= 0 || j > p - window)
+ *                     && (key_mask == NULL || key_mask[b*S + j] > 0.5f)
+ *   o[b,h,i,:] = sum_j softmax_j(scale * q[b,h,i,:] . k[b,g,j,:]) v[b,g,j,:]
+ *   over the allowed j; a row with no allowed key is written as zeros.
+ * Sources: tiny-llm "Week 2 Day 5: Tiled Dense Prefill Attention", Task 1
+ * (layouts, GQA head mapping without replicating K/V, online-softmax merge,
+ * partial-tail guards, BF16 after the final FP32 normalisation) and Task 2
+ * (causality aligned to the end of the cached prefix; fully masked rows are
+ * finite zeros); brotensor "include/brotensor/ops/flash_attention.h"
+ * (flash_attention_decode: window keeps [max(0,p-window+1), p]; key mask is
+ * FP32 1 valid / 0 invalid, dropped when <= 0.5, combined multiplicatively).
+ *
+ * Layout: every tensor is contiguous row-major with the head dimension
+ * innermost, bf16 stored as 16-bit words:
+ *   q, o : [B, Hq,  L, D]        k, v : [B, Hkv, S, D]        key_mask : [B, S] fp32
+ *
+ * Ownership: every pointer passed to tfa_prefill is caller-owned DEVICE memory
+ * on the current CUDA device; the call neither allocates nor frees the tensors
+ * and never reads them on the host.  The library keeps one small status word
+ * per device (allocated on the first call on that device) where the kernel
+ * records a timed-out internal wait.
+ *
+ * Asynchrony: tfa_prefill validates its arguments on the host, then enqueues
+ * the kernel on `stream` and returns; o is fully overwritten when the stream
+ * reaches that point.  Errors found by validation are returned before any
+ * launch, with no side effect.  A device-side failure (a wait that gave up)
+ * is reported by tfa_check_status().
+ */
+#ifndef TFA_H
+#define TFA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *tfa_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    TFA_OK = 0,
+    TFA_ERR_NULL = 1,        /* q, k, v or o is NULL                                      */
+    TFA_ERR_HEADS = 2,       /* Hq < 1, Hkv < 1 or Hq % Hkv != 0                         */
+    TFA_ERR_SHORT_QUERY = 3, /* L < 9: the tiled operator rejects short queries          */
+    TFA_ERR_SHAPE = 4,       /* B < 1, S < L, or a size whose element count overflows    */
+    TFA_ERR_HEAD_DIM = 5,    /* D not 64 or 128                                          */
+    TFA_ERR_WINDOW = 6,      /* window > 0 without causal (no page defines it)           */
+    TFA_ERR_ALIGN = 7,       /* a tensor pointer is not 16-byte aligned, key_mask not 4  */
+    TFA_ERR_CUDA = 8,        /* a CUDA runtime/driver call failed (launch, encode, ...)  */
+    TFA_ERR_TIMEOUT = 9,     /* a kernel wait gave up; the output of that call is invalid */
+    TFA_ERR_SCALE = 10,      /* scale is not finite                                      */
+    TFA_ERR_FLAGS = 11       /* unknown debug flag bits                                  */
+} tfa_status;
+
+/* Minimum query length accepted by the tiled operator (tiny-llm Week 2 Day 5,
+ * Task 1: the direct operator rejects queries shorter than nine rows). */
+#define TFA_MIN_QUERY_ROWS 9
+
+/* tfa_prefill -- tiled dense prefill attention with GQA.
+ *   q        bf16 [B,Hq,L,D] device, 16-byte aligned, read only
+ *   k, v     bf16 [B,Hkv,S,D] device, 16-byte aligned, read only
+ *   o        bf16 [B,Hq,L,D] device, 16-byte aligned, written (every element)
+ *   B        batch, >= 1
+ *   Hq, Hkv  query / KV heads, Hq % Hkv == 0; query head h reads KV head h/(Hq/Hkv)
+ *   L        new query rows, >= TFA_MIN_QUERY_ROWS
+ *   S        keys (cached prefix + L), >= L
+ *   D        head dimension, 64 or 128
+ *   scale    softmax scale applied to q.k (typically 1/sqrt(D)), finite
+ *   causal   nonzero: row i sees keys j <= S-L+i; zero: every key (bidirectional)
+ *   window   > 0 (causal only): additionally j > S-L+i-window; <= 0: no window
+ *   key_mask fp32 [B,S] device (4-byte aligned) or NULL; key j of batch b kept iff > 0.5
+ *   stream   CUDA stream to enqueue on
+ * Returns TFA_OK or a tfa_status code. */
+int tfa_prefill(const void *q, const void *k, const void *v, void *o,
+                int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                int causal, int window, const float *key_mask, tfa_stream_t stream);
+
+/* Debug flags for tfa_prefill_debug. */
+#define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
+#define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */
+#define TFA_DEBUG_SYNC          4u /* synchronize the stream and return the device status */
+
+/* tfa_prefill_debug -- tfa_prefill with debug flags (arguments as above).  With
+ * NO_TILE_SKIP and/or MASK_ALL the result must be bit-identical to tfa_prefill's
+ * (masked-tile skipping is exact: mlx-lm PR "Skip fully masked key tiles in Flint
+ * sliding-window prefill" requires the banded result to equal the single call). */
+int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o,
+                      int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                      int causal, int window, const float *key_mask, tfa_stream_t stream,
+                      unsigned flags);
+
+/* tfa_prefill_host -- the same operation on HOST buffers (q, k, v, key_mask
+ * read, o written; plain or pinned host memory).  The library copies the
+ * inputs to device staging buffers it owns (one set per device, grown on
+ * demand and kept until process exit), runs tfa_prefill on `stream`, copies o
+ * back and synchronizes the stream before returning.  Not safe to call from
+ * two host threads on the same device at once. */
+int tfa_prefill_host(const void *q, const void *k, const void *v, void *o,
+                     int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                     int causal, int window, const float *key_mask, tfa_stream_t stream);
+
+/* tfa_check_status -- synchronizes `stream`, then reads and clears the current
+ * device's status word.  Returns TFA_OK, TFA_ERR_TIMEOUT if a kernel launched
+ * since the last check recorded a wait that gave up, or TFA_ERR_CUDA. */
+int tfa_check_status(tfa_stream_t stream);
+
+/* tfa_status_string -- static description of a status code (never NULL). */
+const char *tfa_status_string(int status);
+
+/* tfa_plan_qtile -- host view of the work enumeration the kernel performs for
+ * one 128-row query tile (rows [128*qtile, min(128*qtile+128, L))):
+ *   *kt_lo, *kt_hi  first and last 128-key tile it visits (kt_hi < kt_lo: none)
+ *   needs_mask      if not NULL, receives kt_hi-kt_lo+1 bytes: 1 where the tile
+ *                   crosses the causal diagonal, the window edge, the key tail
+ *                   or a key mask is present; 0 for interior tiles
+ * Returns TFA_OK, TFA_ERR_SHAPE for an out-of-range tile, or a validation
+ * error for the sizes.  No device work. */
+int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_mask, int qtile,
+                   int *kt_lo, int *kt_hi, unsigned char *needs_mask, int needs_mask_len);
+
+/* Tile sizes of the kernel: 128 query rows x 128 keys per tensor-core tile. */
+#define TFA_BLOCK_Q 128
+#define TFA_BLOCK_K 128
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TFA_H */

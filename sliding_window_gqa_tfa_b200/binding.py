@@ -1,0 +1,220 @@
+"""ctypes binding of libtfa.so -- argument marshalling only.
+
+Every entry point of ``include/tfa.h`` is exposed under the same name and
+takes the same arguments (pointers as Python ints).  ``prefill`` is the
+convenience wrapper a PyTorch user calls: it checks dtypes/devices, allocates
+the output with PyTorch and passes raw pointers and the current stream to
+``tfa_prefill``.  There is no fallback: if the library is missing or the call
+fails, it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libtfa.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "tfa.h")
+
+TFA_OK = 0
+TFA_ERR_NULL = 1
+TFA_ERR_HEADS = 2
+TFA_ERR_SHORT_QUERY = 3
+TFA_ERR_SHAPE = 4
+TFA_ERR_HEAD_DIM = 5
+TFA_ERR_WINDOW = 6
+TFA_ERR_ALIGN = 7
+TFA_ERR_CUDA = 8
+TFA_ERR_TIMEOUT = 9
+TFA_ERR_SCALE = 10
+TFA_ERR_FLAGS = 11
+
+TFA_DEBUG_NO_TILE_SKIP = 1
+TFA_DEBUG_MASK_ALL = 2
+TFA_DEBUG_SYNC = 4
+
+MIN_QUERY_ROWS = 9
+BLOCK_Q = 128
+BLOCK_K = 128
+
+_lock = threading.Lock()
+_lib = None
+
+
+class TfaError(RuntimeError):
+    def __init__(self, code: int, where: str = "tfa_prefill"):
+        self.code = code
+        super().__init__(f"{where} failed with status {code}: {status_string(code)}")
+
+
+def lib():
+    """Load libtfa.so; raise if it has not been built (no fallback path exists)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m sliding_window_gqa_tfa_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, i32, u32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint, ctypes.c_float
+            common = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P, P]
+            L.tfa_prefill.argtypes = common
+            L.tfa_prefill.restype = i32
+            L.tfa_prefill_debug.argtypes = common + [u32]
+            L.tfa_prefill_debug.restype = i32
+            L.tfa_prefill_host.argtypes = common
+            L.tfa_prefill_host.restype = i32
+            L.tfa_check_status.argtypes = [P]
+            L.tfa_check_status.restype = i32
+            L.tfa_status_string.argtypes = [i32]
+            L.tfa_status_string.restype = ctypes.c_char_p
+            L.tfa_plan_qtile.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(i32),
+                                         ctypes.POINTER(i32), P, i32]
+            L.tfa_plan_qtile.restype = i32
+            _lib = L
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Names of the functions include/tfa.h declares."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|const char \*)\s*(tfa_\w+)\s*\(", text, re.M)))
+
+
+def status_string(code: int) -> str:
+    return lib().tfa_status_string(int(code)).decode()
+
+
+# ----------------------------------------------------------- raw entry points
+def tfa_prefill(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, stream) -> int:
+    return lib().tfa_prefill(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                             stream)
+
+
+def tfa_prefill_debug(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, stream,
+                      flags) -> int:
+    return lib().tfa_prefill_debug(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window,
+                                   key_mask, stream, flags)
+
+
+def tfa_prefill_host(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                     stream) -> int:
+    return lib().tfa_prefill_host(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window,
+                                  key_mask, stream)
+
+
+def tfa_check_status(stream) -> int:
+    return lib().tfa_check_status(stream)
+
+
+def tfa_plan_qtile(L, S, causal, window, has_key_mask, qtile):
+    """Returns (status, kt_lo, kt_hi, needs_mask list)."""
+    lo, hi = ctypes.c_int(0), ctypes.c_int(0)
+    buf = (ctypes.c_ubyte * (S // BLOCK_K + 2))()
+    rc = lib().tfa_plan_qtile(L, S, int(causal), window, int(has_key_mask), qtile,
+                              ctypes.byref(lo), ctypes.byref(hi),
+                              ctypes.cast(buf, ctypes.c_void_p), len(buf))
+    if rc:
+        return rc, None, None, None
+    return rc, lo.value, hi.value, [bool(buf[i]) for i in range(hi.value - lo.value + 1)]
+
+
+# ---------------------------------------------------------- torch wrapper
+def _stream_handle(stream):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(t, name, dtype, ndim):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=None, stream=None,
+            debug_flags=0):
+    """Attention output [B,Hq,L,D] bf16 for bf16 q [B,Hq,L,D], k/v [B,Hkv,S,D] on one GPU.
+
+    key_mask: optional fp32 [B,S] (1 keep / 0 drop).  Raises TfaError on a
+    nonzero status from the library."""
+    import torch
+
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k, "k", torch.bfloat16, 4)
+    _check(v, "v", torch.bfloat16, 4)
+    B, Hq, L, D = q.shape
+    Bk, Hkv, S, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k and v must have the same shape")
+    if Bk != B or Dk != D:
+        raise ValueError("q and k disagree on batch or head dimension")
+    if key_mask is not None:
+        _check(key_mask, "key_mask", torch.float32, 2)
+        if tuple(key_mask.shape) != (B, S):
+            raise ValueError("key_mask must be [B, S]")
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check(out, "out", torch.bfloat16, 4)
+        if tuple(out.shape) != tuple(q.shape):
+            raise ValueError("out must have q's shape")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    args = (ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()), B, Hq, Hkv, L, S, D,
+            float(scale), int(bool(causal)), int(window),
+            ctypes.c_void_p(key_mask.data_ptr()) if key_mask is not None else None,
+            _stream_handle(stream))
+    rc = tfa_prefill_debug(*args, debug_flags) if debug_flags else tfa_prefill(*args)
+    if rc != TFA_OK:
+        raise TfaError(rc)
+    return out
+
+
+def check_status(stream=None) -> None:
+    """Synchronize `stream` and raise TfaError if a kernel recorded a timed-out wait."""
+    rc = tfa_check_status(_stream_handle(stream))
+    if rc != TFA_OK:
+        raise TfaError(rc, "tfa_check_status")
+
+
+def prefill_host(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=None,
+                 stream=None):
+    """The same operation on CPU tensors (pinned or pageable) through tfa_prefill_host."""
+    import torch
+
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor")
+    B, Hq, L, D = q.shape
+    _, Hkv, S, _ = k.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    km = None
+    if key_mask is not None:
+        if key_mask.dtype != torch.float32 or key_mask.is_cuda or not key_mask.is_contiguous():
+            raise ValueError("key_mask must be a contiguous fp32 CPU tensor")
+        km = ctypes.c_void_p(key_mask.data_ptr())
+    rc = tfa_prefill_host(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                          ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                          B, Hq, Hkv, L, S, D, float(scale), int(bool(causal)), int(window), km,
+                          _stream_handle(stream))
+    if rc != TFA_OK:
+        raise TfaError(rc, "tfa_prefill_host")
+    return out

@@ -1,0 +1,280 @@
+// tfa.cu -- C-ABI boundary of the tiled GQA prefill attention library:
+// argument validation, TMA descriptor encoding, launch of the sm_100a kernel,
+// the device status word and the host-buffer entry point.
+//
+// The rejection rules follow tiny-llm "Week 2 Day 5: Tiled Dense Prefill
+// Attention", Task 1: BF16 inputs (by the ABI's contract), equal K/V shapes and
+// matching batch/head dimensions (one B, Hkv, S for both), Hq % Hkv == 0, and
+// the direct operator rejects queries shorter than nine rows.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "../../include/tfa.h"
+#include "tfa_kernel.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool init = false;
+    int sm_count = 0;
+    unsigned *status = nullptr;  // device status word (TFA_DEVICE_TIMEOUT bits)
+    bool smem_attr[2] = {false, false};
+    // staging buffers of tfa_prefill_host
+    void *h_buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
+    size_t h_cap[5] = {0, 0, 0, 0, 0};
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode_fn() {
+    if (g_encode) return TFA_OK;
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return TFA_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return TFA_OK;
+}
+
+// Per-device state, created on first use with that device current.  The
+// status word is cleared on `stream` so it is ordered before the first launch.
+int device_state(cudaStream_t stream, DeviceState **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TFA_ERR_CUDA;
+    DeviceState &st = g_dev[dev];
+    if (!st.init) {
+        if (cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return TFA_ERR_CUDA;
+        if (cudaMalloc(&st.status, 256) != cudaSuccess) return TFA_ERR_CUDA;
+        if (cudaMemsetAsync(st.status, 0, 256, stream) != cudaSuccess) return TFA_ERR_CUDA;
+        if (get_encode_fn() != TFA_OK) return TFA_ERR_CUDA;
+        st.init = true;
+    }
+    *out = &st;
+    return TFA_OK;
+}
+
+int validate(const void *q, const void *k, const void *v, const void *o, int B, int Hq, int Hkv,
+             int L, int S, int D, float scale, int causal, int window, const float *key_mask,
+             bool check_pointers) {
+    if (check_pointers && (!q || !k || !v || !o)) return TFA_ERR_NULL;
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TFA_ERR_HEADS;
+    if (L < TFA_MIN_QUERY_ROWS) return TFA_ERR_SHORT_QUERY;
+    if (B < 1 || S < L) return TFA_ERR_SHAPE;
+    // element counts and every index the kernel forms must stay in range
+    const long long qrows = static_cast<long long>(B) * Hq * L;
+    const long long krows = static_cast<long long>(B) * Hkv * S;
+    if (qrows > (1ll << 31) - 1 || krows > (1ll << 31) - 1 || S > (1 << 30)) return TFA_ERR_SHAPE;
+    const long long n_items = static_cast<long long>(B) * Hq * ((L + 2 * tfa::kBlockQ - 1) / (2 * tfa::kBlockQ));
+    if (n_items > (1ll << 30)) return TFA_ERR_SHAPE;
+    if (D != 64 && D != 128) return TFA_ERR_HEAD_DIM;
+    if (window > 0 && !causal) return TFA_ERR_WINDOW;
+    if (check_pointers) {
+        auto mis16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+        if (mis16(q) || mis16(k) || mis16(v) || mis16(o)) return TFA_ERR_ALIGN;
+        if (key_mask && (reinterpret_cast<uintptr_t>(key_mask) & 3u)) return TFA_ERR_ALIGN;
+    }
+    if (!std::isfinite(scale)) return TFA_ERR_SCALE;
+    return TFA_OK;
+}
+
+// 3-D view [planes][rows][D] of a contiguous bf16 tensor, boxes of 128 rows x
+// 64 columns (128 bytes) with 128-byte swizzle; rows past the end read as 0.
+int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(planes)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
+                             static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(D) * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(tfa::kBlockQ), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? TFA_OK : TFA_ERR_CUDA;
+}
+
+template <int D>
+int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o, int B, int Hq,
+           int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
+           cudaStream_t stream, unsigned flags) {
+    using C = tfa::Cfg<D>;
+    CUtensorMap mq, mk, mv;
+    if (encode_map(&mq, q, L, B * Hq, D) || encode_map(&mk, k, S, B * Hkv, D) ||
+        encode_map(&mv, v, S, B * Hkv, D))
+        return TFA_ERR_CUDA;
+    auto kern = tfa::tfa_prefill_kernel<D>;
+    const int which = D == 128 ? 1 : 0;
+    if (!st.smem_attr[which]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+            cudaSuccess)
+            return TFA_ERR_CUDA;
+        st.smem_attr[which] = true;
+    }
+    tfa::Params p;
+    p.o = static_cast<__nv_bfloat16 *>(o);
+    p.key_mask = key_mask;
+    p.status = st.status;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.L = L;
+    p.S = S;
+    p.G = Hq / Hkv;
+    p.n_qp = (L + 2 * tfa::kBlockQ - 1) / (2 * tfa::kBlockQ);
+    p.n_items = B * Hq * p.n_qp;
+    p.causal = causal ? 1 : 0;
+    p.window = (causal && window > 0) ? window : 0;
+    p.flags = flags;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int grid = p.n_items < st.sm_count ? p.n_items : st.sm_count;
+    kern<<<grid, tfa::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    return cudaGetLastError() == cudaSuccess ? TFA_OK : TFA_ERR_CUDA;
+}
+
+int prefill_impl(const void *q, const void *k, const void *v, void *o, int B, int Hq, int Hkv,
+                 int L, int S, int D, float scale, int causal, int window, const float *key_mask,
+                 cudaStream_t stream, unsigned flags) {
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
+    if (rc) return rc;
+    if (flags & ~(TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL | TFA_DEBUG_SYNC)) return TFA_ERR_FLAGS;
+    DeviceState *st = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mutex);
+        rc = device_state(stream, &st);
+    }
+    if (rc) return rc;
+    const unsigned kflags = flags & (TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL);
+    rc = (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                  key_mask, stream, kflags)
+                    : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                 key_mask, stream, kflags);
+    if (rc) return rc;
+    if (flags & TFA_DEBUG_SYNC) return tfa_check_status(reinterpret_cast<tfa_stream_t>(stream));
+    return TFA_OK;
+}
+
+int ensure_capacity(DeviceState &st, int i, size_t bytes) {
+    if (st.h_cap[i] >= bytes) return TFA_OK;
+    if (st.h_buf[i]) cudaFree(st.h_buf[i]);
+    st.h_buf[i] = nullptr;
+    st.h_cap[i] = 0;
+    if (cudaMalloc(&st.h_buf[i], bytes) != cudaSuccess) return TFA_ERR_CUDA;
+    st.h_cap[i] = bytes;
+    return TFA_OK;
+}
+
+}  // namespace
+
+extern "C" int tfa_prefill(const void *q, const void *k, const void *v, void *o, int B, int Hq,
+                           int Hkv, int L, int S, int D, float scale, int causal, int window,
+                           const float *key_mask, tfa_stream_t stream) {
+    return prefill_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                        reinterpret_cast<cudaStream_t>(stream), 0u);
+}
+
+extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o, int B,
+                                 int Hq, int Hkv, int L, int S, int D, float scale, int causal,
+                                 int window, const float *key_mask, tfa_stream_t stream,
+                                 unsigned flags) {
+    return prefill_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                        reinterpret_cast<cudaStream_t>(stream), flags);
+}
+
+extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, void *o, int B,
+                                int Hq, int Hkv, int L, int S, int D, float scale, int causal,
+                                int window, const float *key_mask, tfa_stream_t stream) {
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t qbytes = static_cast<size_t>(B) * Hq * L * D * 2;
+    const size_t kbytes = static_cast<size_t>(B) * Hkv * S * D * 2;
+    const size_t mbytes = key_mask ? static_cast<size_t>(B) * S * sizeof(float) : 0;
+    DeviceState *st = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st))) return rc;
+    if ((rc = ensure_capacity(*st, 0, qbytes)) || (rc = ensure_capacity(*st, 1, kbytes)) ||
+        (rc = ensure_capacity(*st, 2, kbytes)) || (rc = ensure_capacity(*st, 3, qbytes)) ||
+        (mbytes && (rc = ensure_capacity(*st, 4, mbytes))))
+        return rc;
+    if (cudaMemcpyAsync(st->h_buf[0], q, qbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(st->h_buf[1], k, kbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(st->h_buf[2], v, kbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        (mbytes && cudaMemcpyAsync(st->h_buf[4], key_mask, mbytes, cudaMemcpyHostToDevice, s) !=
+                       cudaSuccess))
+        return TFA_ERR_CUDA;
+    const float *dmask = mbytes ? static_cast<const float *>(st->h_buf[4]) : nullptr;
+    rc = (D == 128) ? launch<128>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
+                                  Hkv, L, S, scale, causal, window, dmask, s, 0u)
+                    : launch<64>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
+                                 Hkv, L, S, scale, causal, window, dmask, s, 0u);
+    if (rc) return rc;
+    if (cudaMemcpyAsync(o, st->h_buf[3], qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return TFA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return TFA_ERR_CUDA;
+    return TFA_OK;
+}
+
+extern "C" int tfa_check_status(tfa_stream_t stream) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TFA_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TFA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    DeviceState &st = g_dev[dev];
+    if (!st.init) return TFA_OK;
+    unsigned word = 0;
+    if (cudaMemcpy(&word, st.status, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return TFA_ERR_CUDA;
+    if (word == 0) return TFA_OK;
+    if (cudaMemset(st.status, 0, sizeof word) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return TFA_ERR_CUDA;
+    return TFA_ERR_TIMEOUT;
+}
+
+extern "C" const char *tfa_status_string(int status) {
+    switch (status) {
+        case TFA_OK: return "ok";
+        case TFA_ERR_NULL: return "a tensor pointer is NULL";
+        case TFA_ERR_HEADS: return "query heads must be a positive multiple of KV heads";
+        case TFA_ERR_SHORT_QUERY: return "query shorter than the tiled operator's minimum (9 rows)";
+        case TFA_ERR_SHAPE: return "invalid shape (B < 1, S < L, or sizes out of range)";
+        case TFA_ERR_HEAD_DIM: return "head dimension must be 64 or 128";
+        case TFA_ERR_WINDOW: return "a sliding window requires causal attention";
+        case TFA_ERR_ALIGN: return "tensor pointers must be 16-byte aligned (key mask 4-byte)";
+        case TFA_ERR_CUDA: return "a CUDA call failed";
+        case TFA_ERR_TIMEOUT: return "a kernel wait timed out; the output is invalid";
+        case TFA_ERR_SCALE: return "scale must be finite";
+        case TFA_ERR_FLAGS: return "unknown debug flags";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_mask, int qtile,
+                              int *kt_lo, int *kt_hi, unsigned char *needs_mask, int needs_mask_len) {
+    int rc = validate(nullptr, nullptr, nullptr, nullptr, 1, 1, 1, L, S, 128, 1.0f, causal, window,
+                      nullptr, false);
+    if (rc) return rc;
+    if (!kt_lo || !kt_hi) return TFA_ERR_NULL;
+    const int q0 = qtile * tfa::kBlockQ;
+    if (qtile < 0 || q0 >= L) return TFA_ERR_SHAPE;
+    const tfa::KeyRange r = tfa::qtile_key_range(L, S, causal, causal ? window : 0, q0, 0u);
+    *kt_lo = r.lo;
+    *kt_hi = r.hi;
+    if (needs_mask) {
+        if (needs_mask_len < r.hi - r.lo + 1) return TFA_ERR_SHAPE;
+        for (int j = r.lo; j <= r.hi; ++j)
+            needs_mask[j - r.lo] = tfa::key_tile_needs_mask(L, S, causal, causal ? window : 0,
+                                                            has_key_mask, q0, j, 0u) ? 1 : 0;
+    }
+    return TFA_OK;
+}

@@ -1,0 +1,491 @@
+// tfa_kernel.cuh -- persistent, warp-specialised sm_100a kernel for tiled GQA
+// prefill attention (online softmax; tcgen05 tensor cores with TMEM
+// accumulators; TMA into 128-byte-swizzled shared memory).
+//
+// What it computes is tiny-llm "Week 2 Day 5: Tiled Dense Prefill Attention"
+// (Task 1: per query row an FP32 running max m, sum l and accumulator a merged
+// tile by tile as m' = max(m, m_b), l' = e^(m-m') l + e^(m_b-m') l_b,
+// a' = e^(m-m') a + e^(m_b-m') a_b, out = a'/l'; Task 2: causality aligned to
+// the end of the cached prefix, fully masked rows finite zeros) with the
+// sliding window and key mask of brotensor's flash_attention.h.
+//
+// Work unit ("item"): batch b, query head h and a pair of consecutive 128-row
+// query tiles t = 0, 1 (rows [256 qp, 256 qp + 256)).  The two tiles share
+// every K/V tile they both reach, and ping-pong on the tensor core: while
+// tile 0's softmax runs, the tensor core computes tile 1's products and vice
+// versa.  Items are handed out statically to a persistent grid of one CTA per
+// SM, longest first (causal items with the most key tiles first), with the
+// query heads that share a KV head next to each other so their K/V reads hit L2.
+//
+// Roles (320 threads):
+//   warps 0-3   softmax + epilogue for query tile 0 (thread = one query row)
+//   warps 4-7   softmax + epilogue for query tile 1
+//   warp 8      TMA producer (lane 0): Q tiles, then K_j, V_j into a ring of slots
+//   warp 9      tensor-core issuer (lane 0)
+// Tensor memory (512 columns, fp32): S_0 [0,128), S_1 [128,256), O_0 and O_1 at
+// 256 and 256 + D.  P (bf16, two per column) overwrites S_t's columns [64,128)
+// and feeds the P.V product straight from tensor memory.
+//
+// Per key tile j the issuer runs, for t = 0, 1:  O_t += P_t(j) V_j (after the
+// softmax of tile t published P_t(j)), then S_t = Q_t K_{j+1}^T.  tcgen05
+// operations from one thread execute in order, so S_t(j+1) never overwrites
+// P_t(j) before P_t(j) V_j has read it, and the commit that signals S_t(j+1)
+// also covers O_t's update -- the softmax may rescale O_t right after it.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "tfa_plan.h"
+#include "tfa_ptx.cuh"
+
+namespace tfa {
+
+constexpr int kThreads = 320;
+// Lazy rescale: keep the stale row maximum until the true one exceeds it by
+// more than 2^8 in the exp2 domain (P values then stay <= 256).
+constexpr float kRescaleThresholdLog2 = 8.0f;
+
+template <int D>
+struct Cfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kTileBytes = 128 * D * 2;        // 128 rows x D bf16 (Q, K or V tile)
+    static constexpr int kColBlocks = D / 64;             // 64-element (128-byte) column blocks
+    static constexpr int kColBlockBytes = 128 * 128;      // one 128-row x 128-byte block
+    static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
+    static constexpr int kNumBars = 10 + 2 * kSlots + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kTmemS = 0;                 // S_t at kTmemS + 128 t
+    static constexpr uint32_t kTmemO = 256;               // O_t at kTmemO + D t
+    static constexpr uint32_t kTmemP = 64;                // P_t at S_t + 64
+};
+
+struct Params {
+    __nv_bfloat16 *o;
+    const float *key_mask;
+    unsigned *status;
+    int B, Hq, Hkv, L, S, G;
+    int n_qp, n_items;
+    int causal, window;
+    unsigned flags;
+    float scale_log2;  // softmax scale * log2(e)
+};
+
+struct ItemPlan {
+    int b, h, g;
+    int q0[2];
+    bool present[2];
+    int lo[2], hi[2];
+    int jl, jh;
+};
+
+__device__ __forceinline__ ItemPlan plan_item(const Params &p, int item) {
+    ItemPlan ip;
+    const int bh = p.B * p.Hq;
+    const int r = item / bh;
+    const int rem = item - r * bh;
+    ip.b = rem / p.Hq;
+    ip.h = rem - ip.b * p.Hq;
+    ip.g = ip.h / p.G;
+    const int qp = p.causal ? (p.n_qp - 1 - r) : r;
+    ip.jl = 0x7fffffff;
+    ip.jh = -1;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+        ip.q0[t] = qp * 2 * kBlockQ + t * kBlockQ;
+        ip.present[t] = ip.q0[t] < p.L;
+        const KeyRange kr = qtile_key_range(p.L, p.S, p.causal, p.window, ip.q0[t], p.flags);
+        ip.lo[t] = kr.lo;
+        ip.hi[t] = ip.present[t] ? kr.hi : -1;
+        if (ip.present[t]) {
+            ip.jl = imin(ip.jl, kr.lo);
+            ip.jh = imax(ip.jh, kr.hi);
+        }
+    }
+    return ip;
+}
+
+struct Bars {
+    uint32_t base;
+    int slots;
+    __device__ __forceinline__ uint32_t q_full(int t) const { return base + 8 * (0 + t); }
+    __device__ __forceinline__ uint32_t q_empty(int t) const { return base + 8 * (2 + t); }
+    __device__ __forceinline__ uint32_t s_full(int t) const { return base + 8 * (4 + t); }
+    __device__ __forceinline__ uint32_t p_full(int t) const { return base + 8 * (6 + t); }
+    __device__ __forceinline__ uint32_t o_full(int t) const { return base + 8 * (8 + t); }
+    __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8 * (10 + s); }
+    __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8 * (10 + slots + s); }
+    __device__ __forceinline__ uint32_t done() const { return base + 8 * (10 + 2 * slots); }
+};
+
+// ------------------------------------------------------------------ producer
+template <int D>
+__device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                          const CUtensorMap *tm_v, uint32_t sbase, const Bars &bar,
+                          volatile int *abort_flag) {
+    using C = Cfg<D>;
+    uint32_t kv_prod = 0;
+    uint32_t q_use[2] = {0, 0};
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+        const ItemPlan ip = plan_item(p, item);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (!ip.present[t]) continue;
+            if (q_use[t] > 0 && !mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status))
+                goto out;
+            mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
+            for (int cb = 0; cb < C::kColBlocks; ++cb)
+                tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes, tm_q,
+                            bar.q_full(t), cb * 64, ip.q0[t], ip.b * p.Hq + ip.h);
+            ++q_use[t];
+        }
+        for (int j = ip.jl; j <= ip.jh; ++j) {
+            for (int which = 0; which < 2; ++which) {  // K_j then V_j
+                const uint32_t s = kv_prod % C::kSlots;
+                const uint32_t round = kv_prod / C::kSlots;
+                if (round > 0 && !mbar_wait(bar.kv_empty(s), (round - 1) & 1, abort_flag, p.status))
+                    goto out;
+                mbar_arrive_expect_tx(bar.kv_full(s), C::kTileBytes);
+                for (int cb = 0; cb < C::kColBlocks; ++cb)
+                    tma_load_3d(sbase + C::kKVOff + s * C::kTileBytes + cb * C::kColBlockBytes,
+                                which ? tm_v : tm_k, bar.kv_full(s), cb * 64, j * kBlockK,
+                                ip.b * p.Hkv + ip.g);
+                ++kv_prod;
+            }
+        }
+    }
+out:
+    // Every copy this thread started must land before the CTA may exit.
+    for (uint32_t s = 0; s < (uint32_t)C::kSlots; ++s) {
+        if (kv_prod > s) {
+            const uint32_t armed = (kv_prod - s - 1) / C::kSlots + 1;
+            mbar_drain(bar.kv_full(s), (armed - 1) & 1);
+        }
+    }
+    for (int t = 0; t < 2; ++t)
+        if (q_use[t] > 0) mbar_drain(bar.q_full(t), (q_use[t] - 1) & 1);
+}
+
+// ------------------------------------------------------------ tensor cores
+template <int D>
+__device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const Bars &bar,
+                         volatile int *abort_flag) {
+    using C = Cfg<D>;
+    constexpr uint32_t kIdescQK = idesc_bf16_f32(128, kBlockK, 0);  // S = Q K^T, both K-major
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);        // O += P V, V MN-major
+    const uint32_t q_smem = sbase + C::kQOff;
+    const uint32_t kv_smem = sbase + C::kKVOff;
+
+    // S_t = Q_t K^T: A = Q tile, B = K tile, both [128 rows][D] K-major with
+    // 128-byte swizzle; a K-step of 16 elements advances 32 bytes inside a
+    // 128-byte row and moves to the next column block every 4 steps.
+    auto issue_qk = [&](int t, uint32_t slot) {
+        const uint32_t qa = q_smem + t * C::kTileBytes;
+        const uint32_t ka = kv_smem + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::kColBlockBytes + (kk & 3) * 32;
+            umma_ss(tmem + C::kTmemS + t * 128, smem_desc_sw128(qa + off, 16, 1024),
+                    smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+    };
+    // O_t += P_t V: A = P_t in tensor memory (8 columns per 16 keys), B = V tile
+    // read MN-major (D contiguous): 8 key rows per 1 KB swizzle atom (SBO), the
+    // next 64 head-dim columns one column block further (LBO).
+    auto issue_pv = [&](int t, uint32_t slot, bool accumulate) {
+        const uint32_t va = kv_smem + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBlockK / 16; ++kk) {
+            umma_ts(tmem + C::kTmemO + t * D, tmem + C::kTmemS + t * 128 + C::kTmemP + kk * 8,
+                    smem_desc_sw128(va + kk * 16 * 128, C::kColBlockBytes, 1024), kIdescPV,
+                    (accumulate || kk > 0) ? 1u : 0u);
+        }
+    };
+
+    uint32_t kv_cons = 0;
+    uint32_t q_use[2] = {0, 0};
+    uint32_t p_cnt[2] = {0, 0};
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+        const ItemPlan ip = plan_item(p, item);
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            if (!ip.present[t]) continue;
+            if (!mbar_wait(bar.q_full(t), q_use[t] & 1, abort_flag, p.status)) goto out;
+            ++q_use[t];
+        }
+        {
+            const uint32_t s = kv_cons % C::kSlots;
+            if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+            ++kv_cons;
+            tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (ip.present[t] && ip.lo[t] <= ip.jl) {
+                    issue_qk(t, s);
+                    umma_commit(bar.s_full(t));
+                    if (ip.hi[t] == ip.jl) umma_commit(bar.q_empty(t));
+                }
+            }
+            umma_commit(bar.kv_empty(s));
+        }
+        bool acc[2] = {false, false};
+        for (int j = ip.jl; j <= ip.jh; ++j) {
+            const uint32_t sv = kv_cons % C::kSlots;
+            if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+            ++kv_cons;
+            const bool next = j < ip.jh;
+            uint32_t sk = 0;
+            if (next) {
+                sk = kv_cons % C::kSlots;
+                if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status))
+                    goto out;
+                ++kv_cons;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (!ip.present[t]) continue;
+                if (ip.lo[t] <= j && j <= ip.hi[t]) {
+                    if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                    ++p_cnt[t];
+                    tc_fence_after();
+                    issue_pv(t, sv, acc[t]);
+                    acc[t] = true;
+                    if (j == ip.hi[t]) umma_commit(bar.o_full(t));
+                }
+                if (next && ip.lo[t] <= j + 1 && j + 1 <= ip.hi[t]) {
+                    issue_qk(t, sk);
+                    umma_commit(bar.s_full(t));
+                    if (j + 1 == ip.hi[t]) umma_commit(bar.q_empty(t));
+                }
+            }
+            umma_commit(bar.kv_empty(sv));
+            if (next) umma_commit(bar.kv_empty(sk));
+        }
+    }
+out:
+    // Nothing may leave tensor memory in flight when the CTA frees it.
+    umma_commit(bar.done());
+    mbar_drain(bar.done(), 0);
+}
+
+// ---------------------------------------------------- softmax and epilogue
+template <int D, int t>
+__device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
+                             volatile int *abort_flag) {
+    using C = Cfg<D>;
+    const int r = threadIdx.x - t * 128;  // row inside the query tile
+    const uint32_t lane_base = (static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u) << 16;
+    const uint32_t tS = tmem + C::kTmemS + t * 128 + lane_base;
+    const uint32_t tP = tS + C::kTmemP;
+    const uint32_t tO = tmem + C::kTmemO + t * D + lane_base;
+    const float c = p.scale_log2;
+    const bool has_km = p.key_mask != nullptr;
+    const int lane = threadIdx.x & 31;
+    uint32_t s_cnt = 0, o_cnt = 0;
+
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+        const ItemPlan ip = plan_item(p, item);
+        if (!ip.present[t]) continue;
+        const int row = ip.q0[t] + r;
+        const int pos = (p.S - p.L) + row;  // absolute position of this query row
+        const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
+        const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
+        const float *km_row = has_km ? p.key_mask + static_cast<size_t>(ip.b) * p.S : nullptr;
+        float m_ref = -CUDART_INF_F;  // row maximum the exponentials are taken against
+        float l = 0.f;
+        bool first = true;
+
+        for (int j = ip.lo[t]; j <= ip.hi[t]; ++j) {
+            // all lanes leave together: the tcgen05 loads below are warp-collective
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(t), s_cnt & 1, abort_flag, p.status)))
+                return;
+            ++s_cnt;
+            tc_fence_after();
+            uint32_t s[128];
+            tmem_ld128(tS, s);
+
+            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, has_km, ip.q0[t], j, p.flags)) {
+                const int k0 = j * kBlockK;
+                const int lo_c = lo_abs - k0;
+                const int hi_c = hi_abs - k0;
+                uint32_t kmw[4] = {~0u, ~0u, ~0u, ~0u};
+                if (has_km) {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const int col = k0 + 32 * w + lane;
+                        const float mv = col < p.S ? __ldg(km_row + col) : 0.f;
+                        kmw[w] = __ballot_sync(0xffffffffu, mv > 0.5f);
+                    }
+                }
+#pragma unroll
+                for (int cidx = 0; cidx < 128; ++cidx) {
+                    const bool keep = cidx >= lo_c && cidx <= hi_c && ((kmw[cidx >> 5] >> (cidx & 31)) & 1u);
+                    if (!keep) s[cidx] = 0xff800000u;  // -inf
+                }
+            }
+
+            float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
+            float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+#pragma unroll
+            for (int i = 4; i < 128; i += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(s[i]));
+                mx1 = fmaxf(mx1, __uint_as_float(s[i + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(s[i + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(s[i + 3]));
+            }
+            const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+
+            // Decide the lazy rescale first; O_t itself is rescaled after P is
+            // stored, once the S registers are dead.
+            float alpha = 1.f;
+            bool rescale = false;
+            if (first) {
+                m_ref = m_new;  // the first P.V overwrites O, nothing to rescale
+                first = false;
+            } else {
+                // (m_new - m_ref) is NaN when both are -inf (row still empty: keep),
+                // +inf when the row sees its first key (rescale by 0).
+                const bool need = (m_new - m_ref) * c > kRescaleThresholdLog2;
+                rescale = __any_sync(0xffffffffu, need);
+                if (need) {
+                    alpha = (m_ref == -CUDART_INF_F) ? 0.f : ex2((m_ref - m_new) * c);
+                    m_ref = m_new;
+                }
+            }
+
+            const float mc = (m_ref == -CUDART_INF_F) ? 0.f : m_ref * c;
+            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int i = 0; i < 64; i += 2) {
+                const float a0 = ex2(fmaf(__uint_as_float(s[2 * i]), c, -mc));
+                const float a1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), c, -mc));
+                const float a2 = ex2(fmaf(__uint_as_float(s[2 * i + 2]), c, -mc));
+                const float a3 = ex2(fmaf(__uint_as_float(s[2 * i + 3]), c, -mc));
+                l0 += a0;
+                l1 += a1;
+                l2 += a2;
+                l3 += a3;
+                pk[i] = pack_bf16(a0, a1);
+                pk[i + 1] = pack_bf16(a2, a3);
+            }
+            l = l * alpha + ((l0 + l1) + (l2 + l3));
+            tmem_st32(tP, pk);
+            tmem_st32(tP + 32, pk + 32);
+            if (rescale) {
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + cc * 32, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + cc * 32, o);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar.p_full(t));
+        }
+
+        // Epilogue: final FP32 normalisation, then BF16 (a row with no allowed
+        // key has l == 0 and is written as zeros).
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(t), o_cnt & 1, abort_flag, p.status)))
+            return;
+        ++o_cnt;
+        tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+        __nv_bfloat16 *orow =
+            p.o + (static_cast<size_t>(ip.b * p.Hq + ip.h) * p.L + row) * static_cast<size_t>(D);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            if (row < p.L) {
+                uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int D>
+__global__ void __maxnreg__(200)
+    tfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const Params p) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t sbase = (raw + 1023u) & ~1023u;  // 128-byte swizzle wants 1 KB alignment
+    uint8_t *gbase = smem_raw + (sbase - raw);
+    Bars bar{sbase + C::kBarOff, C::kSlots};
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(gbase + C::kMiscOff);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(gbase + C::kMiscOff + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar.q_full(t), 1);
+            mbar_init(bar.q_empty(t), 1);
+            mbar_init(bar.s_full(t), 1);
+            mbar_init(bar.p_full(t), 128);
+            mbar_init(bar.o_full(t), 1);
+        }
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(bar.kv_full(s), 1);
+            mbar_init(bar.kv_empty(s), 1);
+        }
+        mbar_init(bar.done(), 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp < 8) {
+        if (warp < 4)
+            softmax_role<D, 0>(p, tmem, bar, abort_flag);
+        else
+            softmax_role<D, 1>(p, tmem, bar, abort_flag);
+    } else if (warp == 8) {
+        if (lane == 0) load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, bar, abort_flag);
+    } else if (warp == 9) {
+        if (lane == 0) mma_role<D>(p, sbase, tmem, bar, abort_flag);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace tfa

@@ -1,0 +1,154 @@
+"""CPU-side checks of the CUDA library: it loads, exports every declared entry
+point, rejects bad arguments before touching the GPU, and its work
+enumeration (the tile scheduler's host view) is exact against the oracle's
+visibility rule.  No compute call runs here."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sliding_window_gqa_tfa_b200 import binding as tb
+from sliding_window_gqa_tfa_b200.flops import allowed_pairs
+from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_inputs, shaped
+
+
+def test_library_exports_every_declared_symbol():
+    names = tb.declared_symbols()
+    assert {"tfa_prefill", "tfa_prefill_debug", "tfa_prefill_host", "tfa_check_status",
+            "tfa_status_string", "tfa_plan_qtile"} <= set(names)
+    lib = tb.lib()
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for code in range(12):
+        s = tb.status_string(code)
+        assert s and s != "unknown status"
+    assert tb.status_string(99) == "unknown status"
+
+
+# pointers that are never dereferenced: validation fails before any CUDA call
+A16 = ctypes.c_void_p(0x10000)
+MIS = ctypes.c_void_p(0x10008)
+
+
+def _call(**over):
+    a = dict(q=A16, k=A16, v=A16, o=A16, B=1, Hq=8, Hkv=2, L=33, S=47, D=128, scale=0.088,
+             causal=1, window=0, key_mask=None, stream=None)
+    a.update(over)
+    return tb.tfa_prefill(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(q=None), tb.TFA_ERR_NULL),
+    (dict(o=None), tb.TFA_ERR_NULL),
+    (dict(Hq=7, Hkv=2), tb.TFA_ERR_HEADS),
+    (dict(Hkv=0), tb.TFA_ERR_HEADS),
+    (dict(L=8, S=47), tb.TFA_ERR_SHORT_QUERY),
+    (dict(L=1, S=1), tb.TFA_ERR_SHORT_QUERY),
+    (dict(B=0), tb.TFA_ERR_SHAPE),
+    (dict(L=33, S=32), tb.TFA_ERR_SHAPE),
+    (dict(D=96), tb.TFA_ERR_HEAD_DIM),
+    (dict(D=256), tb.TFA_ERR_HEAD_DIM),
+    (dict(causal=0, window=16), tb.TFA_ERR_WINDOW),
+    (dict(q=MIS), tb.TFA_ERR_ALIGN),
+    (dict(v=MIS), tb.TFA_ERR_ALIGN),
+    (dict(key_mask=ctypes.c_void_p(0x10002)), tb.TFA_ERR_ALIGN),
+    (dict(scale=float("nan")), tb.TFA_ERR_SCALE),
+    (dict(scale=float("inf")), tb.TFA_ERR_SCALE),
+])
+def test_rejections_happen_before_launch(over, code):
+    assert _call(**over) == code
+
+
+def test_debug_rejects_unknown_flags_before_launch():
+    assert tb.tfa_prefill_debug(A16, A16, A16, A16, 1, 8, 2, 33, 47, 128, 0.1, 1, 0, None, None,
+                                64) == tb.TFA_ERR_FLAGS
+
+
+def test_host_entry_validates_first():
+    assert tb.tfa_prefill_host(A16, A16, A16, A16, 1, 6, 4, 33, 47, 128, 0.1, 1, 0, None,
+                               None) == tb.TFA_ERR_HEADS
+
+
+def _plan_cases():
+    cases = []
+    for name, w in WORKLOADS.items():
+        if w.L * w.S <= 2048 * 8192:
+            cases.append((name, w.L, w.S, w.causal, w.window, w.key_mask_keep is not None))
+    cases += [("ragged", 300, 301, True, 0, False), ("tiny", 9, 9, True, 0, False),
+              ("win1", 130, 700, True, 1, False), ("win129", 257, 1000, True, 129, False),
+              ("bidir_ragged", 200, 333, False, 0, False), ("wide", 200, 333, True, 5000, False),
+              ("w127", 383, 1111, True, 127, False)]
+    return cases
+
+
+@pytest.mark.parametrize("case", _plan_cases(), ids=lambda c: c[0])
+def test_tile_enumeration_is_exact(case):
+    """Every allowed (row, key) pair lies in a visited key tile; the first and
+    last visited tiles each hold an allowed pair (nothing reachable is skipped,
+    nothing skipped is reachable); tiles marked interior need no mask for any
+    valid row."""
+    _, L, S, causal, window, has_km = case
+    P = S - L
+    nqt = (L + 127) // 128
+    for qt in range(nqt):
+        rc, lo, hi, needs = tb.tfa_plan_qtile(L, S, causal, window, has_km, qt)
+        assert rc == 0
+        r0, r1 = qt * 128, min(qt * 128 + 128, L)
+        rows = np.arange(r0, r1)[:, None]
+        keys = np.arange(S)[None, :]
+        pos = P + rows
+        allowed = np.ones((r1 - r0, S), dtype=bool)
+        if causal:
+            allowed &= keys <= pos
+            if window > 0:
+                allowed &= keys > pos - window
+        tiles = np.nonzero(allowed.any(0))[0] // 128
+        assert tiles.min() == lo and tiles.max() == hi
+        for j in range(lo, hi + 1):
+            blk = allowed[:, j * 128:min(j * 128 + 128, S)]
+            full = blk.shape[1] == 128 and blk.all()
+            if not needs[j - lo]:
+                assert full, (qt, j)
+            if has_km:
+                assert needs[j - lo]
+    # the same rule, counted by the oracle's brute force, for small cases
+    if L * S <= 400 * 1200:
+        assert allowed_pairs(1, 1, L, S, causal=causal, window=window) == \
+            oracle.count_pairs(1, 1, L, S, causal=causal, window=window)
+
+
+def test_visibility_rule_matches_oracle_on_small_shapes():
+    for L, S, causal, window in [(9, 9, True, 0), (10, 40, True, 3), (12, 30, False, 0),
+                                 (33, 47, True, 0), (20, 25, True, 1)]:
+        vis = oracle.visibility(L, S, causal=causal, window=window)
+        P = S - L
+        rows = np.arange(L)[:, None] + P
+        keys = np.arange(S)[None, :]
+        mine = np.ones((L, S), dtype=bool)
+        if causal:
+            mine &= keys <= rows
+            if window > 0:
+                mine &= keys > rows - window
+        assert np.array_equal(vis, mine)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_flop_count_matches_oracle_count(name):
+    w = WORKLOADS[name]
+    km = None
+    if w.key_mask_keep is not None:
+        km = make_inputs(w.with_(Hq=1, Hkv=1, D=8), seed=0)[3]
+    assert allowed_pairs(w.B, w.Hq, w.L, w.S, causal=w.causal, window=w.window, key_mask=km) == \
+        oracle.count_pairs(w.B, w.Hq, w.L, w.S, causal=w.causal, window=w.window, key_mask=km)
+
+
+def test_flop_count_small_key_mask_cases():
+    for (B, L, S, causal, window) in [(2, 10, 30, True, 0), (3, 9, 9, True, 4), (2, 12, 20, False, 0)]:
+        km = (torch.rand(B, S, generator=torch.Generator().manual_seed(1)) > 0.3).float()
+        assert allowed_pairs(B, 3, L, S, causal=causal, window=window, key_mask=km) == \
+            oracle.count_pairs(B, 3, L, S, causal=causal, window=window, key_mask=km)
