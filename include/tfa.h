@@ -115,6 +115,11 @@ int tfa_prefill_host(const void *q, const void *k, const void *v, void *o,
  * since the last check recorded a wait that gave up, or TFA_ERR_CUDA. */
 int tfa_check_status(tfa_stream_t stream);
 
+/* tfa_last_error -- for the calling host thread, a description of the last CUDA
+ * runtime/driver call that failed inside the library (the call and its error
+ * string), or "" if none has.  Never NULL; valid until the next library call. */
+const char *tfa_last_error(void);
+
 /* tfa_status_string -- static description of a status code (never NULL). */
 const char *tfa_status_string(int status);
 

@@ -47,7 +47,8 @@ _lib = None
 class TfaError(RuntimeError):
     def __init__(self, code: int, where: str = "tfa_prefill"):
         self.code = code
-        super().__init__(f"{where} failed with status {code}: {status_string(code)}")
+        detail = f" [{last_error()}]" if code == TFA_ERR_CUDA else ""
+        super().__init__(f"{where} failed with status {code}: {status_string(code)}{detail}")
 
 
 def lib():
@@ -69,6 +70,8 @@ def lib():
             L.tfa_prefill_host.restype = i32
             L.tfa_check_status.argtypes = [P]
             L.tfa_check_status.restype = i32
+            L.tfa_last_error.argtypes = []
+            L.tfa_last_error.restype = ctypes.c_char_p
             L.tfa_status_string.argtypes = [i32]
             L.tfa_status_string.restype = ctypes.c_char_p
             L.tfa_plan_qtile.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(i32),
@@ -82,6 +85,10 @@ def declared_symbols() -> list[str]:
     """Names of the functions include/tfa.h declares."""
     text = open(HEADER).read()
     return sorted(set(re.findall(r"^\s*(?:int|const char \*)\s*(tfa_\w+)\s*\(", text, re.M)))
+
+
+def last_error() -> str:
+    return lib().tfa_last_error().decode()
 
 
 def status_string(code: int) -> str:

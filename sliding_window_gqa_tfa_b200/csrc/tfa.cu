@@ -8,6 +8,7 @@
 // the direct operator rejects queries shorter than nine rows.
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 
@@ -35,14 +36,27 @@ struct DeviceState {
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+thread_local char g_last_error[256] = "";
+
+// Record which CUDA call failed (readable through tfa_last_error) and map it to TFA_ERR_CUDA.
+int cuda_fail(const char *what, cudaError_t e) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s (%d)", what, cudaGetErrorString(e),
+             static_cast<int>(e));
+    return TFA_ERR_CUDA;
+}
+int drv_fail(const char *what, int code) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: CUresult %d", what, code);
+    return TFA_ERR_CUDA;
+}
 
 int get_encode_fn() {
     if (g_encode) return TFA_OK;
     void *fn = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || fn == nullptr)
-        return TFA_ERR_CUDA;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDriverEntryPoint", e);
+    if (q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return drv_fail("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled) query", static_cast<int>(q));
     g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     return TFA_OK;
 }
@@ -51,14 +65,17 @@ int get_encode_fn() {
 // status word is cleared on `stream` so it is ordered before the first launch.
 int device_state(cudaStream_t stream, DeviceState **out) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TFA_ERR_CUDA;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return drv_fail("device index out of range", dev);
     DeviceState &st = g_dev[dev];
     if (!st.init) {
-        if (cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return TFA_ERR_CUDA;
-        if (cudaMalloc(&st.status, 256) != cudaSuccess) return TFA_ERR_CUDA;
-        if (cudaMemsetAsync(st.status, 0, 256, stream) != cudaSuccess) return TFA_ERR_CUDA;
-        if (get_encode_fn() != TFA_OK) return TFA_ERR_CUDA;
+        if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail("cudaDeviceGetAttribute", e);
+        if ((e = cudaMalloc(&st.status, 256)) != cudaSuccess) return cuda_fail("cudaMalloc(status)", e);
+        if ((e = cudaMemsetAsync(st.status, 0, 256, stream)) != cudaSuccess)
+            return cuda_fail("cudaMemsetAsync(status)", e);
+        if (int rc = get_encode_fn()) return rc;
         st.init = true;
     }
     *out = &st;
@@ -101,7 +118,7 @@ int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D) {
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? TFA_OK : TFA_ERR_CUDA;
+    return r == CUDA_SUCCESS ? TFA_OK : drv_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
 }
 
 template <int D>
@@ -116,9 +133,21 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     auto kern = tfa::tfa_prefill_kernel<D>;
     const int which = D == 128 ? 1 : 0;
     if (!st.smem_attr[which]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
-            cudaSuccess)
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess)
+            return cuda_fail("cudaFuncGetAttributes", e);
+        // The setmaxnreg split inside the kernel is sized for exactly kRegsLaunch
+        // registers per thread at launch; any other count could leave a warpgroup
+        // waiting for registers that do not exist, so refuse to launch.
+        if (fa.maxThreadsPerBlock < tfa::kThreads || fa.numRegs != tfa::kRegsLaunch) {
+            snprintf(g_last_error, sizeof g_last_error,
+                     "kernel uses %d registers/thread (%d expected), at most %d threads fit, %d needed",
+                     fa.numRegs, tfa::kRegsLaunch, fa.maxThreadsPerBlock, tfa::kThreads);
             return TFA_ERR_CUDA;
+        }
         st.smem_attr[which] = true;
     }
     tfa::Params p;
@@ -139,7 +168,8 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.scale_log2 = scale * 1.4426950408889634f;
     const int grid = p.n_items < st.sm_count ? p.n_items : st.sm_count;
     kern<<<grid, tfa::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
-    return cudaGetLastError() == cudaSuccess ? TFA_OK : TFA_ERR_CUDA;
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TFA_OK : cuda_fail("kernel launch", e);
 }
 
 int prefill_impl(const void *q, const void *k, const void *v, void *o, int B, int Hq, int Hkv,
@@ -240,6 +270,8 @@ extern "C" int tfa_check_status(tfa_stream_t stream) {
         return TFA_ERR_CUDA;
     return TFA_ERR_TIMEOUT;
 }
+
+extern "C" const char *tfa_last_error(void) { return g_last_error; }
 
 extern "C" const char *tfa_status_string(int status) {
     switch (status) {

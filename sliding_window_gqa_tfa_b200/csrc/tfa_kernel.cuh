@@ -17,11 +17,12 @@
 // SM, longest first (causal items with the most key tiles first), with the
 // query heads that share a KV head next to each other so their K/V reads hit L2.
 //
-// Roles (320 threads):
+// Roles (384 threads, three warpgroups):
 //   warps 0-3   softmax + epilogue for query tile 0 (thread = one query row)
 //   warps 4-7   softmax + epilogue for query tile 1
 //   warp 8      TMA producer (lane 0): Q tiles, then K_j, V_j into a ring of slots
 //   warp 9      tensor-core issuer (lane 0)
+//   warps 10-11 idle (their registers go to the softmax warpgroups)
 // Tensor memory (512 columns, fp32): S_0 [0,128), S_1 [128,256), O_0 and O_1 at
 // 256 and 256 + D.  P (bf16, two per column) overwrites S_t's columns [64,128)
 // and feeds the P.V product straight from tensor memory.
@@ -43,7 +44,17 @@
 
 namespace tfa {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Registers: the kernel is compiled for 168 per thread at launch (384 x 168 =
+// 64512, the most three warps per SM sub-partition can hold).  The producer
+// warpgroup then gives back down to kRegsOther and the two softmax
+// warpgroups grow to kRegsSoftmax; 2*128*kRegsSoftmax + 128*kRegsOther must not
+// exceed 384*kRegsLaunch, or setmaxnreg.inc would wait forever.
+constexpr int kRegsLaunch = 168;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsOther = 104;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch,
+              "register split exceeds the launch pool");
 // Lazy rescale: keep the stale row maximum until the true one exceeds it by
 // more than 2^8 in the exp2 domain (P values then stay <= 256).
 constexpr float kRescaleThresholdLog2 = 8.0f;
@@ -424,7 +435,7 @@ __device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
 
 // ------------------------------------------------------------------ kernel
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kThreads, 1)
     tfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const Params p) {
@@ -470,14 +481,15 @@ __global__ void __maxnreg__(200)
     const uint32_t tmem = *tmem_slot;
 
     if (warp < 8) {
+        reg_alloc<kRegsSoftmax>();
         if (warp < 4)
             softmax_role<D, 0>(p, tmem, bar, abort_flag);
         else
             softmax_role<D, 1>(p, tmem, bar, abort_flag);
-    } else if (warp == 8) {
-        if (lane == 0) load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, bar, abort_flag);
-    } else if (warp == 9) {
-        if (lane == 0) mma_role<D>(p, sbase, tmem, bar, abort_flag);
+    } else {
+        reg_dealloc<kRegsOther>();
+        if (warp == 8 && lane == 0) load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, bar, abort_flag);
+        if (warp == 9 && lane == 0) mma_role<D>(p, sbase, tmem, bar, abort_flag);
     }
 
     tc_fence_before();
