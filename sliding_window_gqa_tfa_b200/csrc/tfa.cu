@@ -273,6 +273,16 @@ extern "C" int tfa_check_status(tfa_stream_t stream) {
 
 extern "C" const char *tfa_last_error(void) { return g_last_error; }
 
+#ifdef TFA_TRACE
+// Trace builds only: copy CTA 0's timeline (4 roles x kTraceSlots clocks) to host.
+extern "C" int tfa_trace_read(unsigned long long *host, size_t n) {
+    const size_t bytes = sizeof(tfa::g_tfa_trace);
+    if (n * sizeof(unsigned long long) < bytes) return TFA_ERR_SHAPE;
+    cudaError_t e = cudaMemcpyFromSymbol(host, tfa::g_tfa_trace, bytes);
+    return e == cudaSuccess ? TFA_OK : cuda_fail("cudaMemcpyFromSymbol(trace)", e);
+}
+#endif
+
 extern "C" const char *tfa_status_string(int status) {
     switch (status) {
         case TFA_OK: return "ok";

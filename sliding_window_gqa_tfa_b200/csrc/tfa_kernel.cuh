@@ -44,6 +44,24 @@
 
 namespace tfa {
 
+// Optional timeline trace of CTA 0 (compile with -DTFA_TRACE; compiled out
+// otherwise).  Role r in {0: softmax tile 0, 1: softmax tile 1, 2: MMA issuer,
+// 3: TMA producer, 4-7: warps 0-3 of softmax tile 0}; slot = 8 * step + event,
+// SM clock.
+#ifdef TFA_TRACE
+constexpr int kTraceSlots = 2048;
+__device__ unsigned long long g_tfa_trace[8][kTraceSlots];
+#define TFA_TR(role, step, ev)                                                      \
+    do {                                                                            \
+        const int _i = 8 * (step) + (ev);                                           \
+        if (blockIdx.x == 0 && _i < kTraceSlots) g_tfa_trace[role][_i] = clock64(); \
+    } while (0)
+#else
+#define TFA_TR(role, step, ev) \
+    do {                       \
+    } while (0)
+#endif
+
 constexpr int kThreads = 384;
 // Registers: the kernel is compiled for 168 per thread at launch (384 x 168 =
 // 64512, the most three warps per SM sub-partition can hold).  The producer
@@ -58,6 +76,16 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunc
 // Lazy rescale: keep the stale row maximum until the true one exceeds it by
 // more than 2^8 in the exp2 domain (P values then stay <= 256).
 constexpr float kRescaleThresholdLog2 = 8.0f;
+// One pair of exponentials in every kPolyPeriod goes to the FMA-pipe polynomial
+// instead of the MUFU unit (0: all on MUFU).  The MUFU unit alone (16/clk/SM)
+// needs as long for a 128 x 128 tile as the tensor core needs for its two MMAs,
+// but with one warp per row block the loop is latency-bound, not MUFU-bound, and
+// measured fastest with every exponential on MUFU; the polynomial path is kept
+// (tested) for configurations where the MUFU unit becomes the limit.
+#ifndef TFA_POLY_PERIOD
+#define TFA_POLY_PERIOD 0
+#endif
+constexpr int kPolyPeriod = TFA_POLY_PERIOD;
 
 template <int D>
 struct Cfg {
@@ -121,6 +149,27 @@ __device__ __forceinline__ ItemPlan plan_item(const Params &p, int item) {
         }
     }
     return ip;
+}
+
+// Query tile t of an item: first row q0, whether it exists, its key-tile range.
+struct TilePlan {
+    int b, h, q0, lo, hi;
+    bool present;
+};
+__device__ __forceinline__ TilePlan plan_tile(const Params &p, int item, int t) {
+    TilePlan tp;
+    const int bh = p.B * p.Hq;
+    const int r = item / bh;
+    const int rem = item - r * bh;
+    tp.b = rem / p.Hq;
+    tp.h = rem - tp.b * p.Hq;
+    const int qp = p.causal ? (p.n_qp - 1 - r) : r;
+    tp.q0 = qp * 2 * kBlockQ + t * kBlockQ;
+    tp.present = tp.q0 < p.L;
+    const KeyRange kr = qtile_key_range(p.L, p.S, p.causal, p.window, tp.q0, p.flags);
+    tp.lo = kr.lo;
+    tp.hi = kr.hi;
+    return tp;
 }
 
 struct Bars {
@@ -223,6 +272,8 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     uint32_t kv_cons = 0;
     uint32_t q_use[2] = {0, 0};
     uint32_t p_cnt[2] = {0, 0};
+    int trace_step = 0;
+    (void)trace_step;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
         const ItemPlan ip = plan_item(p, item);
 #pragma unroll
@@ -248,6 +299,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
         }
         bool acc[2] = {false, false};
         for (int j = ip.jl; j <= ip.jh; ++j) {
+            TFA_TR(2, trace_step, 0);
             const uint32_t sv = kv_cons % C::kSlots;
             if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
             ++kv_cons;
@@ -259,12 +311,14 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                     goto out;
                 ++kv_cons;
             }
+            TFA_TR(2, trace_step, 1);
             tc_fence_after();
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (!ip.present[t]) continue;
                 if (ip.lo[t] <= j && j <= ip.hi[t]) {
                     if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                    TFA_TR(2, trace_step, 2 + 2 * t);
                     ++p_cnt[t];
                     tc_fence_after();
                     issue_pv(t, sv, acc[t]);
@@ -276,7 +330,9 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                     umma_commit(bar.s_full(t));
                     if (j + 1 == ip.hi[t]) umma_commit(bar.q_empty(t));
                 }
+                TFA_TR(2, trace_step, 3 + 2 * t);
             }
+            ++trace_step;
             umma_commit(bar.kv_empty(sv));
             if (next) umma_commit(bar.kv_empty(sk));
         }
@@ -288,9 +344,9 @@ out:
 }
 
 // ---------------------------------------------------- softmax and epilogue
-template <int D, int t>
-__device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
-                             volatile int *abort_flag) {
+template <int D>
+__device__ __forceinline__ void softmax_role(const Params &p, const int t, uint32_t tmem,
+                                          const Bars &bar, volatile int *abort_flag) {
     using C = Cfg<D>;
     const int r = threadIdx.x - t * 128;  // row inside the query tile
     const uint32_t lane_base = (static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u) << 16;
@@ -301,11 +357,13 @@ __device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
     const bool has_km = p.key_mask != nullptr;
     const int lane = threadIdx.x & 31;
     uint32_t s_cnt = 0, o_cnt = 0;
+    int trace_step = 0;
+    (void)trace_step;
 
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-        const ItemPlan ip = plan_item(p, item);
-        if (!ip.present[t]) continue;
-        const int row = ip.q0[t] + r;
+        const TilePlan ip = plan_tile(p, item, t);
+        if (!ip.present) continue;
+        const int row = ip.q0 + r;
         const int pos = (p.S - p.L) + row;  // absolute position of this query row
         const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
         const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
@@ -314,28 +372,36 @@ __device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
         float l = 0.f;
         bool first = true;
 
-        for (int j = ip.lo[t]; j <= ip.hi[t]; ++j) {
+        for (int j = ip.lo; j <= ip.hi; ++j) {
+            if (r == 0) TFA_TR(t, trace_step, 0);
+            // key-mask values of this key tile, fetched before the wait so the
+            // load latency hides behind it (lane i holds columns i, i+32, ...)
+            float kmv[4] = {1.f, 1.f, 1.f, 1.f};
+            if (has_km) {
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    const int col = j * kBlockK + 32 * w + lane;
+                    kmv[w] = col < p.S ? __ldg(km_row + col) : 0.f;
+                }
+            }
             // all lanes leave together: the tcgen05 loads below are warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(t), s_cnt & 1, abort_flag, p.status)))
                 return;
             ++s_cnt;
+            if (r == 0) TFA_TR(t, trace_step, 1);
             tc_fence_after();
             uint32_t s[128];
             tmem_ld128(tS, s);
+            if (r == 0) TFA_TR(t, trace_step, 2);
+            if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 0);
 
-            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, has_km, ip.q0[t], j, p.flags)) {
+            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, has_km, ip.q0, j, p.flags)) {
                 const int k0 = j * kBlockK;
                 const int lo_c = lo_abs - k0;
                 const int hi_c = hi_abs - k0;
-                uint32_t kmw[4] = {~0u, ~0u, ~0u, ~0u};
-                if (has_km) {
+                uint32_t kmw[4];
 #pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        const int col = k0 + 32 * w + lane;
-                        const float mv = col < p.S ? __ldg(km_row + col) : 0.f;
-                        kmw[w] = __ballot_sync(0xffffffffu, mv > 0.5f);
-                    }
-                }
+                for (int w = 0; w < 4; ++w) kmw[w] = __ballot_sync(0xffffffffu, kmv[w] > 0.5f);
 #pragma unroll
                 for (int cidx = 0; cidx < 128; ++cidx) {
                     const bool keep = cidx >= lo_c && cidx <= hi_c && ((kmw[cidx >> 5] >> (cidx & 31)) & 1u);
@@ -343,16 +409,19 @@ __device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
                 }
             }
 
-            float mx0 = __uint_as_float(s[0]), mx1 = __uint_as_float(s[1]);
-            float mx2 = __uint_as_float(s[2]), mx3 = __uint_as_float(s[3]);
+            // row maximum: three-input max in four independent chains
+#define TFA_F(i) __uint_as_float(s[i])
+            float mx0 = fmaxf(TFA_F(0), TFA_F(4)), mx1 = fmaxf(TFA_F(1), TFA_F(5));
+            float mx2 = fmaxf(TFA_F(2), TFA_F(6)), mx3 = fmaxf(TFA_F(3), TFA_F(7));
 #pragma unroll
-            for (int i = 4; i < 128; i += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(s[i]));
-                mx1 = fmaxf(mx1, __uint_as_float(s[i + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(s[i + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(s[i + 3]));
+            for (int i = 8; i < 128; i += 8) {
+                mx0 = fmax3(mx0, TFA_F(i), TFA_F(i + 4));
+                mx1 = fmax3(mx1, TFA_F(i + 1), TFA_F(i + 5));
+                mx2 = fmax3(mx2, TFA_F(i + 2), TFA_F(i + 6));
+                mx3 = fmax3(mx3, TFA_F(i + 3), TFA_F(i + 7));
             }
-            const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)));
+            const float m_new = fmax3(m_ref, fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 1);
 
             // Decide the lazy rescale first; O_t itself is rescaled after P is
             // stored, once the S registers are dead.
@@ -373,22 +442,28 @@ __device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
             }
 
             const float mc = (m_ref == -CUDART_INF_F) ? 0.f : m_ref * c;
-            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+            const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
+            float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
             uint32_t pk[64];
 #pragma unroll
-            for (int i = 0; i < 64; i += 2) {
-                const float a0 = ex2(fmaf(__uint_as_float(s[2 * i]), c, -mc));
-                const float a1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), c, -mc));
-                const float a2 = ex2(fmaf(__uint_as_float(s[2 * i + 2]), c, -mc));
-                const float a3 = ex2(fmaf(__uint_as_float(s[2 * i + 3]), c, -mc));
-                l0 += a0;
-                l1 += a1;
-                l2 += a2;
-                l3 += a3;
-                pk[i] = pack_bf16(a0, a1);
-                pk[i + 1] = pack_bf16(a2, a3);
+            for (int i = 0; i < 64; ++i) {
+                const float2 x = fma2(make_float2(TFA_F(2 * i), TFA_F(2 * i + 1)), c2, nmc2);
+                float2 e;
+                if (kPolyPeriod > 0 && (i % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) {
+                    e = exp2_poly2(x);  // FMA pipe
+                } else {
+                    e.x = ex2(x.x);  // MUFU
+                    e.y = ex2(x.y);
+                }
+                if (i & 1)
+                    acc1 = add2(acc1, e);
+                else
+                    acc0 = add2(acc0, e);
+                pk[i] = pack_bf16(e.x, e.y);
             }
-            l = l * alpha + ((l0 + l1) + (l2 + l3));
+#undef TFA_F
+            const float2 acc = add2(acc0, acc1);
+            l = l * alpha + (acc.x + acc.y);
             tmem_st32(tP, pk);
             tmem_st32(tP + 32, pk + 32);
             if (rescale) {
@@ -401,9 +476,14 @@ __device__ void softmax_role(const Params &p, uint32_t tmem, const Bars &bar,
                     tmem_st32(tO + cc * 32, o);
                 }
             }
+            if (r == 0) TFA_TR(t, trace_step, 3);
+            if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 2);
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar.p_full(t));
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.p_full(t));  // one arrival per warp
+            if (r == 0) TFA_TR(t, trace_step, 4);
+            ++trace_step;
         }
 
         // Epilogue: final FP32 normalisation, then BF16 (a row with no allowed
@@ -455,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar.q_full(t), 1);
             mbar_init(bar.q_empty(t), 1);
             mbar_init(bar.s_full(t), 1);
-            mbar_init(bar.p_full(t), 128);
+            mbar_init(bar.p_full(t), 4);
             mbar_init(bar.o_full(t), 1);
         }
         for (int s = 0; s < C::kSlots; ++s) {
@@ -482,10 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         reg_alloc<kRegsSoftmax>();
-        if (warp < 4)
-            softmax_role<D, 0>(p, tmem, bar, abort_flag);
-        else
-            softmax_role<D, 1>(p, tmem, bar, abort_flag);
+        softmax_role<D>(p, warp >> 2, tmem, bar, abort_flag);
     } else {
         reg_dealloc<kRegsOther>();
         if (warp == 8 && lane == 0) load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, bar, abort_flag);
