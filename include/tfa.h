@@ -110,9 +110,32 @@ int tfa_prefill_host(const void *q, const void *k, const void *v, void *o,
                      int B, int Hq, int Hkv, int L, int S, int D, float scale,
                      int causal, int window, const float *key_mask, tfa_stream_t stream);
 
+/* tfa_prefill_noalloc -- tfa_prefill for callers that cannot allocate device
+ * memory (a caching or arena allocator owns all of it, allocation is not
+ * allowed at the point of the call, or the host runtime only hands out its own
+ * buffers).  No counterpart on the pages: it exists for those callers.
+ * Arguments, layout and results are exactly tfa_prefill's; the caller still
+ * passes every input and output.  The difference is the kernel's scratch (its
+ * status word): it lives in a fixed 256-byte device array inside the library,
+ * which every GPU that loads the library holds until the process exits, and
+ * the call makes no cudaMalloc, cudaFree or other allocating call.
+ *   - The first call on a device sets the array up (looks up its address and
+ *     clears it with that device current); make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other threads) race on it.
+ *   - A call whose scratch would exceed the 256-byte maximum is rejected with
+ *     TFA_ERR_SHAPE and a message in tfa_last_error(); today's kernel needs
+ *     4 bytes for every size tfa_prefill accepts.
+ *   - A timed-out kernel wait is reported by tfa_check_status, as for tfa_prefill. */
+int tfa_prefill_noalloc(const void *q, const void *k, const void *v, void *o,
+                        int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                        int causal, int window, const float *key_mask, tfa_stream_t stream);
+
 /* tfa_check_status -- synchronizes `stream`, then reads and clears the current
- * device's status word.  Returns TFA_OK, TFA_ERR_TIMEOUT if a kernel launched
- * since the last check recorded a wait that gave up, or TFA_ERR_CUDA. */
+ * device's status words (tfa_prefill's and, once set up, tfa_prefill_noalloc's).
+ * Returns TFA_OK, TFA_ERR_TIMEOUT if a kernel launched since the last check
+ * recorded a wait that gave up, or TFA_ERR_CUDA. */
 int tfa_check_status(tfa_stream_t stream);
 
 /* tfa_last_error -- for the calling host thread, a description of the last CUDA

@@ -68,6 +68,8 @@ def lib():
             L.tfa_prefill_debug.restype = i32
             L.tfa_prefill_host.argtypes = common
             L.tfa_prefill_host.restype = i32
+            L.tfa_prefill_noalloc.argtypes = common
+            L.tfa_prefill_noalloc.restype = i32
             L.tfa_check_status.argtypes = [P]
             L.tfa_check_status.restype = i32
             L.tfa_last_error.argtypes = []
@@ -111,6 +113,12 @@ def tfa_prefill_host(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key
                      stream) -> int:
     return lib().tfa_prefill_host(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window,
                                   key_mask, stream)
+
+
+def tfa_prefill_noalloc(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                        stream) -> int:
+    return lib().tfa_prefill_noalloc(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window,
+                                     key_mask, stream)
 
 
 def tfa_check_status(stream) -> int:

@@ -255,20 +255,91 @@ extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, voi
     return TFA_OK;
 }
 
+// ------------------------------------------------------------------------
+// No-allocation variant.
+//
+// Some callers cannot call cudaMalloc at all: code that runs under a caching
+// or arena allocator that owns all device memory, code that must not allocate
+// while a graph is being recorded or while latency-critical work is running,
+// and embedded runtimes that hand the library only their own buffers.  For
+// them, tfa_prefill_noalloc runs the same kernel as tfa_prefill, but the
+// kernel's scratch (its status word) lives in this file-scope device array,
+// which every GPU that loads the library holds until the process exits.  In
+// host code the array's name is only a host-side stand-in, never a device
+// address: its real address is looked up with cudaGetSymbolAddress once per
+// device, with that device current, and passed to the kernel.
+constexpr size_t kNoAllocScratchBytes = 256;            // the stated maximum
+constexpr size_t kKernelScratchBytes = sizeof(unsigned);  // what the kernel needs today
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+DeviceState g_noalloc_dev[kMaxDevices];  // set up by the first tfa_prefill_noalloc per device
+
+int noalloc_state(cudaStream_t stream, DeviceState **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return drv_fail("device index out of range", dev);
+    DeviceState &st = g_noalloc_dev[dev];
+    if (!st.init) {
+        void *ptr = nullptr;
+        if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess)
+            return cuda_fail("cudaGetSymbolAddress(no-alloc scratch)", e);
+        // the status word must start at zero; clearing is not an allocation
+        if ((e = cudaMemsetAsync(ptr, 0, kNoAllocScratchBytes, stream)) != cudaSuccess)
+            return cuda_fail("cudaMemsetAsync(no-alloc scratch)", e);
+        if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail("cudaDeviceGetAttribute", e);
+        if (int rc = get_encode_fn()) return rc;
+        st.status = static_cast<unsigned *>(ptr);
+        st.init = true;
+    }
+    *out = &st;
+    return TFA_OK;
+}
+
+// Reads and clears one status word (synchronous); TFA_OK, TFA_ERR_TIMEOUT or TFA_ERR_CUDA.
+int take_status_word(unsigned *status) {
+    unsigned word = 0;
+    if (cudaMemcpy(&word, status, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return TFA_ERR_CUDA;
+    if (word == 0) return TFA_OK;
+    if (cudaMemset(status, 0, sizeof word) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
+        return TFA_ERR_CUDA;
+    return TFA_ERR_TIMEOUT;
+}
+}  // namespace
+
+extern "C" int tfa_prefill_noalloc(const void *q, const void *k, const void *v, void *o, int B,
+                                   int Hq, int Hkv, int L, int S, int D, float scale, int causal,
+                                   int window, const float *key_mask, tfa_stream_t stream) {
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
+    if (rc) return rc;
+    if (kKernelScratchBytes > kNoAllocScratchBytes) {
+        snprintf(g_last_error, sizeof g_last_error,
+                 "this call needs %zu bytes of scratch, more than the %zu-byte no-alloc maximum",
+                 kKernelScratchBytes, kNoAllocScratchBytes);
+        return TFA_ERR_SHAPE;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = noalloc_state(s, &st))) return rc;
+    return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                    key_mask, s, 0u)
+                      : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                   key_mask, s, 0u);
+}
+
 extern "C" int tfa_check_status(tfa_stream_t stream) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TFA_ERR_CUDA;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TFA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mutex);
-    DeviceState &st = g_dev[dev];
-    if (!st.init) return TFA_OK;
-    unsigned word = 0;
-    if (cudaMemcpy(&word, st.status, sizeof word, cudaMemcpyDeviceToHost) != cudaSuccess)
-        return TFA_ERR_CUDA;
-    if (word == 0) return TFA_OK;
-    if (cudaMemset(st.status, 0, sizeof word) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
-        return TFA_ERR_CUDA;
-    return TFA_ERR_TIMEOUT;
+    int rc = TFA_OK;
+    if (g_dev[dev].init) rc = take_status_word(g_dev[dev].status);
+    if (rc == TFA_OK && g_noalloc_dev[dev].init) rc = take_status_word(g_noalloc_dev[dev].status);
+    return rc;
 }
 
 extern "C" const char *tfa_last_error(void) { return g_last_error; }
