@@ -90,6 +90,11 @@ int tfa_prefill(const void *q, const void *k, const void *v, void *o,
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
 #define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */
 #define TFA_DEBUG_SYNC          4u /* synchronize the stream and return the device status */
+#define TFA_DEBUG_NO_SPLIT      8u /* deal whole work items round-robin instead of splitting
+                                      key ranges evenly across the CTAs (no partial merges) */
+#define TFA_DEBUG_FORCE_SPLIT  16u /* always split key ranges evenly across the CTAs (by
+                                      default the library picks the schedule it estimates
+                                      finishes first) */
 
 /* tfa_prefill_debug -- tfa_prefill with debug flags (arguments as above).  With
  * NO_TILE_SKIP and/or MASK_ALL the result must be bit-identical to tfa_prefill's
@@ -156,6 +161,24 @@ const char *tfa_status_string(int status);
  * error for the sizes.  No device work. */
 int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_mask, int qtile,
                    int *kt_lo, int *kt_hi, unsigned char *needs_mask, int needs_mask_len);
+
+/* tfa_plan_pieces -- host view of the work one CTA of a grid of `grid` CTAs
+ * performs (no device work).  The work of (batch, query head, pair of 128-row
+ * query tiles) is the union of the two tiles' key-tile ranges.  With split != 0
+ * (tfa_prefill's schedule) the concatenated key-tile steps of all such items
+ * are cut into `grid` contiguous ranges of almost equal length; a cut item is
+ * finished by the piece holding a tile's first key tile, which merges the
+ * others' partial softmax statistics.  With split == 0 items go round-robin.
+ *   out          10 ints per piece: item, qp, b, h, first key tile, last key
+ *                tile, role of tile 0, role of tile 1 (bit 0 active, bit 1
+ *                finalizer, bit 2 complete), and for a finalizer that must
+ *                merge, the last CTA contributing to tile 0 / tile 1 (else -1)
+ *   *n_pieces    number of pieces of this CTA (written even when > max_pieces)
+ *   total_steps  if not NULL, the total number of key-tile steps
+ * Returns TFA_OK, TFA_ERR_SHAPE (bad grid/cta, or more than max_pieces), or a
+ * validation error for the sizes (Hkv is taken equal to Hq, D as 128). */
+int tfa_plan_pieces(int B, int Hq, int L, int S, int causal, int window, int grid, int split,
+                    int cta, int *out, int max_pieces, int *n_pieces, long long *total_steps);
 
 /* Tile sizes of the kernel: 128 query rows x 128 keys per tensor-core tile. */
 #define TFA_BLOCK_Q 128

@@ -35,6 +35,8 @@ TFA_ERR_FLAGS = 11
 TFA_DEBUG_NO_TILE_SKIP = 1
 TFA_DEBUG_MASK_ALL = 2
 TFA_DEBUG_SYNC = 4
+TFA_DEBUG_NO_SPLIT = 8
+TFA_DEBUG_FORCE_SPLIT = 16
 
 MIN_QUERY_ROWS = 9
 BLOCK_Q = 128
@@ -79,6 +81,9 @@ def lib():
             L.tfa_plan_qtile.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(i32),
                                          ctypes.POINTER(i32), P, i32]
             L.tfa_plan_qtile.restype = i32
+            L.tfa_plan_pieces.argtypes = [i32] * 9 + [P, i32, ctypes.POINTER(i32),
+                                                      ctypes.POINTER(ctypes.c_longlong)]
+            L.tfa_plan_pieces.restype = i32
             _lib = L
     return _lib
 
@@ -135,6 +140,19 @@ def tfa_plan_qtile(L, S, causal, window, has_key_mask, qtile):
     if rc:
         return rc, None, None, None
     return rc, lo.value, hi.value, [bool(buf[i]) for i in range(hi.value - lo.value + 1)]
+
+
+def tfa_plan_pieces(B, Hq, L, S, causal, window, grid, split, cta, max_pieces=4096):
+    """Returns (status, total_steps, pieces) with pieces as tuples of 10 ints."""
+    buf = (ctypes.c_int * (10 * max_pieces))()
+    n = ctypes.c_int(0)
+    w = ctypes.c_longlong(0)
+    rc = lib().tfa_plan_pieces(B, Hq, L, S, int(causal), window, grid, int(split), cta,
+                               ctypes.cast(buf, ctypes.c_void_p), max_pieces, ctypes.byref(n),
+                               ctypes.byref(w))
+    if rc:
+        return rc, None, None
+    return rc, w.value, [tuple(buf[10 * i:10 * i + 10]) for i in range(n.value)]
 
 
 # ---------------------------------------------------------- torch wrapper

@@ -11,6 +11,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -23,11 +24,21 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Scratch of the split schedule, one set per (device, stream) so that calls on
+// different streams never share it: a partial slot and a ready flag per
+// (CTA, query tile), and the epoch that marks this stream's latest launch.
+struct SplitScratch {
+    float *partial = nullptr;
+    unsigned *ready = nullptr;
+    unsigned epoch = 0;
+};
+
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
     unsigned *status = nullptr;  // device status word (TFA_DEVICE_TIMEOUT bits)
     bool smem_attr[2] = {false, false};
+    std::unordered_map<cudaStream_t, SplitScratch> split;
     // staging buffers of tfa_prefill_host
     void *h_buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
     size_t h_cap[5] = {0, 0, 0, 0, 0};
@@ -82,6 +93,28 @@ int device_state(cudaStream_t stream, DeviceState **out) {
     return TFA_OK;
 }
 
+// The split schedule's scratch for `stream`, allocated on first use: 2 slots of
+// partial_slot_floats<128> floats and 2 flags per CTA (one CTA per SM at most).
+int split_scratch(DeviceState &st, cudaStream_t stream, SplitScratch **out) {
+    auto found = st.split.find(stream);
+    if (found != st.split.end()) {
+        *out = &found->second;
+        return TFA_OK;
+    }
+    SplitScratch ss;
+    const size_t slots = 2 * static_cast<size_t>(st.sm_count);
+    cudaError_t e = cudaMalloc(&ss.partial, slots * tfa::partial_slot_floats<128>() * sizeof(float));
+    if (e != cudaSuccess) return cuda_fail("cudaMalloc(split partials)", e);
+    if ((e = cudaMalloc(&ss.ready, slots * sizeof(unsigned))) != cudaSuccess) {
+        cudaFree(ss.partial);
+        return cuda_fail("cudaMalloc(split flags)", e);
+    }
+    if ((e = cudaMemsetAsync(ss.ready, 0, slots * sizeof(unsigned), stream)) != cudaSuccess)
+        return cuda_fail("cudaMemsetAsync(split flags)", e);
+    *out = &st.split.emplace(stream, ss).first->second;
+    return TFA_OK;
+}
+
 int validate(const void *q, const void *k, const void *v, const void *o, int B, int Hq, int Hkv,
              int L, int S, int D, float scale, int causal, int window, const float *key_mask,
              bool check_pointers) {
@@ -124,7 +157,7 @@ int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D) {
 template <int D>
 int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o, int B, int Hq,
            int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
-           cudaStream_t stream, unsigned flags) {
+           cudaStream_t stream, unsigned flags, SplitScratch *ss, bool force_split = false) {
     using C = tfa::Cfg<D>;
     CUtensorMap mq, mk, mv;
     if (encode_map(&mq, q, L, B * Hq, D) || encode_map(&mk, k, S, B * Hkv, D) ||
@@ -160,13 +193,40 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.L = L;
     p.S = S;
     p.G = Hq / Hkv;
-    p.n_qp = (L + 2 * tfa::kBlockQ - 1) / (2 * tfa::kBlockQ);
-    p.n_items = B * Hq * p.n_qp;
     p.causal = causal ? 1 : 0;
     p.window = (causal && window > 0) ? window : 0;
     p.flags = flags;
     p.scale_log2 = scale * 1.4426950408889634f;
-    const int grid = p.n_items < st.sm_count ? p.n_items : st.sm_count;
+    tfa::Shape &sh = p.shape;
+    sh.B = B;
+    sh.Hq = Hq;
+    sh.L = L;
+    sh.S = S;
+    sh.causal = p.causal;
+    sh.window = p.window;
+    sh.flags = flags;
+    sh.n_qp = tfa::shape_n_qp(L);
+    const long long n_items = static_cast<long long>(B) * Hq * sh.n_qp;
+    p.W = tfa::total_steps(sh);
+    // whole-item schedule, and the split one when scratch exists and the
+    // estimate says it finishes sooner (few, large items per CTA)
+    sh.split = 0;
+    sh.grid = n_items < st.sm_count ? static_cast<int>(n_items) : st.sm_count;
+    if (ss != nullptr && (n_items <= (1 << 16) || force_split)) {
+        tfa::Shape sp = sh;
+        sp.split = 1;
+        sp.grid = p.W < st.sm_count ? static_cast<int>(p.W) : st.sm_count;
+        if (force_split || tfa::makespan_estimate(sp, p.W) < tfa::makespan_estimate(sh, p.W)) sh = sp;
+    }
+    if (!sh.split) ss = nullptr;
+    const int grid = sh.grid;
+    p.partial = ss ? ss->partial : nullptr;
+    p.ready = ss ? ss->ready : nullptr;
+    p.epoch = 0;
+    if (ss) {
+        if (++ss->epoch == 0) ++ss->epoch;  // 0 is the flags' initial value
+        p.epoch = ss->epoch;
+    }
     kern<<<grid, tfa::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFA_OK : cuda_fail("kernel launch", e);
@@ -177,20 +237,22 @@ int prefill_impl(const void *q, const void *k, const void *v, void *o, int B, in
                  cudaStream_t stream, unsigned flags) {
     int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
     if (rc) return rc;
-    if (flags & ~(TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL | TFA_DEBUG_SYNC)) return TFA_ERR_FLAGS;
+    if (flags & ~(TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL | TFA_DEBUG_SYNC | TFA_DEBUG_NO_SPLIT |
+                  TFA_DEBUG_FORCE_SPLIT) ||
+        ((flags & TFA_DEBUG_NO_SPLIT) && (flags & TFA_DEBUG_FORCE_SPLIT)))
+        return TFA_ERR_FLAGS;
+    const bool force_split = (flags & TFA_DEBUG_FORCE_SPLIT) != 0;
     DeviceState *st = nullptr;
-    {
-        std::lock_guard<std::mutex> lk(g_mutex);
-        rc = device_state(stream, &st);
-    }
-    if (rc) return rc;
+    SplitScratch *ss = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(stream, &st))) return rc;
+    if (!(flags & TFA_DEBUG_NO_SPLIT) && (rc = split_scratch(*st, stream, &ss))) return rc;
     const unsigned kflags = flags & (TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL);
     rc = (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
-                                  key_mask, stream, kflags)
+                                  key_mask, stream, kflags, ss, force_split)
                     : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
-                                 key_mask, stream, kflags);
+                                 key_mask, stream, kflags, ss, force_split);
     if (rc) return rc;
-    if (flags & TFA_DEBUG_SYNC) return tfa_check_status(reinterpret_cast<tfa_stream_t>(stream));
     return TFA_OK;
 }
 
@@ -217,8 +279,10 @@ extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, vo
                                  int Hq, int Hkv, int L, int S, int D, float scale, int causal,
                                  int window, const float *key_mask, tfa_stream_t stream,
                                  unsigned flags) {
-    return prefill_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
-                        reinterpret_cast<cudaStream_t>(stream), flags);
+    const int rc = prefill_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                                reinterpret_cast<cudaStream_t>(stream), flags);
+    if (rc == TFA_OK && (flags & TFA_DEBUG_SYNC)) return tfa_check_status(stream);
+    return rc;
 }
 
 extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, void *o, int B,
@@ -244,10 +308,12 @@ extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, voi
                        cudaSuccess))
         return TFA_ERR_CUDA;
     const float *dmask = mbytes ? static_cast<const float *>(st->h_buf[4]) : nullptr;
+    SplitScratch *ss = nullptr;
+    if ((rc = split_scratch(*st, s, &ss))) return rc;
     rc = (D == 128) ? launch<128>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
-                                  Hkv, L, S, scale, causal, window, dmask, s, 0u)
+                                  Hkv, L, S, scale, causal, window, dmask, s, 0u, ss)
                     : launch<64>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
-                                 Hkv, L, S, scale, causal, window, dmask, s, 0u);
+                                 Hkv, L, S, scale, causal, window, dmask, s, 0u, ss);
     if (rc) return rc;
     if (cudaMemcpyAsync(o, st->h_buf[3], qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return TFA_ERR_CUDA;
@@ -325,10 +391,11 @@ extern "C" int tfa_prefill_noalloc(const void *q, const void *k, const void *v, 
     DeviceState *st = nullptr;
     std::lock_guard<std::mutex> lk(g_mutex);
     if ((rc = noalloc_state(s, &st))) return rc;
+    // whole-item schedule: the split schedule's partials would not fit the static array
     return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
-                                    key_mask, s, 0u)
+                                    key_mask, s, 0u, nullptr)
                       : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
-                                   key_mask, s, 0u);
+                                   key_mask, s, 0u, nullptr);
 }
 
 extern "C" int tfa_check_status(tfa_stream_t stream) {
@@ -351,6 +418,13 @@ extern "C" int tfa_trace_read(unsigned long long *host, size_t n) {
     if (n * sizeof(unsigned long long) < bytes) return TFA_ERR_SHAPE;
     cudaError_t e = cudaMemcpyFromSymbol(host, tfa::g_tfa_trace, bytes);
     return e == cudaSuccess ? TFA_OK : cuda_fail("cudaMemcpyFromSymbol(trace)", e);
+}
+// Trace builds only: per-CTA start / end global-timer stamps (1024 x 2).
+extern "C" int tfa_trace_cta_times(unsigned long long *host, size_t n) {
+    const size_t bytes = sizeof(tfa::g_tfa_cta_time);
+    if (n * sizeof(unsigned long long) < bytes) return TFA_ERR_SHAPE;
+    cudaError_t e = cudaMemcpyFromSymbol(host, tfa::g_tfa_cta_time, bytes);
+    return e == cudaSuccess ? TFA_OK : cuda_fail("cudaMemcpyFromSymbol(cta times)", e);
 }
 #endif
 
@@ -390,4 +464,54 @@ extern "C" int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_
                                                             has_key_mask, q0, j, 0u) ? 1 : 0;
     }
     return TFA_OK;
+}
+
+extern "C" int tfa_plan_pieces(int B, int Hq, int L, int S, int causal, int window, int grid,
+                               int split, int cta, int *out, int max_pieces, int *n_pieces,
+                               long long *total_steps) {
+    int rc = validate(nullptr, nullptr, nullptr, nullptr, B, Hq, Hq, L, S, 128, 1.0f, causal,
+                      window, nullptr, false);
+    if (rc) return rc;
+    if (!n_pieces || (max_pieces > 0 && !out)) return TFA_ERR_NULL;
+    tfa::Shape sh;
+    sh.B = B;
+    sh.Hq = Hq;
+    sh.L = L;
+    sh.S = S;
+    sh.causal = causal ? 1 : 0;
+    sh.window = (causal && window > 0) ? window : 0;
+    sh.flags = 0;
+    sh.n_qp = tfa::shape_n_qp(L);
+    sh.split = split ? 1 : 0;
+    sh.grid = grid;
+    const long long W = tfa::total_steps(sh);
+    if (total_steps) *total_steps = W;
+    const long long units = sh.split ? W : static_cast<long long>(B) * Hq * sh.n_qp;
+    if (grid < 1 || grid > units || cta < 0 || cta >= grid) return TFA_ERR_SHAPE;
+    tfa::SegIter it;
+    it.init(sh, W, cta);
+    tfa::Segment seg;
+    int n = 0;
+    while (it.next(sh, seg)) {
+        if (n < max_pieces) {
+            const tfa::ItemSpan sp = tfa::item_span(sh, seg.qp);
+            int *o = out + 10 * n;
+            o[0] = seg.item;
+            o[1] = seg.qp;
+            o[2] = seg.b;
+            o[3] = seg.h;
+            o[4] = seg.jb;
+            o[5] = seg.je;
+            for (int t = 0; t < 2; ++t) {
+                const tfa::TileRole tr = tfa::tile_role(sh, seg, sp, t);
+                o[6 + t] = (tr.active ? 1 : 0) | (tr.finalizer ? 2 : 0) | (tr.complete ? 4 : 0);
+                o[8 + t] = (tr.active && tr.finalizer && !tr.complete)
+                               ? tfa::last_contributor(W, grid, cta, seg, sp, t)
+                               : -1;
+            }
+        }
+        ++n;
+    }
+    *n_pieces = n;
+    return n <= max_pieces ? TFA_OK : TFA_ERR_SHAPE;
 }

@@ -41,6 +41,7 @@
 
 #include "tfa_plan.h"
 #include "tfa_ptx.cuh"
+#include "tfa_sched.h"
 
 namespace tfa {
 
@@ -51,6 +52,7 @@ namespace tfa {
 #ifdef TFA_TRACE
 constexpr int kTraceSlots = 2048;
 __device__ unsigned long long g_tfa_trace[8][kTraceSlots];
+__device__ unsigned long long g_tfa_cta_time[1024][2];  // global-timer ns at start / end
 #define TFA_TR(role, step, ev)                                                      \
     do {                                                                            \
         const int _i = 8 * (step) + (ev);                                           \
@@ -69,8 +71,8 @@ constexpr int kThreads = 384;
 // warpgroups grow to kRegsSoftmax; 2*128*kRegsSoftmax + 128*kRegsOther must not
 // exceed 384*kRegsLaunch, or setmaxnreg.inc would wait forever.
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsSoftmax = 200;
-constexpr int kRegsOther = 104;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsOther = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch,
               "register split exceeds the launch pool");
 // Lazy rescale: keep the stale row maximum until the true one exceeds it by
@@ -97,7 +99,7 @@ struct Cfg {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-    static constexpr int kNumBars = 10 + 2 * kSlots + 1;
+    static constexpr int kNumBars = 10 + 2 * kSlots + 1 + 4;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
     static constexpr uint32_t kTmemCols = 512;
@@ -110,12 +112,20 @@ struct Params {
     __nv_bfloat16 *o;
     const float *key_mask;
     unsigned *status;
+    float *partial;    // split schedule: per (CTA, tile) partial m, l, accumulator
+    unsigned *ready;   // split schedule: per (CTA, tile) flag, == epoch when published
+    unsigned epoch;    // nonzero, different for every launch that uses `ready`
     int B, Hq, Hkv, L, S, G;
-    int n_qp, n_items;
     int causal, window;
     unsigned flags;
     float scale_log2;  // softmax scale * log2(e)
+    long long W;       // total key-tile steps (split schedule)
+    Shape shape;
 };
+
+// Floats of one partial slot: the accumulator [128][D], then m[128], l[128].
+template <int D>
+__host__ __device__ constexpr int partial_slot_floats() { return 128 * D + 256; }
 
 struct ItemPlan {
     int b, h, g;
@@ -125,51 +135,24 @@ struct ItemPlan {
     int jl, jh;
 };
 
-__device__ __forceinline__ ItemPlan plan_item(const Params &p, int item) {
+// The two query tiles of one piece of work, clipped to the piece's key tiles.
+__device__ __forceinline__ ItemPlan plan_piece(const Params &p, const Segment &seg) {
     ItemPlan ip;
-    const int bh = p.B * p.Hq;
-    const int r = item / bh;
-    const int rem = item - r * bh;
-    ip.b = rem / p.Hq;
-    ip.h = rem - ip.b * p.Hq;
-    ip.g = ip.h / p.G;
-    const int qp = p.causal ? (p.n_qp - 1 - r) : r;
-    ip.jl = 0x7fffffff;
-    ip.jh = -1;
+    ip.b = seg.b;
+    ip.h = seg.h;
+    ip.g = seg.h / p.G;
+    ip.jl = seg.jb;
+    ip.jh = seg.je;
+    const ItemSpan sp = item_span(p.shape, seg.qp);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-        ip.q0[t] = qp * 2 * kBlockQ + t * kBlockQ;
-        ip.present[t] = ip.q0[t] < p.L;
-        const KeyRange kr = qtile_key_range(p.L, p.S, p.causal, p.window, ip.q0[t], p.flags);
-        ip.lo[t] = kr.lo;
-        ip.hi[t] = ip.present[t] ? kr.hi : -1;
-        if (ip.present[t]) {
-            ip.jl = imin(ip.jl, kr.lo);
-            ip.jh = imax(ip.jh, kr.hi);
-        }
+        const TileRole tr = tile_role(p.shape, seg, sp, t);
+        ip.q0[t] = seg.qp * 2 * kBlockQ + t * kBlockQ;
+        ip.present[t] = tr.active;
+        ip.lo[t] = tr.lo;
+        ip.hi[t] = tr.active ? tr.hi : -1;
     }
     return ip;
-}
-
-// Query tile t of an item: first row q0, whether it exists, its key-tile range.
-struct TilePlan {
-    int b, h, q0, lo, hi;
-    bool present;
-};
-__device__ __forceinline__ TilePlan plan_tile(const Params &p, int item, int t) {
-    TilePlan tp;
-    const int bh = p.B * p.Hq;
-    const int r = item / bh;
-    const int rem = item - r * bh;
-    tp.b = rem / p.Hq;
-    tp.h = rem - tp.b * p.Hq;
-    const int qp = p.causal ? (p.n_qp - 1 - r) : r;
-    tp.q0 = qp * 2 * kBlockQ + t * kBlockQ;
-    tp.present = tp.q0 < p.L;
-    const KeyRange kr = qtile_key_range(p.L, p.S, p.causal, p.window, tp.q0, p.flags);
-    tp.lo = kr.lo;
-    tp.hi = kr.hi;
-    return tp;
 }
 
 struct Bars {
@@ -183,6 +166,10 @@ struct Bars {
     __device__ __forceinline__ uint32_t kv_full(int s) const { return base + 8 * (10 + s); }
     __device__ __forceinline__ uint32_t kv_empty(int s) const { return base + 8 * (10 + slots + s); }
     __device__ __forceinline__ uint32_t done() const { return base + 8 * (10 + 2 * slots); }
+    // split schedule: the four warps of tile t stored their partial / the
+    // finalizer thread saw every contributor's flag
+    __device__ __forceinline__ uint32_t pub(int t) const { return base + 8 * (11 + 2 * slots + t); }
+    __device__ __forceinline__ uint32_t fin(int t) const { return base + 8 * (13 + 2 * slots + t); }
 };
 
 // ------------------------------------------------------------------ producer
@@ -193,8 +180,11 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
     using C = Cfg<D>;
     uint32_t kv_prod = 0;
     uint32_t q_use[2] = {0, 0};
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-        const ItemPlan ip = plan_item(p, item);
+    SegIter it;
+    it.init(p.shape, p.W, blockIdx.x);
+    Segment seg;
+    while (it.next(p.shape, seg)) {
+        const ItemPlan ip = plan_piece(p, seg);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (!ip.present[t]) continue;
@@ -274,8 +264,11 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     uint32_t p_cnt[2] = {0, 0};
     int trace_step = 0;
     (void)trace_step;
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-        const ItemPlan ip = plan_item(p, item);
+    SegIter it;
+    it.init(p.shape, p.W, blockIdx.x);
+    Segment seg;
+    while (it.next(p.shape, seg)) {
+        const ItemPlan ip = plan_piece(p, seg);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (!ip.present[t]) continue;
@@ -356,18 +349,22 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     const float c = p.scale_log2;
     const bool has_km = p.key_mask != nullptr;
     const int lane = threadIdx.x & 31;
-    uint32_t s_cnt = 0, o_cnt = 0;
+    uint32_t s_cnt = 0, o_cnt = 0, pub_cnt = 0, fin_cnt = 0;
     int trace_step = 0;
     (void)trace_step;
 
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-        const TilePlan ip = plan_tile(p, item, t);
-        if (!ip.present) continue;
-        const int row = ip.q0 + r;
+    SegIter it;
+    it.init(p.shape, p.W, blockIdx.x);
+    Segment seg;
+    while (it.next(p.shape, seg)) {
+        const ItemSpan sp = item_span(p.shape, seg.qp);
+        const TileRole ip = tile_role(p.shape, seg, sp, t);
+        if (!ip.active) continue;
+        const int row = seg.qp * 2 * kBlockQ + t * kBlockQ + r;
         const int pos = (p.S - p.L) + row;  // absolute position of this query row
         const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
         const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
-        const float *km_row = has_km ? p.key_mask + static_cast<size_t>(ip.b) * p.S : nullptr;
+        const float *km_row = has_km ? p.key_mask + static_cast<size_t>(seg.b) * p.S : nullptr;
         float m_ref = -CUDART_INF_F;  // row maximum the exponentials are taken against
         float l = 0.f;
         bool first = true;
@@ -395,7 +392,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (r == 0) TFA_TR(t, trace_step, 2);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 0);
 
-            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, has_km, ip.q0, j, p.flags)) {
+            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, has_km, row - r, j, p.flags)) {
                 const int k0 = j * kBlockK;
                 const int lo_c = lo_abs - k0;
                 const int hi_c = hi_abs - k0;
@@ -486,19 +483,95 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             ++trace_step;
         }
 
-        // Epilogue: final FP32 normalisation, then BF16 (a row with no allowed
-        // key has l == 0 and is written as zeros).
         if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(t), o_cnt & 1, abort_flag, p.status)))
             return;
         ++o_cnt;
         tc_fence_after();
+
+        if (!ip.complete && !ip.finalizer) {
+            // A later piece of this tile's key range: publish the partial
+            // (unscaled accumulator, row max, row sum) for the finalizer.
+            float *slot = p.partial + static_cast<size_t>(blockIdx.x * 2 + t) * partial_slot_floats<D>();
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld32(tO + cc * 32, o);
+                float4 *dst = reinterpret_cast<float4 *>(slot + r * D + cc * 32);
+#pragma unroll
+                for (int v4 = 0; v4 < 8; ++v4)
+                    __stcg(dst + v4, make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
+                                                 __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3])));
+            }
+            __stcg(slot + 128 * D + r, m_ref);
+            __stcg(slot + 128 * D + 128 + r, l);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.pub(t));
+            if (r == 0 && mbar_wait(bar.pub(t), pub_cnt & 1, abort_flag, p.status)) {
+                __threadfence();
+                st_release_gpu(p.ready + blockIdx.x * 2 + t, p.epoch);
+            }
+            ++pub_cnt;
+            continue;
+        }
+
+        // Finalizer of a split tile: merge the partials of the CTAs that hold
+        // the rest of its key range (tiny-llm Week 2 Day 5, Task 1 merge).
+        float f_own = 1.f, m_star = m_ref;
+        int c_last = blockIdx.x;
+        if (!ip.complete) {
+            c_last = last_contributor(p.W, gridDim.x, blockIdx.x, seg, sp, t);
+            if (r == 0) {
+                bool ok = true;
+                for (int k = blockIdx.x + 1; k <= c_last && ok; ++k)
+                    ok = flag_wait(p.ready + k * 2 + t, p.epoch, abort_flag, p.status);
+                mbar_arrive(bar.fin(t));  // arrive even on failure; the abort flag tells
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.fin(t), fin_cnt & 1, abort_flag, p.status)))
+                return;
+            ++fin_cnt;
+            if (*abort_flag) return;
+            for (int k = blockIdx.x + 1; k <= c_last; ++k) {
+                (void)ld_acquire_gpu(p.ready + k * 2 + t);
+                const float *slot = p.partial + static_cast<size_t>(k * 2 + t) * partial_slot_floats<D>();
+                m_star = fmaxf(m_star, __ldcg(slot + 128 * D + r));
+            }
+            f_own = (m_ref == -CUDART_INF_F) ? 0.f : ex2((m_ref - m_star) * c);
+            l *= f_own;
+            for (int k = blockIdx.x + 1; k <= c_last; ++k) {
+                const float *slot = p.partial + static_cast<size_t>(k * 2 + t) * partial_slot_floats<D>();
+                const float mk = __ldcg(slot + 128 * D + r);
+                const float fk = (mk == -CUDART_INF_F) ? 0.f : ex2((mk - m_star) * c);
+                l += fk * __ldcg(slot + 128 * D + 128 + r);
+            }
+        }
+
+        // Final FP32 normalisation, then BF16 (a row with no allowed key has
+        // l == 0 and is written as zeros).
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16 *orow =
-            p.o + (static_cast<size_t>(ip.b * p.Hq + ip.h) * p.L + row) * static_cast<size_t>(D);
+            p.o + (static_cast<size_t>(seg.b * p.Hq + seg.h) * p.L + row) * static_cast<size_t>(D);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
+            if (!ip.complete) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f_own);
+                for (int k = blockIdx.x + 1; k <= c_last; ++k) {
+                    const float *slot = p.partial + static_cast<size_t>(k * 2 + t) * partial_slot_floats<D>();
+                    const float mk = __ldcg(slot + 128 * D + r);
+                    const float fk = (mk == -CUDART_INF_F) ? 0.f : ex2((mk - m_star) * c);
+                    const float4 *src = reinterpret_cast<const float4 *>(slot + r * D + cc * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 8; ++v4) {
+                        const float4 a = __ldcg(src + v4);
+                        o[4 * v4] = __float_as_uint(fmaf(fk, a.x, __uint_as_float(o[4 * v4])));
+                        o[4 * v4 + 1] = __float_as_uint(fmaf(fk, a.y, __uint_as_float(o[4 * v4 + 1])));
+                        o[4 * v4 + 2] = __float_as_uint(fmaf(fk, a.z, __uint_as_float(o[4 * v4 + 2])));
+                        o[4 * v4 + 3] = __float_as_uint(fmaf(fk, a.w, __uint_as_float(o[4 * v4 + 3])));
+                    }
+                }
+            }
             uint32_t w[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i)
@@ -543,6 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar.kv_empty(s), 1);
         }
         mbar_init(bar.done(), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(bar.pub(t), 4);
+            mbar_init(bar.fin(t), 1);
+        }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -559,6 +636,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+#ifdef TFA_TRACE
+    if (threadIdx.x == 0 && blockIdx.x < 1024) g_tfa_cta_time[blockIdx.x][0] = globaltimer_ns();
+#endif
 
     if (warp < 8) {
         reg_alloc<kRegsSoftmax>();
@@ -571,6 +651,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     tc_fence_before();
     __syncthreads();
+#ifdef TFA_TRACE
+    if (threadIdx.x == 0 && blockIdx.x < 1024) g_tfa_cta_time[blockIdx.x][1] = globaltimer_ns();
+#endif
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);

@@ -15,6 +15,12 @@ namespace tfa {
 constexpr long long TFA_WAIT_LIMIT_CYCLES = 8ll << 30;  // ~4 s at 2 GHz
 constexpr unsigned TFA_DEVICE_TIMEOUT = 1u;
 
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -185,6 +191,35 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 #undef TFA_W8
+
+// Named barrier `id` (1..15) over `n` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// GPU-scope publication / observation of a flag in global memory.
+__device__ __forceinline__ void st_release_gpu(unsigned *addr, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *addr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    return v;
+}
+// Wait, bounded like mbar_wait, until *flag == value (written by another CTA).
+__device__ __forceinline__ bool flag_wait(const unsigned *flag, unsigned value,
+                                          volatile int *abort_flag, unsigned *status) {
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(flag) != value) {
+        if (*abort_flag) return false;
+        if (clock64() - t0 > TFA_WAIT_LIMIT_CYCLES) {
+            *abort_flag = 1;
+            atomicOr(status, TFA_DEVICE_TIMEOUT);
+            return false;
+        }
+        __nanosleep(100);
+    }
+    return true;
+}
 
 // Per-warpgroup register budget (all four warps of the warpgroup execute it).
 template <int N>

@@ -73,13 +73,17 @@ SMALL = [
 ]
 
 
+SCHEDULES = {"chosen": 0, "split": tb.TFA_DEBUG_FORCE_SPLIT, "whole": tb.TFA_DEBUG_NO_SPLIT}
+
+
+@pytest.mark.parametrize("schedule", sorted(SCHEDULES))
 @pytest.mark.parametrize("name,w", SMALL, ids=[n for n, _ in SMALL])
-def test_parity_small(name, w):
-    o, (q, k, v, km) = _run(w, seed=1)
+def test_parity_small(name, w, schedule):
+    o, (q, k, v, km) = _run(w, seed=1, flags=SCHEDULES[schedule])
     ref = oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
                            key_mask=km)
     err = _assert_close(o, ref, name)
-    print(f"{name}: max abs err {err:.3e}")
+    print(f"{name} [{schedule}]: max abs err {err:.3e}")
 
 
 def test_fully_masked_rows_are_exact_zeros():
@@ -194,3 +198,24 @@ def test_parity_full_size_sampled(name):
     of = o.float()
     assert torch.isfinite(of).all().item()
     print(f"{name}: {rows.size} sampled rows, max abs err {err:.3e}")
+
+
+@pytest.mark.parametrize("w", [
+    shaped(1, 1, 1, 256, 65536, 128, name="one_item_over_every_cta"),
+    shaped(1, 2, 1, 300, 40000, 64, window=30000, key_mask_keep=0.95, name="split_d64_window_mask"),
+    shaped(2, 4, 2, 1000, 5000, 128, causal=False, k_scale=4.0, name="split_bidirectional"),
+], ids=lambda w: w.name)
+def test_split_key_ranges_merge_exactly(w):
+    """Query tiles whose key range is cut across CTAs and merged (online-softmax
+    merge of partial max/sum/accumulator) against the oracle, and against the
+    whole-item schedule that never cuts."""
+    o, (q, k, v, km) = _run(w, seed=9, flags=tb.TFA_DEBUG_FORCE_SPLIT)
+    o_whole, _ = _run(w, inputs=(q, k, v, km), flags=tb.TFA_DEBUG_NO_SPLIT)
+    rows = _sample_rows(w, n_per_head=min(w.L, 64))
+    ref = oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                           key_mask=km, rows=rows)
+    idx = torch.as_tensor(rows, device=o.device)
+    _assert_close(o.reshape(-1, w.D)[idx], ref, w.name + " split")
+    _assert_close(o_whole.reshape(-1, w.D)[idx], ref, w.name + " whole items")
+    _assert_close(o.float().cpu().double().numpy(), o_whole.float().cpu().double().numpy(),
+                  w.name + " split vs whole")
