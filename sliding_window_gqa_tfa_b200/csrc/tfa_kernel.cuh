@@ -71,8 +71,8 @@ constexpr int kThreads = 384;
 // warpgroups grow to kRegsSoftmax; 2*128*kRegsSoftmax + 128*kRegsOther must not
 // exceed 384*kRegsLaunch, or setmaxnreg.inc would wait forever.
 constexpr int kRegsLaunch = 168;
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsOther = 88;
+constexpr int kRegsSoftmax = 200;
+constexpr int kRegsOther = 104;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunch,
               "register split exceeds the launch pool");
 // Lazy rescale: keep the stale row maximum until the true one exceeds it by
@@ -88,6 +88,10 @@ constexpr float kRescaleThresholdLog2 = 8.0f;
 #define TFA_POLY_PERIOD 0
 #endif
 constexpr int kPolyPeriod = TFA_POLY_PERIOD;
+// The softmax publishes P in two parts: keys [0, kPartKeys) first, so the P.V
+// product runs on them while the last keys' exponentials are computed.
+constexpr int kPartKeys = 96;
+static_assert(kPartKeys % 32 == 0 && kPartKeys % 16 == 0 && kPartKeys < 128, "P split");
 
 template <int D>
 struct Cfg {
@@ -99,7 +103,7 @@ struct Cfg {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
     static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-    static constexpr int kNumBars = 10 + 2 * kSlots + 1 + 4;
+    static constexpr int kNumBars = 10 + 2 * kSlots + 1 + 4 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
     static constexpr uint32_t kTmemCols = 512;
@@ -170,6 +174,9 @@ struct Bars {
     // finalizer thread saw every contributor's flag
     __device__ __forceinline__ uint32_t pub(int t) const { return base + 8 * (11 + 2 * slots + t); }
     __device__ __forceinline__ uint32_t fin(int t) const { return base + 8 * (13 + 2 * slots + t); }
+    // P_t's first kPartKeys key columns are in tensor memory (the P.V product
+    // may start on them while the softmax finishes the rest)
+    __device__ __forceinline__ uint32_t p_part(int t) const { return base + 8 * (15 + 2 * slots + t); }
 };
 
 // ------------------------------------------------------------------ producer
@@ -249,10 +256,9 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     // O_t += P_t V: A = P_t in tensor memory (8 columns per 16 keys), B = V tile
     // read MN-major (D contiguous): 8 key rows per 1 KB swizzle atom (SBO), the
     // next 64 head-dim columns one column block further (LBO).
-    auto issue_pv = [&](int t, uint32_t slot, bool accumulate) {
+    auto issue_pv = [&](int t, uint32_t slot, bool accumulate, int kk_begin, int kk_end) {
         const uint32_t va = kv_smem + slot * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBlockK / 16; ++kk) {
+        for (int kk = kk_begin; kk < kk_end; ++kk) {
             umma_ts(tmem + C::kTmemO + t * D, tmem + C::kTmemS + t * 128 + C::kTmemP + kk * 8,
                     smem_desc_sw128(va + kk * 16 * 128, C::kColBlockBytes, 1024), kIdescPV,
                     (accumulate || kk > 0) ? 1u : 0u);
@@ -310,11 +316,16 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
             for (int t = 0; t < 2; ++t) {
                 if (!ip.present[t]) continue;
                 if (ip.lo[t] <= j && j <= ip.hi[t]) {
-                    if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                    // first part of P_t, then the rest (the tensor core works on
+                    // the first part meanwhile)
+                    if (!mbar_wait(bar.p_part(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
                     TFA_TR(2, trace_step, 2 + 2 * t);
+                    tc_fence_after();
+                    issue_pv(t, sv, acc[t], 0, kPartKeys / 16);
+                    if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
                     ++p_cnt[t];
                     tc_fence_after();
-                    issue_pv(t, sv, acc[t]);
+                    issue_pv(t, sv, true, kPartKeys / 16, kBlockK / 16);
                     acc[t] = true;
                     if (j == ip.hi[t]) umma_commit(bar.o_full(t));
                 }
@@ -438,41 +449,56 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
                 }
             }
 
+            // O_t must be rescaled before any of P_t is published: the P.V
+            // product may start as soon as the first part is.
+            if (rescale) {  // rare; 8 columns at a time while the scores are live
+                for (int cc = 0; cc < D / 8; ++cc) {
+                    uint32_t o[8];
+                    tmem_ld8(tO + cc * 8, o);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st8(tO + cc * 8, o);
+                }
+            }
+
             const float mc = (m_ref == -CUDART_INF_F) ? 0.f : m_ref * c;
             const float2 c2 = make_float2(c, c), nmc2 = make_float2(-mc, -mc);
             float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
             uint32_t pk[64];
+#define TFA_EXP_PAIR(i)                                                                    \
+    do {                                                                                   \
+        const float2 x = fma2(make_float2(TFA_F(2 * (i)), TFA_F(2 * (i) + 1)), c2, nmc2);  \
+        float2 e;                                                                          \
+        if (kPolyPeriod > 0 && ((i) % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) { \
+            e = exp2_poly2(x); /* FMA pipe */                                              \
+        } else {                                                                           \
+            e.x = ex2(x.x); /* MUFU */                                                     \
+            e.y = ex2(x.y);                                                                \
+        }                                                                                  \
+        if ((i) & 1)                                                                       \
+            acc1 = add2(acc1, e);                                                          \
+        else                                                                               \
+            acc0 = add2(acc0, e);                                                          \
+        pk[i] = pack_bf16(e.x, e.y);                                                       \
+    } while (0)
+            // keys [0, kPartKeys): publish, then the rest
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
-                const float2 x = fma2(make_float2(TFA_F(2 * i), TFA_F(2 * i + 1)), c2, nmc2);
-                float2 e;
-                if (kPolyPeriod > 0 && (i % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) {
-                    e = exp2_poly2(x);  // FMA pipe
-                } else {
-                    e.x = ex2(x.x);  // MUFU
-                    e.y = ex2(x.y);
-                }
-                if (i & 1)
-                    acc1 = add2(acc1, e);
-                else
-                    acc0 = add2(acc0, e);
-                pk[i] = pack_bf16(e.x, e.y);
-            }
+            for (int i = 0; i < kPartKeys / 2; ++i) TFA_EXP_PAIR(i);
+#pragma unroll
+            for (int c32 = 0; c32 < kPartKeys / 64; ++c32) tmem_st32(tP + 32 * c32, pk + 32 * c32);
+            if ((kPartKeys / 2) % 32) tmem_st16(tP + (kPartKeys / 64) * 32, pk + (kPartKeys / 64) * 32);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.p_part(t));
+#pragma unroll
+            for (int i = kPartKeys / 2; i < 64; ++i) TFA_EXP_PAIR(i);
+#undef TFA_EXP_PAIR
 #undef TFA_F
             const float2 acc = add2(acc0, acc1);
             l = l * alpha + (acc.x + acc.y);
-            tmem_st32(tP, pk);
-            tmem_st32(tP + 32, pk + 32);
-            if (rescale) {
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + cc * 32, o);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                    tmem_st32(tO + cc * 32, o);
-                }
-            }
+            for (int c16 = kPartKeys / 32; c16 < 4; ++c16) tmem_st16(tP + 16 * c16, pk + 16 * c16);
             if (r == 0) TFA_TR(t, trace_step, 3);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 2);
             tmem_wait_st();
@@ -619,6 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t) {
             mbar_init(bar.pub(t), 4);
             mbar_init(bar.fin(t), 1);
+            mbar_init(bar.p_part(t), 4);
         }
         *abort_flag = 0;
         fence_barrier_init();
