@@ -166,8 +166,8 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     auto kern = tfa::tfa_prefill_kernel<D>;
     const int which = D == 128 ? 1 : 0;
     if (!st.smem_attr[which]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytesKeyMask);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
         cudaFuncAttributes fa;
         if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess)
@@ -227,7 +227,8 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
         if (++ss->epoch == 0) ++ss->epoch;  // 0 is the flags' initial value
         p.epoch = ss->epoch;
     }
-    kern<<<grid, tfa::kThreads, C::kSmemBytes, stream>>>(mq, mk, mv, p);
+    const int smem = key_mask ? C::kSmemBytesKeyMask : C::kSmemBytes;
+    kern<<<grid, tfa::kThreads, smem, stream>>>(mq, mk, mv, p);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFA_OK : cuda_fail("kernel launch", e);
 }

@@ -102,10 +102,20 @@ struct Cfg {
     static constexpr int kSlots = (D == 128) ? 4 : 8;     // K/V ring depth
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kTileBytes;
+    // Key-mask bias: per K/V slot a [128 keys][16] bf16 block whose column 0
+    // is 0 (key kept) or -inf (key dropped), and one [128 rows][16] block of
+    // "ones" (column 0 = 1); one extra K=16 MMA adds bias[key] to every row of
+    // S.  Both blocks are K-major without swizzle (see bias_offset).
+    // They sit at the end of the layout: launches without a key mask do not
+    // request that shared memory at all (it would shrink the L1 carve-out).
+    static constexpr int kBiasBytes = 128 * 16 * 2;
     static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
     static constexpr int kNumBars = 10 + 2 * kSlots + 1 + 4 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
+    static constexpr int kBiasOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
+    static constexpr int kOnesOff = kBiasOff + kSlots * kBiasBytes;
+    static constexpr int kSmemBytesKeyMask = kOnesOff + kBiasBytes + 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kTmemS = 0;                 // S_t at kTmemS + 128 t
     static constexpr uint32_t kTmemO = 256;               // O_t at kTmemO + D t
@@ -126,6 +136,13 @@ struct Params {
     long long W;       // total key-tile steps (split schedule)
     Shape shape;
 };
+
+// Byte offset of element (row, k) of a [128][16] bf16 K-major block without
+// swizzle: core matrices of 8 rows x 16 bytes; the two halves of k 128 bytes
+// apart (LBO), consecutive 8-row groups 256 bytes apart (SBO).
+__host__ __device__ constexpr uint32_t bias_offset(int row, int k) {
+    return (row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
+}
 
 // Floats of one partial slot: the accumulator [128][D], then m[128], l[128].
 template <int D>
@@ -182,9 +199,15 @@ struct Bars {
 // ------------------------------------------------------------------ producer
 template <int D>
 __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                          const CUtensorMap *tm_v, uint32_t sbase, const Bars &bar,
+                          const CUtensorMap *tm_v, uint32_t sbase, uint8_t *gbase, const Bars &bar,
                           volatile int *abort_flag) {
+    // With a key mask the whole warp runs this loop (lane 0 issues the copies
+    // and arms the barriers, all lanes write each K tile's bias); without one
+    // only lane 0 does.
     using C = Cfg<D>;
+    const int lane = threadIdx.x & 31;
+    const bool has_km = p.key_mask != nullptr;
+    const unsigned lanes = has_km ? 0xffffffffu : 1u;
     uint32_t kv_prod = 0;
     uint32_t q_use[2] = {0, 0};
     SegIter it;
@@ -195,31 +218,52 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (!ip.present[t]) continue;
-            if (q_use[t] > 0 && !mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status))
+            if (q_use[t] > 0 &&
+                !__all_sync(lanes, mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status)))
                 goto out;
-            mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
-            for (int cb = 0; cb < C::kColBlocks; ++cb)
-                tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes, tm_q,
-                            bar.q_full(t), cb * 64, ip.q0[t], ip.b * p.Hq + ip.h);
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
+                for (int cb = 0; cb < C::kColBlocks; ++cb)
+                    tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes, tm_q,
+                                bar.q_full(t), cb * 64, ip.q0[t], ip.b * p.Hq + ip.h);
+            }
             ++q_use[t];
         }
         for (int j = ip.jl; j <= ip.jh; ++j) {
             for (int which = 0; which < 2; ++which) {  // K_j then V_j
                 const uint32_t s = kv_prod % C::kSlots;
                 const uint32_t round = kv_prod / C::kSlots;
-                if (round > 0 && !mbar_wait(bar.kv_empty(s), (round - 1) & 1, abort_flag, p.status))
+                if (round > 0 &&
+                    !__all_sync(lanes, mbar_wait(bar.kv_empty(s), (round - 1) & 1, abort_flag, p.status)))
                     goto out;
-                mbar_arrive_expect_tx(bar.kv_full(s), C::kTileBytes);
-                for (int cb = 0; cb < C::kColBlocks; ++cb)
-                    tma_load_3d(sbase + C::kKVOff + s * C::kTileBytes + cb * C::kColBlockBytes,
-                                which ? tm_v : tm_k, bar.kv_full(s), cb * 64, j * kBlockK,
-                                ip.b * p.Hkv + ip.g);
+                if (which == 0 && has_km) {
+                    // bias column of this K tile: 0 for kept keys, -inf otherwise
+                    const float *km_row = p.key_mask + static_cast<size_t>(ip.b) * p.S;
+                    uint8_t *blk = gbase + C::kBiasOff + s * C::kBiasBytes;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int n = 32 * i + lane;
+                        const int key = j * kBlockK + n;
+                        const bool keep = key < p.S && __ldg(km_row + key) > 0.5f;
+                        *reinterpret_cast<uint16_t *>(blk + bias_offset(n, 0)) = keep ? 0x0000u : 0xFF80u;
+                    }
+                    fence_proxy_async_smem();  // the tensor core reads it through the async proxy
+                    __syncwarp();
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(bar.kv_full(s), C::kTileBytes);
+                    for (int cb = 0; cb < C::kColBlocks; ++cb)
+                        tma_load_3d(sbase + C::kKVOff + s * C::kTileBytes + cb * C::kColBlockBytes,
+                                    which ? tm_v : tm_k, bar.kv_full(s), cb * 64, j * kBlockK,
+                                    ip.b * p.Hkv + ip.g);
+                }
                 ++kv_prod;
             }
         }
     }
 out:
-    // Every copy this thread started must land before the CTA may exit.
+    if (lane != 0) return;
+    // Every copy lane 0 started must land before the CTA may exit.
     for (uint32_t s = 0; s < (uint32_t)C::kSlots; ++s) {
         if (kv_prod > s) {
             const uint32_t armed = (kv_prod - s - 1) / C::kSlots + 1;
@@ -239,6 +283,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);        // O += P V, V MN-major
     const uint32_t q_smem = sbase + C::kQOff;
     const uint32_t kv_smem = sbase + C::kKVOff;
+    const bool has_km = p.key_mask != nullptr;
 
     // S_t = Q_t K^T: A = Q tile, B = K tile, both [128 rows][D] K-major with
     // 128-byte swizzle; a K-step of 16 elements advances 32 bytes inside a
@@ -252,6 +297,10 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
             umma_ss(tmem + C::kTmemS + t * 128, smem_desc_sw128(qa + off, 16, 1024),
                     smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
         }
+        if (has_km)  // S += ones * bias^T: the key mask as a per-column 0 / -inf
+            umma_ss(tmem + C::kTmemS + t * 128, smem_desc_noswizzle(sbase + C::kOnesOff, 128, 256),
+                    smem_desc_noswizzle(sbase + C::kBiasOff + slot * C::kBiasBytes, 128, 256),
+                    kIdescQK, 1u);
     };
     // O_t += P_t V: A = P_t in tensor memory (8 columns per 16 keys), B = V tile
     // read MN-major (D contiguous): 8 key rows per 1 KB swizzle atom (SBO), the
@@ -358,7 +407,6 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     const uint32_t tP = tS + C::kTmemP;
     const uint32_t tO = tmem + C::kTmemO + t * D + lane_base;
     const float c = p.scale_log2;
-    const bool has_km = p.key_mask != nullptr;
     const int lane = threadIdx.x & 31;
     uint32_t s_cnt = 0, o_cnt = 0, pub_cnt = 0, fin_cnt = 0;
     int trace_step = 0;
@@ -375,23 +423,12 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         const int pos = (p.S - p.L) + row;  // absolute position of this query row
         const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
         const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
-        const float *km_row = has_km ? p.key_mask + static_cast<size_t>(seg.b) * p.S : nullptr;
         float m_ref = -CUDART_INF_F;  // row maximum the exponentials are taken against
         float l = 0.f;
         bool first = true;
 
         for (int j = ip.lo; j <= ip.hi; ++j) {
             if (r == 0) TFA_TR(t, trace_step, 0);
-            // key-mask values of this key tile, fetched before the wait so the
-            // load latency hides behind it (lane i holds columns i, i+32, ...)
-            float kmv[4] = {1.f, 1.f, 1.f, 1.f};
-            if (has_km) {
-#pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    const int col = j * kBlockK + 32 * w + lane;
-                    kmv[w] = col < p.S ? __ldg(km_row + col) : 0.f;
-                }
-            }
             // all lanes leave together: the tcgen05 loads below are warp-collective
             if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(t), s_cnt & 1, abort_flag, p.status)))
                 return;
@@ -403,16 +440,15 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (r == 0) TFA_TR(t, trace_step, 2);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 0);
 
-            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, has_km, row - r, j, p.flags)) {
+            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, 0, row - r, j, p.flags)) {
                 const int k0 = j * kBlockK;
                 const int lo_c = lo_abs - k0;
                 const int hi_c = hi_abs - k0;
-                uint32_t kmw[4];
-#pragma unroll
-                for (int w = 0; w < 4; ++w) kmw[w] = __ballot_sync(0xffffffffu, kmv[w] > 0.5f);
 #pragma unroll
                 for (int cidx = 0; cidx < 128; ++cidx) {
-                    const bool keep = cidx >= lo_c && cidx <= hi_c && ((kmw[cidx >> 5] >> (cidx & 31)) & 1u);
+                    // causal / window / key-tail predicate; the key mask arrived
+                    // through the bias MMA already
+                    const bool keep = cidx >= lo_c && cidx <= hi_c;
                     if (!keep) s[cidx] = 0xff800000u;  // -inf
                 }
             }
@@ -654,6 +690,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
+    if (warp == 8 && p.key_mask != nullptr) {
+        // ones block (column 0 = 1.0) and all-zero bias blocks; the load warp
+        // later rewrites only the bias blocks' column 0
+        uint32_t *z = reinterpret_cast<uint32_t *>(gbase + C::kBiasOff);
+        for (int i = lane; i < (C::kSlots + 1) * C::kBiasBytes / 4; i += 32) z[i] = 0u;
+        __syncwarp();
+        for (int n = lane; n < 128; n += 32)
+            *reinterpret_cast<uint16_t *>(gbase + C::kOnesOff + bias_offset(n, 0)) = 0x3F80u;
+        fence_proxy_async_smem();
+    }
     if (warp == 8 && lane == 0) {
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -672,7 +718,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         softmax_role<D>(p, warp >> 2, tmem, bar, abort_flag);
     } else {
         reg_dealloc<kRegsOther>();
-        if (warp == 8 && lane == 0) load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, bar, abort_flag);
+        if (warp == 8 && (lane == 0 || p.key_mask != nullptr))
+            load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
         if (warp == 9 && lane == 0) mma_role<D>(p, sbase, tmem, bar, abort_flag);
     }
 
