@@ -37,7 +37,7 @@ struct DeviceState {
     bool init = false;
     int sm_count = 0;
     unsigned *status = nullptr;  // device status word (TFA_DEVICE_TIMEOUT bits)
-    bool smem_attr[2] = {false, false};
+    bool smem_attr[4] = {false, false, false, false};
     std::unordered_map<cudaStream_t, SplitScratch> split;
     // staging buffers of tfa_prefill_host
     void *h_buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -163,11 +163,13 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     if (encode_map(&mq, q, L, B * Hq, D) || encode_map(&mk, k, S, B * Hkv, D) ||
         encode_map(&mv, v, S, B * Hkv, D))
         return TFA_ERR_CUDA;
-    auto kern = tfa::tfa_prefill_kernel<D>;
-    const int which = D == 128 ? 1 : 0;
+    // separate instantiations with and without a key mask (the mask costs an
+    // extra MMA per score tile and extra shared memory; unmasked calls carry neither)
+    auto kern = key_mask ? tfa::tfa_prefill_kernel<D, true> : tfa::tfa_prefill_kernel<D, false>;
+    const int smem = key_mask ? C::kSmemBytesKeyMask : C::kSmemBytes;
+    const int which = (D == 128 ? 2 : 0) + (key_mask ? 1 : 0);
     if (!st.smem_attr[which]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::kSmemBytesKeyMask);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
         cudaFuncAttributes fa;
         if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess)
@@ -227,7 +229,6 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
         if (++ss->epoch == 0) ++ss->epoch;  // 0 is the flags' initial value
         p.epoch = ss->epoch;
     }
-    const int smem = key_mask ? C::kSmemBytesKeyMask : C::kSmemBytes;
     kern<<<grid, tfa::kThreads, smem, stream>>>(mq, mk, mv, p);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFA_OK : cuda_fail("kernel launch", e);

@@ -197,7 +197,7 @@ struct Bars {
 };
 
 // ------------------------------------------------------------------ producer
-template <int D>
+template <int D, bool KM>
 __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                           const CUtensorMap *tm_v, uint32_t sbase, uint8_t *gbase, const Bars &bar,
                           volatile int *abort_flag) {
@@ -206,8 +206,8 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
     // only lane 0 does.
     using C = Cfg<D>;
     const int lane = threadIdx.x & 31;
-    const bool has_km = p.key_mask != nullptr;
-    const unsigned lanes = has_km ? 0xffffffffu : 1u;
+    constexpr bool has_km = KM;
+    constexpr unsigned lanes = KM ? 0xffffffffu : 1u;
     uint32_t kv_prod = 0;
     uint32_t q_use[2] = {0, 0};
     SegIter it;
@@ -275,7 +275,7 @@ out:
 }
 
 // ------------------------------------------------------------ tensor cores
-template <int D>
+template <int D, bool KM>
 __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const Bars &bar,
                          volatile int *abort_flag) {
     using C = Cfg<D>;
@@ -283,7 +283,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 1);        // O += P V, V MN-major
     const uint32_t q_smem = sbase + C::kQOff;
     const uint32_t kv_smem = sbase + C::kKVOff;
-    const bool has_km = p.key_mask != nullptr;
+    constexpr bool has_km = KM;
 
     // S_t = Q_t K^T: A = Q tile, B = K tile, both [128 rows][D] K-major with
     // 128-byte swizzle; a K-step of 16 elements advances 32 bytes inside a
@@ -297,7 +297,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
             umma_ss(tmem + C::kTmemS + t * 128, smem_desc_sw128(qa + off, 16, 1024),
                     smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
         }
-        if (has_km)  // S += ones * bias^T: the key mask as a per-column 0 / -inf
+        if constexpr (has_km)  // S += ones * bias^T: the key mask as a per-column 0 / -inf
             umma_ss(tmem + C::kTmemS + t * 128, smem_desc_noswizzle(sbase + C::kOnesOff, 128, 256),
                     smem_desc_noswizzle(sbase + C::kBiasOff + slot * C::kBiasBytes, 128, 256),
                     kIdescQK, 1u);
@@ -649,7 +649,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D>
+template <int D, bool KM>
 __global__ void __launch_bounds__(kThreads, 1)
     tfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -690,7 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 8 && p.key_mask != nullptr) {
+    if (KM && warp == 8) {
         // ones block (column 0 = 1.0) and all-zero bias blocks; the load warp
         // later rewrites only the bias blocks' column 0
         uint32_t *z = reinterpret_cast<uint32_t *>(gbase + C::kBiasOff);
@@ -718,9 +718,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         softmax_role<D>(p, warp >> 2, tmem, bar, abort_flag);
     } else {
         reg_dealloc<kRegsOther>();
-        if (warp == 8 && (lane == 0 || p.key_mask != nullptr))
-            load_role<D>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
-        if (warp == 9 && lane == 0) mma_role<D>(p, sbase, tmem, bar, abort_flag);
+        if (warp == 8 && (lane == 0 || KM))
+            load_role<D, KM>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
+        if (warp == 9 && lane == 0) mma_role<D, KM>(p, sbase, tmem, bar, abort_flag);
     }
 
     tc_fence_before();
