@@ -285,33 +285,43 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     const uint32_t kv_smem = sbase + C::kKVOff;
     constexpr bool has_km = KM;
 
+    // Descriptors are built once: the start-address field holds address >> 4
+    // in its low 14 bits, so moving an operand by `off` bytes (shared memory
+    // stays below 256 KB) adds off >> 4 to the 64-bit descriptor.
     // S_t = Q_t K^T: A = Q tile, B = K tile, both [128 rows][D] K-major with
     // 128-byte swizzle; a K-step of 16 elements advances 32 bytes inside a
     // 128-byte row and moves to the next column block every 4 steps.
-    auto issue_qk = [&](int t, uint32_t slot) {
-        const uint32_t qa = q_smem + t * C::kTileBytes;
-        const uint32_t ka = kv_smem + slot * C::kTileBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::kColBlockBytes + (kk & 3) * 32;
-            umma_ss(tmem + C::kTmemS + t * 128, smem_desc_sw128(qa + off, 16, 1024),
-                    smem_desc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        if constexpr (has_km)  // S += ones * bias^T: the key mask as a per-column 0 / -inf
-            umma_ss(tmem + C::kTmemS + t * 128, smem_desc_noswizzle(sbase + C::kOnesOff, 128, 256),
-                    smem_desc_noswizzle(sbase + C::kBiasOff + slot * C::kBiasBytes, 128, 256),
-                    kIdescQK, 1u);
-    };
+    const uint64_t dq0 = smem_desc_sw128(q_smem, 16, 1024);
+    const uint64_t dkv0 = smem_desc_sw128(kv_smem, 16, 1024);
     // O_t += P_t V: A = P_t in tensor memory (8 columns per 16 keys), B = V tile
     // read MN-major (D contiguous): 8 key rows per 1 KB swizzle atom (SBO), the
     // next 64 head-dim columns one column block further (LBO).
-    auto issue_pv = [&](int t, uint32_t slot, bool accumulate, int kk_begin, int kk_end) {
-        const uint32_t va = kv_smem + slot * C::kTileBytes;
-        for (int kk = kk_begin; kk < kk_end; ++kk) {
-            umma_ts(tmem + C::kTmemO + t * D, tmem + C::kTmemS + t * 128 + C::kTmemP + kk * 8,
-                    smem_desc_sw128(va + kk * 16 * 128, C::kColBlockBytes, 1024), kIdescPV,
-                    (accumulate || kk > 0) ? 1u : 0u);
+    const uint64_t dv0 = smem_desc_sw128(kv_smem, C::kColBlockBytes, 1024);
+    uint64_t d_ones = 0, d_bias0 = 0;
+    if constexpr (KM) {
+        d_ones = smem_desc_noswizzle(sbase + C::kOnesOff, 128, 256);
+        d_bias0 = smem_desc_noswizzle(sbase + C::kBiasOff, 128, 256);
+    }
+    constexpr uint32_t kTileStep = C::kTileBytes >> 4;
+    auto issue_qk = [&](int t, uint32_t slot) {
+        const uint64_t dq = dq0 + t * kTileStep;
+        const uint64_t dk = dkv0 + slot * kTileStep;
+        const uint32_t d_tmem = tmem + C::kTmemS + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4;
+            umma_ss(d_tmem, dq + off, dk + off, kIdescQK, kk > 0 ? 1u : 0u);
         }
+        if constexpr (has_km)  // S += ones * bias^T: the key mask as a per-column 0 / -inf
+            umma_ss(d_tmem, d_ones, d_bias0 + slot * (C::kBiasBytes >> 4), kIdescQK, 1u);
+    };
+    auto issue_pv = [&](int t, uint32_t slot, bool accumulate, int kk_begin, int kk_end) {
+        const uint64_t dv = dv0 + slot * kTileStep;
+        const uint32_t d_tmem = tmem + C::kTmemO + t * D;
+        const uint32_t a_tmem = tmem + C::kTmemS + t * 128 + C::kTmemP;
+        for (int kk = kk_begin; kk < kk_end; ++kk)
+            umma_ts(d_tmem, a_tmem + kk * 8, dv + kk * ((16 * 128) >> 4), kIdescPV,
+                    (accumulate || kk > 0) ? 1u : 0u);
     };
 
     uint32_t kv_cons = 0;
@@ -455,16 +465,16 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 
             // row maximum: three-input max in four independent chains
 #define TFA_F(i) __uint_as_float(s[i])
-            float mx0 = fmaxf(TFA_F(0), TFA_F(4)), mx1 = fmaxf(TFA_F(1), TFA_F(5));
-            float mx2 = fmaxf(TFA_F(2), TFA_F(6)), mx3 = fmaxf(TFA_F(3), TFA_F(7));
+            float mx[8];
 #pragma unroll
-            for (int i = 8; i < 128; i += 8) {
-                mx0 = fmax3(mx0, TFA_F(i), TFA_F(i + 4));
-                mx1 = fmax3(mx1, TFA_F(i + 1), TFA_F(i + 5));
-                mx2 = fmax3(mx2, TFA_F(i + 2), TFA_F(i + 6));
-                mx3 = fmax3(mx3, TFA_F(i + 3), TFA_F(i + 7));
+            for (int k = 0; k < 8; ++k) mx[k] = fmaxf(TFA_F(k), TFA_F(k + 8));
+#pragma unroll
+            for (int i = 16; i < 128; i += 16) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], TFA_F(i + k), TFA_F(i + k + 8));
             }
-            const float m_new = fmax3(m_ref, fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+            const float m_new = fmax3(m_ref, fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                                   fmaxf(mx[6], mx[7])), -CUDART_INF_F);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 1);
 
             // Decide the lazy rescale first; O_t itself is rescaled after P is
