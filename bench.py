@@ -3,7 +3,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one tfa_prefill launch over the whole workload (every query row of
+One step = one launch (tfa_prefill; tfa_decode when L <= 8) over the whole workload (every query row of
 every head).  Inputs are seeded synthetic bf16 tensors resident in HBM before
 the timed region; L2 is flushed (256 MiB memset) between steps, outside each
 step's CUDA events.  Prints one JSON line on rank 0.
@@ -325,8 +325,18 @@ def main():
     d2h = hout.numel() * 2
 
     peaks, peak_kind = load_peaks()
-    peak = float(peaks["bf16_tflops"])
-    achieved = flops / (mean_ms * 1e-3) / 1e12  # per GPU, per launch
+    alg_bytes = algorithmic_bytes(w.B, w.Hq, w.Hkv, w.L, w.S, w.D, key_mask=km is not None)
+    if w.L <= tb.MAX_DECODE_ROWS:
+        # short queries read every K/V byte for a few flops: bounded by HBM
+        bound, roof_unit = "hbm", "GB/s"
+        peak = float(peaks["hbm_gbs"])
+        achieved = alg_bytes / (mean_ms * 1e-3) / 1e9
+        peak_source = f"{peak_kind} hbm_gbs (copy bandwidth)"
+    else:
+        bound, roof_unit = "tensor", "TFLOP/s"
+        peak = float(peaks["bf16_tflops"])
+        achieved = flops / (mean_ms * 1e-3) / 1e12  # per GPU, per launch
+        peak_source = f"{peak_kind} bf16_tflops (burst; kernel timed alone)"
     traffic = recorded_traffic(w.name)
     clocks = clk.summary()
     if rank == 0:
@@ -343,12 +353,11 @@ def main():
             "ms_p10": per_sorted[len(per) // 10], "ms_p50": per_sorted[len(per) // 2],
             "ms_p90": per_sorted[(9 * len(per)) // 10],
             "pct_of_peak": 100.0 * achieved / peak,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak,
-                         "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{peak_kind} bf16_tflops (burst; kernel timed alone)",
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": roof_unit, "frac": achieved / peak,
+                         "peak_source": peak_source,
                          "traffic": traffic,
-                         "algorithmic_bytes": algorithmic_bytes(w.B, w.Hq, w.Hkv, w.L, w.S, w.D,
-                                                                key_mask=km is not None)},
+                         "algorithmic_bytes": alg_bytes},
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "api": "tfa_prefill_host (pinned host buffers)"},

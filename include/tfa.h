@@ -86,6 +86,24 @@ int tfa_prefill(const void *q, const void *k, const void *v, void *o,
                 int B, int Hq, int Hkv, int L, int S, int D, float scale,
                 int causal, int window, const float *key_mask, tfa_stream_t stream);
 
+/* Longest query accepted by tfa_decode. */
+#define TFA_MAX_DECODE_ROWS 8
+
+/* tfa_decode -- the same attention for short queries: 1 <= L <= 8 new rows
+ * (L = 1 is token-by-token decoding), which tfa_prefill rejects.  Arguments,
+ * layouts, masks, ownership and errors are those of tfa_prefill, except that
+ * L must lie in [1, TFA_MAX_DECODE_ROWS] (else TFA_ERR_SHAPE).  The kernel
+ * packs the L rows of several query heads of one KV group into each
+ * 128-row tensor-core tile and spreads the key range of every KV group over
+ * all SMs, merging the pieces' softmax statistics exactly (the online-softmax
+ * merge of tiny-llm "Week 2 Day 5: Tiled Dense Prefill Attention", Task 1).
+ * The pages route such queries to a separate path (tiny-llm's readable
+ * fallback for L <= 8; mlx-lm's sdpa_vector for at most 8 rows; brotensor's
+ * flash_attention_decode for L_q == 1). */
+int tfa_decode(const void *q, const void *k, const void *v, void *o,
+               int B, int Hq, int Hkv, int L, int S, int D, float scale,
+               int causal, int window, const float *key_mask, tfa_stream_t stream);
+
 /* Debug flags for tfa_prefill_debug. */
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
 #define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */
@@ -106,7 +124,8 @@ int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o,
                       unsigned flags);
 
 /* tfa_prefill_host -- the same operation on HOST buffers (q, k, v, key_mask
- * read, o written; plain or pinned host memory).  The library copies the
+ * read, o written; plain or pinned host memory), for L >= 9 as tfa_prefill and
+ * for 1 <= L <= 8 as tfa_decode.  The library copies the
  * inputs to device staging buffers it owns (one set per device, grown on
  * demand and kept until process exit), runs tfa_prefill on `stream`, copies o
  * back and synchronizes the stream before returning.  Not safe to call from
@@ -152,7 +171,8 @@ const char *tfa_last_error(void);
 const char *tfa_status_string(int status);
 
 /* tfa_plan_qtile -- host view of the work enumeration the kernel performs for
- * one 128-row query tile (rows [128*qtile, min(128*qtile+128, L))):
+ * one 128-row query tile (rows [128*qtile, min(128*qtile+128, L))); for
+ * 1 <= L <= 8 (tfa_decode) tile 0 is the key range of every packed tile:
  *   *kt_lo, *kt_hi  first and last 128-key tile it visits (kt_hi < kt_lo: none)
  *   needs_mask      if not NULL, receives kt_hi-kt_lo+1 bytes: 1 where the tile
  *                   crosses the causal diagonal, the window edge, the key tail

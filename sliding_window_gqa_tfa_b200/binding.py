@@ -39,6 +39,7 @@ TFA_DEBUG_NO_SPLIT = 8
 TFA_DEBUG_FORCE_SPLIT = 16
 
 MIN_QUERY_ROWS = 9
+MAX_DECODE_ROWS = 8
 BLOCK_Q = 128
 BLOCK_K = 128
 
@@ -72,6 +73,8 @@ def lib():
             L.tfa_prefill_host.restype = i32
             L.tfa_prefill_noalloc.argtypes = common
             L.tfa_prefill_noalloc.restype = i32
+            L.tfa_decode.argtypes = common
+            L.tfa_decode.restype = i32
             L.tfa_check_status.argtypes = [P]
             L.tfa_check_status.restype = i32
             L.tfa_last_error.argtypes = []
@@ -118,6 +121,11 @@ def tfa_prefill_host(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key
                      stream) -> int:
     return lib().tfa_prefill_host(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window,
                                   key_mask, stream)
+
+
+def tfa_decode(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, stream) -> int:
+    return lib().tfa_decode(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                            stream)
 
 
 def tfa_prefill_noalloc(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
@@ -182,8 +190,8 @@ def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=No
             debug_flags=0):
     """Attention output [B,Hq,L,D] bf16 for bf16 q [B,Hq,L,D], k/v [B,Hkv,S,D] on one GPU.
 
-    key_mask: optional fp32 [B,S] (1 keep / 0 drop).  Raises TfaError on a
-    nonzero status from the library."""
+    L >= 9 goes to tfa_prefill, 1 <= L <= 8 to tfa_decode.  key_mask: optional
+    fp32 [B,S] (1 keep / 0 drop).  Raises TfaError on a nonzero status."""
     import torch
 
     _check(q, "q", torch.bfloat16, 4)
@@ -212,6 +220,13 @@ def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=No
             float(scale), int(bool(causal)), int(window),
             ctypes.c_void_p(key_mask.data_ptr()) if key_mask is not None else None,
             _stream_handle(stream))
+    if L <= MAX_DECODE_ROWS:
+        if debug_flags:
+            raise ValueError("debug flags apply to the prefill path only (L >= 9)")
+        rc = tfa_decode(*args)
+        if rc != TFA_OK:
+            raise TfaError(rc, "tfa_decode")
+        return out
     rc = tfa_prefill_debug(*args, debug_flags) if debug_flags else tfa_prefill(*args)
     if rc != TFA_OK:
         raise TfaError(rc)

@@ -117,10 +117,11 @@ int split_scratch(DeviceState &st, cudaStream_t stream, SplitScratch **out) {
 
 int validate(const void *q, const void *k, const void *v, const void *o, int B, int Hq, int Hkv,
              int L, int S, int D, float scale, int causal, int window, const float *key_mask,
-             bool check_pointers) {
+             bool check_pointers, bool decode = false) {
     if (check_pointers && (!q || !k || !v || !o)) return TFA_ERR_NULL;
     if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TFA_ERR_HEADS;
-    if (L < TFA_MIN_QUERY_ROWS) return TFA_ERR_SHORT_QUERY;
+    if (!decode && L < TFA_MIN_QUERY_ROWS) return TFA_ERR_SHORT_QUERY;
+    if (decode && (L < 1 || L > TFA_MAX_DECODE_ROWS)) return TFA_ERR_SHAPE;
     if (B < 1 || S < L) return TFA_ERR_SHAPE;
     // element counts and every index the kernel forms must stay in range
     const long long qrows = static_cast<long long>(B) * Hq * L;
@@ -141,12 +142,13 @@ int validate(const void *q, const void *k, const void *v, const void *o, int B, 
 
 // 3-D view [planes][rows][D] of a contiguous bf16 tensor, boxes of 128 rows x
 // 64 columns (128 bytes) with 128-byte swizzle; rows past the end read as 0.
-int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D) {
+int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D,
+               int box_rows = tfa::kBlockQ, int box_planes = 1) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(planes)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
                              static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(D) * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(tfa::kBlockQ), 1};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_planes)};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -157,11 +159,17 @@ int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D) {
 template <int D>
 int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o, int B, int Hq,
            int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
-           cudaStream_t stream, unsigned flags, SplitScratch *ss, bool force_split = false) {
+           cudaStream_t stream, unsigned flags, SplitScratch *ss, bool force_split = false,
+           bool packed = false) {
     using C = tfa::Cfg<D>;
+    // Short queries: a tile packs pack_heads query heads of one KV group, all L
+    // rows of each (pack_heads * L <= 128), loaded as one {64, L, pack_heads} box.
+    const int G = Hq / Hkv;
+    const int pack_heads = packed ? (G < tfa::kBlockQ / L ? G : tfa::kBlockQ / L) : 0;
+    const int pack_chunks = packed ? (G + pack_heads - 1) / pack_heads : 0;
     CUtensorMap mq, mk, mv;
-    if (encode_map(&mq, q, L, B * Hq, D) || encode_map(&mk, k, S, B * Hkv, D) ||
-        encode_map(&mv, v, S, B * Hkv, D))
+    if ((packed ? encode_map(&mq, q, L, B * Hq, D, L, pack_heads) : encode_map(&mq, q, L, B * Hq, D)) ||
+        encode_map(&mk, k, S, B * Hkv, D) || encode_map(&mv, v, S, B * Hkv, D))
         return TFA_ERR_CUDA;
     // separate instantiations with and without a key mask (the mask costs an
     // extra MMA per score tile and extra shared memory; unmasked calls carry neither)
@@ -199,16 +207,19 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.window = (causal && window > 0) ? window : 0;
     p.flags = flags;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.packed = packed ? 1 : 0;
+    p.pack_heads = pack_heads;
+    p.pack_chunks = pack_chunks;
     tfa::Shape &sh = p.shape;
     sh.B = B;
-    sh.Hq = Hq;
+    sh.Hq = packed ? Hkv * pack_chunks : Hq;  // one "virtual head" per packed tile
     sh.L = L;
     sh.S = S;
     sh.causal = p.causal;
     sh.window = p.window;
     sh.flags = flags;
     sh.n_qp = tfa::shape_n_qp(L);
-    const long long n_items = static_cast<long long>(B) * Hq * sh.n_qp;
+    const long long n_items = static_cast<long long>(B) * sh.Hq * sh.n_qp;
     p.W = tfa::total_steps(sh);
     // whole-item schedule, and the split one when scratch exists and the
     // estimate says it finishes sooner (few, large items per CTA)
@@ -277,6 +288,22 @@ extern "C" int tfa_prefill(const void *q, const void *k, const void *v, void *o,
                         reinterpret_cast<cudaStream_t>(stream), 0u);
 }
 
+extern "C" int tfa_decode(const void *q, const void *k, const void *v, void *o, int B, int Hq,
+                          int Hkv, int L, int S, int D, float scale, int causal, int window,
+                          const float *key_mask, tfa_stream_t stream) {
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true, true);
+    if (rc) return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    SplitScratch *ss = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st)) || (rc = split_scratch(*st, s, &ss))) return rc;
+    return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                    key_mask, s, 0u, ss, false, true)
+                      : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                   key_mask, s, 0u, ss, false, true);
+}
+
 extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o, int B,
                                  int Hq, int Hkv, int L, int S, int D, float scale, int causal,
                                  int window, const float *key_mask, tfa_stream_t stream,
@@ -290,7 +317,8 @@ extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, vo
 extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, void *o, int B,
                                 int Hq, int Hkv, int L, int S, int D, float scale, int causal,
                                 int window, const float *key_mask, tfa_stream_t stream) {
-    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
+    const bool decode = L >= 1 && L <= TFA_MAX_DECODE_ROWS;
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true, decode);
     if (rc) return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t qbytes = static_cast<size_t>(B) * Hq * L * D * 2;
@@ -313,9 +341,9 @@ extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, voi
     SplitScratch *ss = nullptr;
     if ((rc = split_scratch(*st, s, &ss))) return rc;
     rc = (D == 128) ? launch<128>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
-                                  Hkv, L, S, scale, causal, window, dmask, s, 0u, ss)
+                                  Hkv, L, S, scale, causal, window, dmask, s, 0u, ss, false, decode)
                     : launch<64>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
-                                 Hkv, L, S, scale, causal, window, dmask, s, 0u, ss);
+                                 Hkv, L, S, scale, causal, window, dmask, s, 0u, ss, false, decode);
     if (rc) return rc;
     if (cudaMemcpyAsync(o, st->h_buf[3], qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return TFA_ERR_CUDA;
@@ -421,7 +449,7 @@ extern "C" int tfa_trace_read(unsigned long long *host, size_t n) {
     cudaError_t e = cudaMemcpyFromSymbol(host, tfa::g_tfa_trace, bytes);
     return e == cudaSuccess ? TFA_OK : cuda_fail("cudaMemcpyFromSymbol(trace)", e);
 }
-// Trace builds only: per-CTA start / end global-timer stamps (1024 x 2).
+// Trace builds only: per-CTA global-timer stamps (1024 x 4: start, end, pieces done, spare).
 extern "C" int tfa_trace_cta_times(unsigned long long *host, size_t n) {
     const size_t bytes = sizeof(tfa::g_tfa_cta_time);
     if (n * sizeof(unsigned long long) < bytes) return TFA_ERR_SHAPE;
@@ -451,7 +479,7 @@ extern "C" const char *tfa_status_string(int status) {
 extern "C" int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_mask, int qtile,
                               int *kt_lo, int *kt_hi, unsigned char *needs_mask, int needs_mask_len) {
     int rc = validate(nullptr, nullptr, nullptr, nullptr, 1, 1, 1, L, S, 128, 1.0f, causal, window,
-                      nullptr, false);
+                      nullptr, false, L < TFA_MIN_QUERY_ROWS);
     if (rc) return rc;
     if (!kt_lo || !kt_hi) return TFA_ERR_NULL;
     const int q0 = qtile * tfa::kBlockQ;

@@ -52,7 +52,7 @@ namespace tfa {
 #ifdef TFA_TRACE
 constexpr int kTraceSlots = 2048;
 __device__ unsigned long long g_tfa_trace[8][kTraceSlots];
-__device__ unsigned long long g_tfa_cta_time[1024][2];  // global-timer ns at start / end
+__device__ unsigned long long g_tfa_cta_time[1024][4];  // global-timer ns: start, end, softmax done, spare
 #define TFA_TR(role, step, ev)                                                      \
     do {                                                                            \
         const int _i = 8 * (step) + (ev);                                           \
@@ -135,7 +135,24 @@ struct Params {
     float scale_log2;  // softmax scale * log2(e)
     long long W;       // total key-tile steps (split schedule)
     Shape shape;
+    // Short-query (decode) mapping: a query tile holds the rows of pack_heads
+    // query heads of one KV group, row m = (head m / L, query row m % L);
+    // shape.Hq then counts Hkv * pack_chunks "virtual heads", one per tile.
+    int packed, pack_heads, pack_chunks;
 };
+
+// Rows of one packed tile: first real query head, heads present.
+struct PackedRows {
+    int h0, heads;
+};
+__device__ __forceinline__ PackedRows packed_rows(const Params &p, int vh) {
+    const int g = vh / p.pack_chunks;
+    const int hc = vh - g * p.pack_chunks;
+    PackedRows pr;
+    pr.h0 = g * p.G + hc * p.pack_heads;
+    pr.heads = imin(p.pack_heads, p.G - hc * p.pack_heads);
+    return pr;
+}
 
 // Byte offset of element (row, k) of a [128][16] bf16 K-major block without
 // swizzle: core matrices of 8 rows x 16 bytes; the two halves of k 128 bytes
@@ -144,9 +161,11 @@ __host__ __device__ constexpr uint32_t bias_offset(int row, int k) {
     return (row >> 3) * 256 + (k >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2;
 }
 
-// Floats of one partial slot: the accumulator [128][D], then m[128], l[128].
+// Floats of one partial slot: the accumulator [128][D], then m[128], l[128];
+// one slot per (CTA, query tile) (only a CTA's first piece ever publishes).
 template <int D>
 __host__ __device__ constexpr int partial_slot_floats() { return 128 * D + 256; }
+__host__ __device__ constexpr int partial_slot(int cta, int t) { return cta * 2 + t; }
 
 struct ItemPlan {
     int b, h, g;
@@ -161,7 +180,7 @@ __device__ __forceinline__ ItemPlan plan_piece(const Params &p, const Segment &s
     ItemPlan ip;
     ip.b = seg.b;
     ip.h = seg.h;
-    ip.g = seg.h / p.G;
+    ip.g = p.packed ? seg.h / p.pack_chunks : seg.h / p.G;
     ip.jl = seg.jb;
     ip.jh = seg.je;
     const ItemSpan sp = item_span(p.shape, seg.qp);
@@ -222,10 +241,18 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                 !__all_sync(lanes, mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status)))
                 goto out;
             if (lane == 0) {
-                mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
-                for (int cb = 0; cb < C::kColBlocks; ++cb)
-                    tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes, tm_q,
-                                bar.q_full(t), cb * 64, ip.q0[t], ip.b * p.Hq + ip.h);
+                if (p.packed) {  // box {64, L, pack_heads}: rows (head, query row) in order
+                    const PackedRows pr = packed_rows(p, ip.h);
+                    mbar_arrive_expect_tx(bar.q_full(t), C::kColBlocks * 128 * p.L * p.pack_heads);
+                    for (int cb = 0; cb < C::kColBlocks; ++cb)
+                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
+                                    tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0);
+                } else {
+                    mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
+                    for (int cb = 0; cb < C::kColBlocks; ++cb)
+                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
+                                    tm_q, bar.q_full(t), cb * 64, ip.q0[t], ip.b * p.Hq + ip.h);
+                }
             }
             ++q_use[t];
         }
@@ -429,7 +456,17 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         const ItemSpan sp = item_span(p.shape, seg.qp);
         const TileRole ip = tile_role(p.shape, seg, sp, t);
         if (!ip.active) continue;
-        const int row = seg.qp * 2 * kBlockQ + t * kBlockQ + r;
+        // query row of this thread (its head too, for a packed tile)
+        int row = seg.qp * 2 * kBlockQ + t * kBlockQ + r;
+        int out_head = seg.h;
+        bool row_valid = row < p.L;
+        const int q_tile0 = row - r;  // first row of the tile, for the tile-level mask test
+        if (p.packed) {
+            const PackedRows pr = packed_rows(p, seg.h);
+            row = r % p.L;
+            out_head = pr.h0 + r / p.L;
+            row_valid = r < pr.heads * p.L;
+        }
         const int pos = (p.S - p.L) + row;  // absolute position of this query row
         const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
         const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
@@ -450,7 +487,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (r == 0) TFA_TR(t, trace_step, 2);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 0);
 
-            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, 0, row - r, j, p.flags)) {
+            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, 0, q_tile0, j, p.flags)) {
                 const int k0 = j * kBlockK;
                 const int lo_c = lo_abs - k0;
                 const int hi_c = hi_abs - k0;
@@ -560,34 +597,48 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         ++o_cnt;
         tc_fence_after();
 
+        // Rows of this tile that hold a query row: a packed tile fills
+        // heads * L of its 128 rows, a prefill tile ends at row L.
+        const int n_valid = p.packed ? packed_rows(p, seg.h).heads * p.L : imin(kBlockQ, p.L - q_tile0);
+        const bool warp_live = (r & ~31) < n_valid;  // warp-uniform: tcgen05.ld is warp-collective
+        const bool row_live = r < n_valid;
+
         if (!ip.complete && !ip.finalizer) {
-            // A later piece of this tile's key range: publish the partial
-            // (unscaled accumulator, row max, row sum) for the finalizer.
-            float *slot = p.partial + static_cast<size_t>(blockIdx.x * 2 + t) * partial_slot_floats<D>();
+            // A later piece of a cut tile: publish the partial (unscaled
+            // accumulator, row max, row sum) of the live rows for the finalizer.
+            float *slot = p.partial + static_cast<size_t>(partial_slot(blockIdx.x, t)) * partial_slot_floats<D>();
+            if (warp_live) {
 #pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t o[32];
-                tmem_ld32(tO + cc * 32, o);
-                float4 *dst = reinterpret_cast<float4 *>(slot + r * D + cc * 32);
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + cc * 32, o);
+                    float4 *dst = reinterpret_cast<float4 *>(slot + r * D + cc * 32);
+                    if (row_live) {
 #pragma unroll
-                for (int v4 = 0; v4 < 8; ++v4)
-                    __stcg(dst + v4, make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
-                                                 __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3])));
+                        for (int v4 = 0; v4 < 8; ++v4)
+                            __stcg(dst + v4,
+                                   make_float4(__uint_as_float(o[4 * v4]), __uint_as_float(o[4 * v4 + 1]),
+                                               __uint_as_float(o[4 * v4 + 2]), __uint_as_float(o[4 * v4 + 3])));
+                    }
+                }
+                if (row_live) {
+                    __stcg(slot + 128 * D + r, m_ref);
+                    __stcg(slot + 128 * D + 128 + r, l);
+                }
             }
-            __stcg(slot + 128 * D + r, m_ref);
-            __stcg(slot + 128 * D + 128 + r, l);
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.pub(t));
             if (r == 0 && mbar_wait(bar.pub(t), pub_cnt & 1, abort_flag, p.status)) {
                 __threadfence();
-                st_release_gpu(p.ready + blockIdx.x * 2 + t, p.epoch);
+                st_release_gpu(p.ready + partial_slot(blockIdx.x, t), p.epoch);
             }
             ++pub_cnt;
             continue;
         }
 
-        // Finalizer of a split tile: merge the partials of the CTAs that hold
-        // the rest of its key range (tiny-llm Week 2 Day 5, Task 1 merge).
+        // Finalizer of a cut tile: merge the partials of the CTAs that hold
+        // the rest of its key range (tiny-llm Week 2 Day 5, Task 1 merge:
+        // m* = max m_k, l* = sum e^(m_k - m*) l_k, a* = sum e^(m_k - m*) a_k).
         float f_own = 1.f, m_star = m_ref;
         int c_last = blockIdx.x;
         if (!ip.complete) {
@@ -595,42 +646,47 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (r == 0) {
                 bool ok = true;
                 for (int k = blockIdx.x + 1; k <= c_last && ok; ++k)
-                    ok = flag_wait(p.ready + k * 2 + t, p.epoch, abort_flag, p.status);
+                    ok = flag_wait(p.ready + partial_slot(k, t), p.epoch, abort_flag, p.status);
                 mbar_arrive(bar.fin(t));  // arrive even on failure; the abort flag tells
             }
             if (!__all_sync(0xffffffffu, mbar_wait(bar.fin(t), fin_cnt & 1, abort_flag, p.status)))
                 return;
             ++fin_cnt;
             if (*abort_flag) return;
-            for (int k = blockIdx.x + 1; k <= c_last; ++k) {
-                (void)ld_acquire_gpu(p.ready + k * 2 + t);
-                const float *slot = p.partial + static_cast<size_t>(k * 2 + t) * partial_slot_floats<D>();
-                m_star = fmaxf(m_star, __ldcg(slot + 128 * D + r));
-            }
-            f_own = (m_ref == -CUDART_INF_F) ? 0.f : ex2((m_ref - m_star) * c);
-            l *= f_own;
-            for (int k = blockIdx.x + 1; k <= c_last; ++k) {
-                const float *slot = p.partial + static_cast<size_t>(k * 2 + t) * partial_slot_floats<D>();
-                const float mk = __ldcg(slot + 128 * D + r);
-                const float fk = (mk == -CUDART_INF_F) ? 0.f : ex2((mk - m_star) * c);
-                l += fk * __ldcg(slot + 128 * D + 128 + r);
+            if (row_live) {
+#pragma unroll 4
+                for (int k = blockIdx.x + 1; k <= c_last; ++k)
+                    m_star = fmaxf(m_star, __ldcg(p.partial + static_cast<size_t>(partial_slot(k, t)) *
+                                                                  partial_slot_floats<D>() + 128 * D + r));
+                f_own = (m_ref == -CUDART_INF_F) ? 0.f : ex2((m_ref - m_star) * c);
+                l *= f_own;
+#pragma unroll 4
+                for (int k = blockIdx.x + 1; k <= c_last; ++k) {
+                    const float *slot = p.partial + static_cast<size_t>(partial_slot(k, t)) * partial_slot_floats<D>();
+                    const float mk = __ldcg(slot + 128 * D + r);
+                    const float fk = (mk == -CUDART_INF_F) ? 0.f : ex2((mk - m_star) * c);
+                    l = fmaf(fk, __ldcg(slot + 128 * D + 128 + r), l);
+                }
             }
         }
 
         // Final FP32 normalisation, then BF16 (a row with no allowed key has
         // l == 0 and is written as zeros).
+        if (!warp_live) continue;
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16 *orow =
-            p.o + (static_cast<size_t>(seg.b * p.Hq + seg.h) * p.L + row) * static_cast<size_t>(D);
+        __nv_bfloat16 *orow = row_valid
+            ? p.o + (static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row) * static_cast<size_t>(D)
+            : nullptr;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
             tmem_ld32(tO + cc * 32, o);
-            if (!ip.complete) {
+            if (!ip.complete && row_live) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f_own);
+#pragma unroll 2
                 for (int k = blockIdx.x + 1; k <= c_last; ++k) {
-                    const float *slot = p.partial + static_cast<size_t>(k * 2 + t) * partial_slot_floats<D>();
+                    const float *slot = p.partial + static_cast<size_t>(partial_slot(k, t)) * partial_slot_floats<D>();
                     const float mk = __ldcg(slot + 128 * D + r);
                     const float fk = (mk == -CUDART_INF_F) ? 0.f : ex2((mk - m_star) * c);
                     const float4 *src = reinterpret_cast<const float4 *>(slot + r * D + cc * 32);
@@ -648,7 +704,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-            if (row < p.L) {
+            if (orow) {
                 uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4)
@@ -656,6 +712,9 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             }
         }
     }
+#ifdef TFA_TRACE
+    if (threadIdx.x == 0 && blockIdx.x < 1024) g_tfa_cta_time[blockIdx.x][2] = globaltimer_ns();
+#endif
 }
 
 // ------------------------------------------------------------------ kernel

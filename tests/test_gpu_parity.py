@@ -173,6 +173,7 @@ def _sample_rows(w, n_per_head=24, seed=0):
     """Rows to check at full size: tile edges, tails and random rows, every head."""
     rng = np.random.default_rng(seed)
     L = w.L
+    n_per_head = min(n_per_head, L)  # a short query has fewer rows than the sample size
     fixed = [0, 1, 127, 128, 255, 256, L // 2, L - 129, L - 128, L - 2, L - 1]
     rows = []
     for b in range(w.B):

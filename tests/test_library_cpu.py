@@ -152,3 +152,20 @@ def test_flop_count_small_key_mask_cases():
         km = (torch.rand(B, S, generator=torch.Generator().manual_seed(1)) > 0.3).float()
         assert allowed_pairs(B, 3, L, S, causal=causal, window=window, key_mask=km) == \
             oracle.count_pairs(B, 3, L, S, causal=causal, window=window, key_mask=km)
+
+
+@pytest.mark.parametrize("L,code", [(0, tb.TFA_ERR_SHAPE), (9, tb.TFA_ERR_SHAPE),
+                                    (64, tb.TFA_ERR_SHAPE)])
+def test_decode_accepts_only_short_queries(L, code):
+    assert tb.tfa_decode(A16, A16, A16, A16, 1, 8, 2, L, 100, 128, 0.1, 1, 0, None, None) == code
+
+
+def test_decode_validates_like_prefill():
+    assert tb.tfa_decode(None, A16, A16, A16, 1, 8, 2, 1, 100, 128, 0.1, 1, 0, None,
+                         None) == tb.TFA_ERR_NULL
+    assert tb.tfa_decode(A16, A16, A16, A16, 1, 8, 3, 1, 100, 128, 0.1, 1, 0, None,
+                         None) == tb.TFA_ERR_HEADS
+    assert tb.tfa_decode(A16, A16, A16, A16, 1, 8, 2, 4, 3, 128, 0.1, 1, 0, None,
+                         None) == tb.TFA_ERR_SHAPE
+    assert tb.tfa_decode(A16, A16, A16, A16, 1, 8, 2, 1, 100, 128, 0.1, 0, 16, None,
+                         None) == tb.TFA_ERR_WINDOW

@@ -11,7 +11,7 @@ import pytest
 from sliding_window_gqa_tfa_b200 import binding as tb
 from sliding_window_gqa_tfa_b200.inputs import WORKLOADS
 
-CASES = [(w.B, w.Hq, w.L, w.S, w.causal, w.window) for w in WORKLOADS.values()] + [
+CASES = [(w.B, w.Hq, w.L, w.S, w.causal, w.window) for w in WORKLOADS.values() if w.L >= 9] + [
     (1, 1, 256, 1 << 20, True, 0),      # one item far longer than a CTA's share
     (2, 3, 300, 301, True, 0),
     (1, 4, 130, 700, True, 129),
