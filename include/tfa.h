@@ -28,13 +28,25 @@
  * on the current CUDA device; the call neither allocates nor frees the tensors
  * and never reads them on the host.  The library keeps one small status word
  * per device (allocated on the first call on that device) where the kernel
- * records a timed-out internal wait.
+ * records a timed-out internal wait, and per stream the scratch of the split
+ * schedule (2 x SMs partial slots of 128 x 128 + 256 floats, allocated on the
+ * first call on that stream, kept until process exit).
  *
  * Asynchrony: tfa_prefill validates its arguments on the host, then enqueues
  * the kernel on `stream` and returns; o is fully overwritten when the stream
  * reaches that point.  Errors found by validation are returned before any
  * launch, with no side effect.  A device-side failure (a wait that gave up)
  * is reported by tfa_check_status().
+ *
+ * Graph capture: tfa_prefill and tfa_decode may be captured into a CUDA graph
+ * on a stream that has already seen one call outside capture (that call
+ * creates the device state and the stream's scratch; a first call made during
+ * capture returns TFA_ERR_CAPTURE instead of allocating).  Every replay is a
+ * complete, independent call on the captured pointers, sizes and scale; the
+ * split schedule's synchronisation lives in device memory, not in the
+ * captured arguments.  A replay uses the scratch of the stream it was
+ * captured on, so it must not run concurrently with another replay or call
+ * that uses that stream's scratch (replaying on that stream guarantees it).
  */
 #ifndef TFA_H
 #define TFA_H
@@ -60,7 +72,9 @@ typedef enum {
     TFA_ERR_CUDA = 8,        /* a CUDA runtime/driver call failed (launch, encode, ...)  */
     TFA_ERR_TIMEOUT = 9,     /* a kernel wait gave up; the output of that call is invalid */
     TFA_ERR_SCALE = 10,      /* scale is not finite                                      */
-    TFA_ERR_FLAGS = 11       /* unknown debug flag bits                                  */
+    TFA_ERR_FLAGS = 11,      /* unknown debug flag bits                                  */
+    TFA_ERR_CAPTURE = 12     /* first call on a device or stream made inside a CUDA graph
+                                capture (it would allocate); call once outside capture   */
 } tfa_status;
 
 /* Minimum query length accepted by the tiled operator (tiny-llm Week 2 Day 5,

@@ -31,6 +31,7 @@ TFA_ERR_CUDA = 8
 TFA_ERR_TIMEOUT = 9
 TFA_ERR_SCALE = 10
 TFA_ERR_FLAGS = 11
+TFA_ERR_CAPTURE = 12
 
 TFA_DEBUG_NO_TILE_SKIP = 1
 TFA_DEBUG_MASK_ALL = 2
@@ -50,7 +51,7 @@ _lib = None
 class TfaError(RuntimeError):
     def __init__(self, code: int, where: str = "tfa_prefill"):
         self.code = code
-        detail = f" [{last_error()}]" if code == TFA_ERR_CUDA else ""
+        detail = f" [{last_error()}]" if code in (TFA_ERR_CUDA, TFA_ERR_CAPTURE) else ""
         super().__init__(f"{where} failed with status {code}: {status_string(code)}{detail}")
 
 

@@ -26,11 +26,11 @@ constexpr int kMaxDevices = 64;
 
 // Scratch of the split schedule, one set per (device, stream) so that calls on
 // different streams never share it: a partial slot and a ready flag per
-// (CTA, query tile), and the epoch that marks this stream's latest launch.
+// (CTA, query tile), then two control words (finished launches, finished CTAs).
 struct SplitScratch {
     float *partial = nullptr;
     unsigned *ready = nullptr;
-    unsigned epoch = 0;
+    unsigned *ctl = nullptr;
 };
 
 struct DeviceState {
@@ -72,6 +72,44 @@ int get_encode_fn() {
     return TFA_OK;
 }
 
+// Shared-memory opt-in and the register check for one kernel variant, done
+// once per device at first use (never lazily, so a captured call needs neither).
+template <int D, bool KM>
+int prepare_kernel(DeviceState &st) {
+    using C = tfa::Cfg<D>;
+    auto kern = tfa::tfa_prefill_kernel<D, KM>;
+    const int smem = KM ? C::kSmemBytesKeyMask : C::kSmemBytes;
+    const int which = (D == 128 ? 2 : 0) + (KM ? 1 : 0);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return cuda_fail("cudaFuncGetAttributes", e);
+    // The setmaxnreg split inside the kernel is sized for exactly kRegsLaunch
+    // registers per thread at launch; any other count could leave a warpgroup
+    // waiting for registers that do not exist, so refuse to launch.
+    if (fa.maxThreadsPerBlock < tfa::kThreads || fa.numRegs != tfa::kRegsLaunch) {
+        snprintf(g_last_error, sizeof g_last_error,
+                 "kernel uses %d registers/thread (%d expected), at most %d threads fit, %d needed",
+                 fa.numRegs, tfa::kRegsLaunch, fa.maxThreadsPerBlock, tfa::kThreads);
+        return TFA_ERR_CUDA;
+    }
+    st.smem_attr[which] = true;
+    return TFA_OK;
+}
+
+// First use allocates; that cannot happen inside a CUDA graph capture, so a
+// first call made under capture is refused (one ordinary call on the stream
+// beforehand creates everything a captured call needs).
+int refuse_under_capture(cudaStream_t stream, const char *what) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusNone)
+        return TFA_OK;
+    snprintf(g_last_error, sizeof g_last_error,
+             "first use of %s during graph capture: make one call on this stream before capturing it",
+             what);
+    return TFA_ERR_CAPTURE;
+}
+
 // Per-device state, created on first use with that device current.  The
 // status word is cleared on `stream` so it is ordered before the first launch.
 int device_state(cudaStream_t stream, DeviceState **out) {
@@ -81,12 +119,18 @@ int device_state(cudaStream_t stream, DeviceState **out) {
     if (dev < 0 || dev >= kMaxDevices) return drv_fail("device index out of range", dev);
     DeviceState &st = g_dev[dev];
     if (!st.init) {
+        if (int rc = refuse_under_capture(stream, "the device")) return rc;
         if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail("cudaDeviceGetAttribute", e);
         if ((e = cudaMalloc(&st.status, 256)) != cudaSuccess) return cuda_fail("cudaMalloc(status)", e);
         if ((e = cudaMemsetAsync(st.status, 0, 256, stream)) != cudaSuccess)
             return cuda_fail("cudaMemsetAsync(status)", e);
         if (int rc = get_encode_fn()) return rc;
+        int rc = prepare_kernel<64, false>(st);
+        if (!rc) rc = prepare_kernel<64, true>(st);
+        if (!rc) rc = prepare_kernel<128, false>(st);
+        if (!rc) rc = prepare_kernel<128, true>(st);
+        if (rc) return rc;
         st.init = true;
     }
     *out = &st;
@@ -101,15 +145,17 @@ int split_scratch(DeviceState &st, cudaStream_t stream, SplitScratch **out) {
         *out = &found->second;
         return TFA_OK;
     }
+    if (int rc = refuse_under_capture(stream, "this stream")) return rc;
     SplitScratch ss;
     const size_t slots = 2 * static_cast<size_t>(st.sm_count);
     cudaError_t e = cudaMalloc(&ss.partial, slots * tfa::partial_slot_floats<128>() * sizeof(float));
     if (e != cudaSuccess) return cuda_fail("cudaMalloc(split partials)", e);
-    if ((e = cudaMalloc(&ss.ready, slots * sizeof(unsigned))) != cudaSuccess) {
+    if ((e = cudaMalloc(&ss.ready, (slots + 2) * sizeof(unsigned))) != cudaSuccess) {
         cudaFree(ss.partial);
         return cuda_fail("cudaMalloc(split flags)", e);
     }
-    if ((e = cudaMemsetAsync(ss.ready, 0, slots * sizeof(unsigned), stream)) != cudaSuccess)
+    ss.ctl = ss.ready + slots;
+    if ((e = cudaMemsetAsync(ss.ready, 0, (slots + 2) * sizeof(unsigned), stream)) != cudaSuccess)
         return cuda_fail("cudaMemsetAsync(split flags)", e);
     *out = &st.split.emplace(stream, ss).first->second;
     return TFA_OK;
@@ -176,23 +222,7 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     auto kern = key_mask ? tfa::tfa_prefill_kernel<D, true> : tfa::tfa_prefill_kernel<D, false>;
     const int smem = key_mask ? C::kSmemBytesKeyMask : C::kSmemBytes;
     const int which = (D == 128 ? 2 : 0) + (key_mask ? 1 : 0);
-    if (!st.smem_attr[which]) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
-        cudaFuncAttributes fa;
-        if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess)
-            return cuda_fail("cudaFuncGetAttributes", e);
-        // The setmaxnreg split inside the kernel is sized for exactly kRegsLaunch
-        // registers per thread at launch; any other count could leave a warpgroup
-        // waiting for registers that do not exist, so refuse to launch.
-        if (fa.maxThreadsPerBlock < tfa::kThreads || fa.numRegs != tfa::kRegsLaunch) {
-            snprintf(g_last_error, sizeof g_last_error,
-                     "kernel uses %d registers/thread (%d expected), at most %d threads fit, %d needed",
-                     fa.numRegs, tfa::kRegsLaunch, fa.maxThreadsPerBlock, tfa::kThreads);
-            return TFA_ERR_CUDA;
-        }
-        st.smem_attr[which] = true;
-    }
+    if (!st.smem_attr[which]) return drv_fail("kernel not prepared", which);
     tfa::Params p;
     p.o = static_cast<__nv_bfloat16 *>(o);
     p.key_mask = key_mask;
@@ -235,11 +265,7 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     const int grid = sh.grid;
     p.partial = ss ? ss->partial : nullptr;
     p.ready = ss ? ss->ready : nullptr;
-    p.epoch = 0;
-    if (ss) {
-        if (++ss->epoch == 0) ++ss->epoch;  // 0 is the flags' initial value
-        p.epoch = ss->epoch;
-    }
+    p.ctl = ss ? ss->ctl : nullptr;
     kern<<<grid, tfa::kThreads, smem, stream>>>(mq, mk, mv, p);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFA_OK : cuda_fail("kernel launch", e);
@@ -387,6 +413,11 @@ int noalloc_state(cudaStream_t stream, DeviceState **out) {
         if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail("cudaDeviceGetAttribute", e);
         if (int rc = get_encode_fn()) return rc;
+        int rc = prepare_kernel<64, false>(st);
+        if (!rc) rc = prepare_kernel<64, true>(st);
+        if (!rc) rc = prepare_kernel<128, false>(st);
+        if (!rc) rc = prepare_kernel<128, true>(st);
+        if (rc) return rc;
         st.status = static_cast<unsigned *>(ptr);
         st.init = true;
     }
@@ -471,6 +502,7 @@ extern "C" const char *tfa_status_string(int status) {
         case TFA_ERR_CUDA: return "a CUDA call failed";
         case TFA_ERR_TIMEOUT: return "a kernel wait timed out; the output is invalid";
         case TFA_ERR_SCALE: return "scale must be finite";
+        case TFA_ERR_CAPTURE: return "first use of a device or stream inside a CUDA graph capture";
         case TFA_ERR_FLAGS: return "unknown debug flags";
         default: return "unknown status";
     }

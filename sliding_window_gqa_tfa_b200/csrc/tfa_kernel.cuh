@@ -127,8 +127,11 @@ struct Params {
     const float *key_mask;
     unsigned *status;
     float *partial;    // split schedule: per (CTA, tile) partial m, l, accumulator
-    unsigned *ready;   // split schedule: per (CTA, tile) flag, == epoch when published
-    unsigned epoch;    // nonzero, different for every launch that uses `ready`
+    unsigned *ready;   // split schedule: per (CTA, tile) flag, == the launch's epoch when published
+    // split schedule: ctl[0] counts finished launches (the epoch of a launch is
+    // ctl[0] + 1, read from device memory so a captured graph replays correctly),
+    // ctl[1] counts the CTAs of the running launch that have finished
+    unsigned *ctl;
     int B, Hq, Hkv, L, S, G;
     int causal, window;
     unsigned flags;
@@ -166,6 +169,12 @@ __host__ __device__ constexpr uint32_t bias_offset(int row, int k) {
 template <int D>
 __host__ __device__ constexpr int partial_slot_floats() { return 128 * D + 256; }
 __host__ __device__ constexpr int partial_slot(int cta, int t) { return cta * 2 + t; }
+
+// This launch's epoch (never 0, the flags' initial value).
+__device__ __forceinline__ unsigned launch_epoch(const unsigned *ctl) {
+    const unsigned e = *reinterpret_cast<const volatile unsigned *>(ctl) + 1u;
+    return e == 0u ? 1u : e;
+}
 
 struct ItemPlan {
     int b, h, g;
@@ -446,6 +455,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     const float c = p.scale_log2;
     const int lane = threadIdx.x & 31;
     uint32_t s_cnt = 0, o_cnt = 0, pub_cnt = 0, fin_cnt = 0;
+    const unsigned epoch = p.ctl ? launch_epoch(p.ctl) : 0u;
     int trace_step = 0;
     (void)trace_step;
 
@@ -630,7 +640,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (lane == 0) mbar_arrive(bar.pub(t));
             if (r == 0 && mbar_wait(bar.pub(t), pub_cnt & 1, abort_flag, p.status)) {
                 __threadfence();
-                st_release_gpu(p.ready + partial_slot(blockIdx.x, t), p.epoch);
+                st_release_gpu(p.ready + partial_slot(blockIdx.x, t), epoch);
             }
             ++pub_cnt;
             continue;
@@ -646,7 +656,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (r == 0) {
                 bool ok = true;
                 for (int k = blockIdx.x + 1; k <= c_last && ok; ++k)
-                    ok = flag_wait(p.ready + partial_slot(k, t), p.epoch, abort_flag, p.status);
+                    ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status);
                 mbar_arrive(bar.fin(t));  // arrive even on failure; the abort flag tells
             }
             if (!__all_sync(0xffffffffu, mbar_wait(bar.fin(t), fin_cnt & 1, abort_flag, p.status)))
@@ -800,6 +810,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
+    }
+    // The last CTA to finish advances the epoch for the next launch; every
+    // CTA read it before arriving here, and launches on a stream do not overlap.
+    if (p.ctl && threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.ctl + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.ctl + 1, 0u);
+            atomicAdd(p.ctl, 1u);
+        }
     }
 }
 

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(12):
+    for code in range(13):
         s = tb.status_string(code)
         assert s and s != "unknown status"
     assert tb.status_string(99) == "unknown status"
