@@ -33,6 +33,9 @@ MUTATIONS = {
     "drop_scale": 5,
     "keymask_inverted": 6,
     "empty_row_uniform": 7,
+    "softcap_before_scale": 8,
+    "sink_scaled": 9,
+    "sink_in_numerator": 10,
 }
 
 
@@ -57,8 +60,11 @@ def _load():
             lib.oracle_attention.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                              i32, i32, P, P, i64, i32]
             lib.oracle_attention.restype = i32
+            lib.oracle_attention_ex.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
+                                                i32, i32, P, f64, P, P, i64, i32]
+            lib.oracle_attention_ex.restype = i32
             lib.oracle_attention_mutant.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32,
-                                                    f64, i32, i32, P, i32]
+                                                    f64, i32, i32, P, f64, P, i32]
             lib.oracle_attention_mutant.restype = i32
             lib.oracle_softmax_weights.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                    i32, i32, P, i32, i32, i32]
@@ -107,11 +113,25 @@ def _shape(q, k):
     return B, Hq, Hkv, L, S, D
 
 
-def attention(q, k, v, *, scale, causal, window=0, key_mask=None, rows=None, threads=0):
-    """Plain fp64 definition.  rows: optional flattened (b*Hq+h)*L+i indices."""
+def _sinks(sinks, Hq):
+    if sinks is None:
+        return None
+    if not isinstance(sinks, np.ndarray):
+        sinks = sinks.detach().cpu().float().numpy()
+    sinks = np.ascontiguousarray(sinks, dtype=np.float32).reshape(-1)
+    if sinks.size != Hq:
+        raise ValueError("sinks must hold one logit per query head")
+    return sinks
+
+
+def attention(q, k, v, *, scale, causal, window=0, key_mask=None, softcap=0.0, sinks=None,
+              rows=None, threads=0):
+    """Plain fp64 definition.  softcap: 0 = none; sinks: fp32 [Hq] logits or None;
+    rows: optional flattened (b*Hq+h)*L+i indices."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, Hq, Hkv, L, S, D = _shape(qb, kb)
     km = _mask(key_mask)
+    sk = _sinks(sinks, Hq)
     if rows is None:
         out = np.empty((B, Hq, L, D), dtype=np.float64)
         r_ptr, nr = None, 0
@@ -119,23 +139,25 @@ def attention(q, k, v, *, scale, causal, window=0, key_mask=None, rows=None, thr
         r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         out = np.empty((r.size, D), dtype=np.float64)
         r_ptr, nr = r.ctypes.data_as(ctypes.c_void_p), r.size
-    rc = _load().oracle_attention(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L, S, D,
-                                  float(scale), int(bool(causal)), int(window), _ptr(km),
-                                  r_ptr, nr, int(threads))
+    rc = _load().oracle_attention_ex(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L, S,
+                                     D, float(scale), int(bool(causal)), int(window), _ptr(km),
+                                     float(softcap), _ptr(sk), r_ptr, nr, int(threads))
     if rc:
         raise ValueError(f"oracle_attention rejected its arguments (code {rc})")
     return out
 
 
-def attention_mutant(q, k, v, *, scale, causal, window=0, key_mask=None, mutation):
+def attention_mutant(q, k, v, *, scale, causal, window=0, key_mask=None, softcap=0.0,
+                     sinks=None, mutation):
     qb, kb, vb = _bits(q), _bits(k), _bits(v)
     B, Hq, Hkv, L, S, D = _shape(qb, kb)
     km = _mask(key_mask)
+    sk = _sinks(sinks, Hq)
     out = np.empty((B, Hq, L, D), dtype=np.float64)
     code = MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
     rc = _load().oracle_attention_mutant(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L,
                                          S, D, float(scale), int(bool(causal)), int(window),
-                                         _ptr(km), code)
+                                         _ptr(km), float(softcap), _ptr(sk), code)
     if rc:
         raise ValueError(f"oracle_attention_mutant rejected its arguments (code {rc})")
     return out

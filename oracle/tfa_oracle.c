@@ -18,9 +18,14 @@
  *       (causal && window > 0 => j > p - window) sliding window [p-W+1, p]
  *       (key_mask == NULL || key_mask[b,j] > 0.5) length-S key mask
  *     s_j = scale * sum_d q[b,h,i,d] * k[b,g,j,d]       (fp64, exact bf16 upcast)
+ *     softcap c > 0   -> s_j := c * tanh(s_j / c)       (after the scale)
  *     no allowed key  -> o[b,h,i,:] = 0
  *     otherwise       -> m = max s_j, w_j = exp(s_j - m),
  *                        o[b,h,i,:] = sum_j w_j v[b,g,j,:] / sum_j w_j
+ *     attention sink  -> a per-query-head logit sigma_h joins the softmax
+ *       sigma_h           denominator only: m = max(max_j s_j, sigma_h),
+ *                        o = sum_j w_j v_j / (sum_j w_j + exp(sigma_h - m));
+ *                        a row with no allowed key stays 0
  *
  * Sources (page title, section):
  *   tiny-llm "Week 2 Day 5: Tiled Dense Prefill Attention", Task 1 (layout
@@ -32,7 +37,15 @@
  *     flash_attention_windowed_forward and flash_attention_decode comments
  *     (window keeps keys [max(0, p-window+1), p], window <= 0 = unbounded;
  *     FP32 key mask 1 valid / 0 invalid, positions with mask <= 0.5 dropped,
- *     combined multiplicatively with the causal/window mask).
+ *     combined multiplicatively with the causal/window mask; Gemma-2
+ *     extensions: attn_softcap > 0 replaces each score, after the
+ *     1/sqrt(head_dim) scale and before mask and softmax, by
+ *     attn_softcap * tanh(score / attn_softcap), 0 disables it).
+ *   mlx-lm PR "Add fused prefill SDPA for sliding-window caches",
+ *     Correctness (attention sinks among the tested cases; the page names
+ *     them without a formula: the sink reading above is the plain one, a
+ *     logit with no value row, taken in the same units as the scores and
+ *     neither scaled nor capped).
  *   tinygrad "symbolic llm with prefill" compare view, apps/llm.py
  *     (_attention_inner: scaled_dot_product_attention(..., enable_gqa=True)
  *     with the causal mask full(-inf).triu(start_pos+1)).
@@ -62,6 +75,9 @@ enum {
     MUT_DROP_SCALE = 5,          /* s_j without the scale factor             */
     MUT_KEYMASK_INVERTED = 6,    /* keep mask <= 0.5 instead of > 0.5        */
     MUT_EMPTY_ROW_UNIFORM = 7,   /* fully masked row averages all V rows     */
+    MUT_SOFTCAP_BEFORE_SCALE = 8,/* c * tanh(raw / c) * scale                */
+    MUT_SINK_SCALED = 9,         /* sink logit multiplied by the scale       */
+    MUT_SINK_IN_NUMERATOR = 10,  /* sink weight also added to every output   */
 };
 
 static double bf16_bits_to_f64(uint16_t bits)
@@ -125,8 +141,8 @@ static int check_args(const void *q, const void *k, const void *v, const void *o
 /* One output row, two passes, exact softmax, no tiling. */
 static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
                     int B, int Hq, int Hkv, int L, int S, int D, double scale,
-                    int causal, int window, const float *key_mask, int mutation,
-                    long row, double *s_buf)
+                    int causal, int window, const float *key_mask, double softcap,
+                    const float *sinks, int mutation, long row, double *s_buf)
 {
     long i = row % L;
     long bh = row / L;
@@ -151,6 +167,13 @@ static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
         const uint16_t *kr = kb + (size_t)j * D;
         for (int d = 0; d < D; ++d) acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kr[d]);
         s_buf[j] = sc * acc;
+        if (softcap > 0.0) {
+            /* brotensor flash_attention.h, Gemma-2 extensions: cap after the scale */
+            if (mutation == MUT_SOFTCAP_BEFORE_SCALE)
+                s_buf[j] = softcap * tanh(acc / softcap) * sc;
+            else
+                s_buf[j] = softcap * tanh(s_buf[j] / softcap);
+        }
         if (s_buf[j] > m) m = s_buf[j];
         any = 1;
     }
@@ -163,6 +186,13 @@ static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
         }
         return;
     }
+    /* attention sink: one more logit in the denominator, with no value row */
+    double sigma = -INFINITY;
+    if (sinks) {
+        sigma = (double)sinks[h];
+        if (mutation == MUT_SINK_SCALED) sigma *= scale;
+        if (sigma > m) m = sigma;
+    }
     double denom = 0.0;
     for (long j = 0; j < S; ++j) {
         if (s_buf[j] == -INFINITY) continue;
@@ -171,16 +201,24 @@ static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
         const uint16_t *vr = vb + (size_t)j * D;
         for (int d = 0; d < D; ++d) out[d] += w * bf16_bits_to_f64(vr[d]);
     }
+    if (sinks) {
+        double ws = exp(sigma - m);
+        denom += ws;
+        if (mutation == MUT_SINK_IN_NUMERATOR)
+            for (int d = 0; d < D; ++d) out[d] += ws;
+    }
     for (int d = 0; d < D; ++d) out[d] /= denom;
 }
 
 static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
                           int B, int Hq, int Hkv, int L, int S, int D, double scale,
-                          int causal, int window, const float *key_mask,
-                          const int64_t *rows, int64_t nrows, int nthreads, int mutation)
+                          int causal, int window, const float *key_mask, double softcap,
+                          const float *sinks, const int64_t *rows, int64_t nrows, int nthreads,
+                          int mutation)
 {
     int rc = check_args(q, k, v, o, B, Hq, Hkv, L, S, D);
     if (rc) return rc;
+    if (!(softcap >= 0.0) || isinf(softcap)) return 6;
     int64_t total = rows ? nrows : (int64_t)B * Hq * L;
     if (rows) {
         for (int64_t r = 0; r < nrows; ++r)
@@ -204,7 +242,7 @@ static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *
             if (!s_buf) continue;
             long row = rows ? (long)rows[r] : (long)r;
             one_row(q, k, v, o + (size_t)r * D, B, Hq, Hkv, L, S, D, scale, causal, window,
-                    key_mask, mutation, row, s_buf);
+                    key_mask, softcap, sinks, mutation, row, s_buf);
         }
         free(s_buf);
     }
@@ -220,16 +258,28 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, do
                      const int64_t *rows, int64_t nrows, int nthreads)
 {
     return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
-                          rows, nrows, nthreads, MUT_NONE);
+                          0.0, NULL, rows, nrows, nthreads, MUT_NONE);
+}
+
+/* The definition with the score variants: softcap (0 = none) and sinks
+ * (fp32 [Hq] logits, NULL = none). */
+int oracle_attention_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                        int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                        int causal, int window, const float *key_mask, double softcap,
+                        const float *sinks, const int64_t *rows, int64_t nrows, int nthreads)
+{
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                          softcap, sinks, rows, nrows, nthreads, MUT_NONE);
 }
 
 /* The same definition with one planted mistake; for mutation tests only. */
 int oracle_attention_mutant(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
                             int B, int Hq, int Hkv, int L, int S, int D, double scale,
-                            int causal, int window, const float *key_mask, int mutation)
+                            int causal, int window, const float *key_mask, double softcap,
+                            const float *sinks, int mutation)
 {
     return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
-                          NULL, 0, 1, mutation);
+                          softcap, sinks, NULL, 0, 1, mutation);
 }
 
 /* Row-normalised softmax weights of one (b, h): W is L x S, zero where the

@@ -6,8 +6,10 @@ attention arithmetic.
 
 Recipe: a CPU ``torch.Generator`` seeded with ``seed``; fp32 ``randn`` drawn in
 the order Q, K, V (K multiplied by ``k_scale`` before the cast), then, when the
-workload has a key mask, ``rand(B, S) >= 1 - keep`` as the 1/0 fp32 key mask;
-Q/K/V are cast to bf16 (round to nearest even).  The shapes are the model
+workload has a key mask, ``rand(B, S) >= 1 - keep`` as the 1/0 fp32 key mask,
+then, when it has attention sinks, ``sink_scale * randn(Hq)`` fp32 sink logits;
+Q/K/V are cast to bf16 (round to nearest even).  A logit softcap is a plain
+number of the workload (Gemma-2 uses 50).  The shapes are the model
 shapes the pages use: Qwen3-0.6B (16 query heads, 8 KV heads, head dim 128,
 tiny-llm "Week 2 Day 5"), the Llama geometry of TensorFold PR 3269 (56 query
 heads, 8 KV heads, group 7, head dim 128), the 1024-key sliding window of the
@@ -37,6 +39,8 @@ class Workload:
     key_mask_keep: float | None = None  # None: no key mask; else Bernoulli keep prob
     k_scale: float = 1.0
     scale: float | None = None  # None: 1/sqrt(D)
+    softcap: float = 0.0        # 0: none
+    sink_scale: float | None = None  # None: no sinks; else sinks ~ sink_scale * N(0, 1)
 
     @property
     def softmax_scale(self) -> float:
@@ -79,7 +83,18 @@ HEADLINE = "llama_gqa_chunk_2048x8192"
 
 def make_inputs(w: Workload, seed: int = 0):
     """Return (q, k, v, key_mask) as CPU tensors: bf16 [B,Hq,L,D], bf16 [B,Hkv,S,D] x2,
-    and fp32 [B,S] (or None)."""
+    and fp32 [B,S] (or None).  Sink logits, when the workload has them, come from
+    make_sinks with the same seed."""
+    return _draw(w, seed)[:4]
+
+
+def make_sinks(w: Workload, seed: int = 0):
+    """fp32 [Hq] sink logits of the workload (drawn after q, k, v and the key
+    mask from the same generator), or None."""
+    return _draw(w, seed)[4]
+
+
+def _draw(w: Workload, seed: int):
     g = torch.Generator().manual_seed(seed)
     q = torch.randn(w.B, w.Hq, w.L, w.D, generator=g, dtype=torch.float32)
     k = torch.randn(w.B, w.Hkv, w.S, w.D, generator=g, dtype=torch.float32)
@@ -89,11 +104,15 @@ def make_inputs(w: Workload, seed: int = 0):
     key_mask = None
     if w.key_mask_keep is not None:
         key_mask = (torch.rand(w.B, w.S, generator=g) >= (1.0 - w.key_mask_keep)).float()
-    return q.bfloat16(), k.bfloat16(), v.bfloat16(), key_mask
+    sinks = None
+    if w.sink_scale is not None:
+        sinks = w.sink_scale * torch.randn(w.Hq, generator=g, dtype=torch.float32)
+    return q.bfloat16(), k.bfloat16(), v.bfloat16(), key_mask, sinks
 
 
 def shaped(B, Hq, Hkv, L, S, D, *, causal=True, window=0, key_mask_keep=None, k_scale=1.0,
-           name="custom") -> Workload:
+           softcap=0.0, sink_scale=None, name="custom") -> Workload:
     """A workload of arbitrary shape drawn by the same recipe (for edge-case tests)."""
     return Workload(name, B=B, Hq=Hq, Hkv=Hkv, L=L, S=S, D=D, causal=causal, window=window,
-                    key_mask_keep=key_mask_keep, k_scale=k_scale)
+                    key_mask_keep=key_mask_keep, k_scale=k_scale, softcap=softcap,
+                    sink_scale=sink_scale)

@@ -192,6 +192,69 @@ def pin_chunked_prefix_invariance(attn):
     assert np.allclose(chunkw, fullw[:, :, Sfull - L:], atol=1e-14, rtol=0)
 
 
+def pin_softcap_acts_after_the_scale(attn):
+    """brotensor flash_attention.h, Gemma-2 extensions: the cap applies to the
+    scaled score.  Doubling q (exact in bf16) while halving the scale leaves
+    every scaled score, hence the output, unchanged; a cap taken before the
+    scale would not be invariant.  A small cap must also change the result."""
+    w = shaped(1, 4, 2, 12, 40, 32, k_scale=4.0)
+    q, k, v, _ = make_inputs(w, seed=31)
+    for cap in (2.0, 7.5):
+        a = attn(q, k, v, scale=0.3, causal=True, window=0, softcap=cap)
+        b = attn((q.float() * 2).bfloat16(), k, v, scale=0.15, causal=True, window=0, softcap=cap)
+        assert np.allclose(a, b, atol=1e-13, rtol=0)
+        assert not np.allclose(a, attn(q, k, v, scale=0.3, causal=True, window=0), atol=1e-3)
+
+
+def pin_softcap_limits(attn):
+    """tanh(x) -> x as the cap grows: a huge cap is no cap.  As the cap shrinks
+    every score goes to 0 and the weights to uniform: the output becomes the
+    plain mean of the visible values.  One visible key still returns its value."""
+    w = shaped(1, 4, 2, 10, 30, 16, k_scale=4.0)
+    q, k, v, _ = make_inputs(w, seed=32)
+    base = attn(q, k, v, scale=0.25, causal=True, window=0)
+    assert np.allclose(attn(q, k, v, scale=0.25, causal=True, window=0, softcap=1e9), base,
+                       atol=1e-12, rtol=0)
+    tiny = attn(q, k, v, scale=0.25, causal=False, window=0, softcap=1e-12)
+    mean = v.double().mean(dim=2).numpy()  # [B, Hkv, D]
+    for h in range(4):
+        assert np.allclose(tiny[0, h], mean[0, h // 2][None, :], atol=1e-10)
+    one = attn(q, k, v, scale=0.25, causal=True, window=1, softcap=3.0)
+    for h in range(4):
+        assert np.array_equal(one[0, h], v[0, h // 2, 20:30].double().numpy())
+
+
+def pin_sinks_match_sdpa_with_a_null_key(attn):
+    """A sink is a logit with no value row: torch's SDPA (fp64) over the keys
+    plus one all-zero key and value, whose additive mask entry is the sink
+    logit, gives the same output -- rows with no visible key included (their
+    only mass is the sink's, times a zero value)."""
+    B, Hq, Hkv, L, S, D, W = 2, 6, 2, 11, 37, 32, 9
+    q, k, v, km = make_inputs(shaped(B, Hq, Hkv, L, S, D, key_mask_keep=0.6), seed=33)
+    sinks = torch.tensor([-1.5, 0.0, 0.7, 2.5, -30.0, 6.0], dtype=torch.float32)
+    km[1, :] = 0.0  # batch 1: every row fully masked
+    P = S - L
+    for window in (0, W):
+        allowed = torch.ones(L, S, dtype=torch.bool).tril(diagonal=P)
+        if window:
+            allowed &= ~torch.ones(L, S, dtype=torch.bool).tril(diagonal=P - window)
+        allowed = allowed[None, None] & (km > 0.5)[:, None, None, :]
+        bias = torch.zeros(B, Hq, L, S + 1, dtype=torch.float64)
+        bias[..., :S] = torch.where(allowed, 0.0, -math.inf)
+        bias[..., S] = sinks.double()[None, :, None]
+        kz = torch.cat([k.double(), torch.zeros(B, Hkv, 1, D, dtype=torch.float64)], dim=2)
+        vz = torch.cat([v.double(), torch.zeros(B, Hkv, 1, D, dtype=torch.float64)], dim=2)
+        ref = F.scaled_dot_product_attention(q.double(), kz, vz, attn_mask=bias, scale=0.2,
+                                             enable_gqa=True).numpy()
+        got = attn(q, k, v, scale=0.2, causal=True, window=window, key_mask=km, sinks=sinks)
+        assert np.allclose(got, ref, atol=1e-12, rtol=1e-10)
+        assert np.all(got[1] == 0.0)
+    none = attn(q, k, v, scale=0.2, causal=True, window=0, key_mask=km)
+    neg = attn(q, k, v, scale=0.2, causal=True, window=0, key_mask=km,
+               sinks=torch.full((Hq,), -math.inf))
+    assert np.array_equal(none, neg)
+
+
 ATTENTION_PINS = [
     pin_golden_visibility,
     pin_fully_masked_rows_are_zero,
@@ -202,6 +265,9 @@ ATTENTION_PINS = [
     pin_window_one_returns_own_value,
     pin_wide_window_equals_causal,
     pin_chunked_prefix_invariance,
+    pin_softcap_acts_after_the_scale,
+    pin_softcap_limits,
+    pin_sinks_match_sdpa_with_a_null_key,
 ]
 
 
