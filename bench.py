@@ -34,7 +34,7 @@ sys.path.insert(0, ROOT)
 
 from sliding_window_gqa_tfa_b200 import binding as tb  # noqa: E402
 from sliding_window_gqa_tfa_b200.flops import algorithmic_bytes, useful_flops  # noqa: E402
-from sliding_window_gqa_tfa_b200.inputs import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+from sliding_window_gqa_tfa_b200.inputs import HEADLINE, WORKLOADS, make_inputs, make_sinks  # noqa: E402
 
 METRIC = "prefill attention TFLOP/s (unmasked pairs) and % of B200 BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -193,7 +193,7 @@ def cpu_baseline(w, q, k, v, km, budget_s=12.0):
     while time.perf_counter() - t0 < budget_s:
         rows = np.sort(rng.choice(n_rows, size=chunk, replace=False)).astype(np.int64)
         oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                         key_mask=km, rows=rows)
+                         key_mask=km, softcap=w.softcap, sinks=make_sinks(w, 0), rows=rows)
         done_rows += chunk
         flops += oracle_rows_flops(w, rows)
     dt = time.perf_counter() - t0
@@ -212,6 +212,7 @@ def run_reference(args, w):
 
     oracle.build()
     q, k, v, km = make_inputs(w, seed=0)
+    sinks = make_sinks(w, seed=0)
     rng = np.random.default_rng(1)
     n_rows = w.B * w.Hq * w.L
     per_step = 32
@@ -220,7 +221,7 @@ def run_reference(args, w):
         rows = np.sort(rng.choice(n_rows, size=per_step, replace=False)).astype(np.int64)
         t0 = time.perf_counter()
         oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                         key_mask=km, rows=rows)
+                         key_mask=km, softcap=w.softcap, sinks=sinks, rows=rows)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             times.append(dt)
@@ -235,7 +236,8 @@ def run_reference(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L,
                        "S": w.S, "D": w.D, "causal": w.causal, "window": w.window,
-                       "key_mask": w.key_mask_keep is not None, "sample_rows_per_step": per_step},
+                       "key_mask": w.key_mask_keep is not None, "softcap": w.softcap,
+                       "sinks": w.sink_scale is not None, "sample_rows_per_step": per_step},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -266,8 +268,11 @@ def main():
     tb.lib()  # fail loudly if the library is missing
 
     q, k, v, km = make_inputs(w, seed=rank)
+    sinks = make_sinks(w, seed=rank)
     dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
     dkm = km.to(dev) if km is not None else None
+    dsinks = sinks.to(dev) if sinks is not None else None
+    variant = w.softcap > 0 or sinks is not None  # score variants: tfa_attention_ex
     out = torch.empty_like(dq)
     flops = useful_flops(w.B, w.Hq, w.L, w.S, w.D, causal=w.causal, window=w.window, key_mask=km)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -275,7 +280,7 @@ def main():
 
     def step():
         tb.prefill(dq, dk, dv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                   key_mask=dkm, out=out)
+                   key_mask=dkm, out=out, softcap=w.softcap, sinks=dsinks)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -307,21 +312,42 @@ def main():
     hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
     hkm = km.pin_memory() if km is not None else None
     hout = torch.empty_like(hq).pin_memory()
+    hsinks = sinks.pin_memory() if sinks is not None else None
+    if variant:
+        # tfa_attention_ex takes device pointers: the step copies the pinned
+        # inputs in, calls it, and copies the output back, all on `stream`
+        eq, ek, ev = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
+        ekm = torch.empty_like(dkm) if dkm is not None else None
+        esinks = torch.empty_like(dsinks) if dsinks is not None else None
+        eout = torch.empty_like(dq)
+
+        def e2e_step():
+            for d, h in ((eq, hq), (ek, hk), (ev, hv), (ekm, hkm), (esinks, hsinks)):
+                if d is not None:
+                    d.copy_(h, non_blocking=True)
+            tb.prefill(eq, ek, ev, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                       key_mask=ekm, out=eout, softcap=w.softcap, sinks=esinks)
+            hout.copy_(eout, non_blocking=True)
+        e2e_api = "tfa_attention_ex (pinned host buffers, copies on the stream)"
+    else:
+        def e2e_step():
+            tb.prefill_host(hq, hk, hv, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                            key_mask=hkm, out=hout, stream=stream)
+        e2e_api = "tfa_prefill_host (pinned host buffers)"
     for _ in range(3):
-        tb.prefill_host(hq, hk, hv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                        key_mask=hkm, out=hout, stream=stream)
+        e2e_step()
     barrier(world)
     torch.cuda.synchronize(dev)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.e2e_steps):
-        tb.prefill_host(hq, hk, hv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                        key_mask=hkm, out=hout, stream=stream)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2 + (hkm.numel() * 4 if hkm is not None else 0)
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2 + (hkm.numel() * 4 if hkm is not None else 0) \
+        + (hsinks.numel() * 4 if hsinks is not None else 0)
     d2h = hout.numel() * 2
 
     peaks, peak_kind = load_peaks()
@@ -347,7 +373,8 @@ def main():
             "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L,
                        "S": w.S, "D": w.D, "causal": w.causal, "window": w.window,
-                       "key_mask": w.key_mask_keep is not None, "useful_gflop": flops / 1e9,
+                       "key_mask": w.key_mask_keep is not None, "softcap": w.softcap,
+                       "sinks": w.sink_scale is not None, "useful_gflop": flops / 1e9,
                        "l2": "flushed between steps (256 MiB memset outside the step events)",
                        "parallelism": f"weak x{world}" if world > 1 else "single GPU"},
             "ms_p10": per_sorted[len(per) // 10], "ms_p50": per_sorted[len(per) // 2],
@@ -360,7 +387,7 @@ def main():
                          "algorithmic_bytes": alg_bytes},
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": e2e_ms, "api": "tfa_prefill_host (pinned host buffers)"},
+                    "ms_per_step": e2e_ms, "api": e2e_api},
             "gpu_launches": args.steps,
             "clocks": clocks,
             "wall_s_timed_region": t_wall,

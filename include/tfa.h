@@ -73,8 +73,9 @@ typedef enum {
     TFA_ERR_TIMEOUT = 9,     /* a kernel wait gave up; the output of that call is invalid */
     TFA_ERR_SCALE = 10,      /* scale is not finite                                      */
     TFA_ERR_FLAGS = 11,      /* unknown debug flag bits                                  */
-    TFA_ERR_CAPTURE = 12     /* first call on a device or stream made inside a CUDA graph
+    TFA_ERR_CAPTURE = 12,    /* first call on a device or stream made inside a CUDA graph
                                 capture (it would allocate); call once outside capture   */
+    TFA_ERR_SOFTCAP = 13     /* softcap not finite, negative, or > 0 with scale == 0     */
 } tfa_status;
 
 /* Minimum query length accepted by the tiled operator (tiny-llm Week 2 Day 5,
@@ -117,6 +118,30 @@ int tfa_prefill(const void *q, const void *k, const void *v, void *o,
 int tfa_decode(const void *q, const void *k, const void *v, void *o,
                int B, int Hq, int Hkv, int L, int S, int D, float scale,
                int causal, int window, const float *key_mask, tfa_stream_t stream);
+
+/* tfa_attention_ex -- the same attention with the score variants, for any
+ * L >= 1 (L <= TFA_MAX_DECODE_ROWS takes tfa_decode's packed path, longer
+ * queries tfa_prefill's).  Arguments, layouts, ownership, asynchrony and
+ * errors are those of tfa_prefill/tfa_decode, plus:
+ *   softcap  logit soft-capping (brotensor flash_attention.h, Gemma-2
+ *            extensions): after the scale and before the masks and the
+ *            softmax, each score t becomes softcap * tanh(t / softcap).
+ *            0 disables it; negative, NaN or infinite values, or softcap > 0
+ *            with scale == 0, return TFA_ERR_SOFTCAP.
+ *   sinks    NULL, or caller-owned device fp32 [Hq], 4-byte aligned (else
+ *            TFA_ERR_ALIGN): attention-sink logits (named among the tested
+ *            cases of mlx-lm's sliding-window SDPA PR, without a formula).
+ *            Read here as one extra logit per query head that joins the
+ *            softmax denominator with no value row, in the same units as the
+ *            capped, scaled scores (not scaled, not capped):
+ *            o = sum_j e^(t_j - m) v_j / (sum_j e^(t_j - m) + e^(sink_h - m)).
+ *            A row with no allowed key is still written as zeros.
+ * With softcap = 0 and sinks = NULL the result equals tfa_prefill's
+ * (tfa_decode's for short queries). */
+int tfa_attention_ex(const void *q, const void *k, const void *v, void *o,
+                     int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                     int causal, int window, const float *key_mask, float softcap,
+                     const float *sinks, tfa_stream_t stream);
 
 /* Debug flags for tfa_prefill_debug. */
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */

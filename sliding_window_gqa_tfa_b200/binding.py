@@ -32,6 +32,7 @@ TFA_ERR_TIMEOUT = 9
 TFA_ERR_SCALE = 10
 TFA_ERR_FLAGS = 11
 TFA_ERR_CAPTURE = 12
+TFA_ERR_SOFTCAP = 13
 
 TFA_DEBUG_NO_TILE_SKIP = 1
 TFA_DEBUG_MASK_ALL = 2
@@ -76,6 +77,8 @@ def lib():
             L.tfa_prefill_noalloc.restype = i32
             L.tfa_decode.argtypes = common
             L.tfa_decode.restype = i32
+            L.tfa_attention_ex.argtypes = common[:14] + [f32, P, P]
+            L.tfa_attention_ex.restype = i32
             L.tfa_check_status.argtypes = [P]
             L.tfa_check_status.restype = i32
             L.tfa_last_error.argtypes = []
@@ -107,6 +110,12 @@ def status_string(code: int) -> str:
 
 
 # ----------------------------------------------------------- raw entry points
+def tfa_attention_ex(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, softcap,
+                     sinks, stream) -> int:
+    return lib().tfa_attention_ex(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+                                  softcap, sinks, stream)
+
+
 def tfa_prefill(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, stream) -> int:
     return lib().tfa_prefill(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
                              stream)
@@ -188,10 +197,11 @@ def _check(t, name, dtype, ndim):
 
 
 def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=None, stream=None,
-            debug_flags=0):
+            debug_flags=0, softcap=0.0, sinks=None):
     """Attention output [B,Hq,L,D] bf16 for bf16 q [B,Hq,L,D], k/v [B,Hkv,S,D] on one GPU.
 
-    L >= 9 goes to tfa_prefill, 1 <= L <= 8 to tfa_decode.  key_mask: optional
+    L >= 9 goes to tfa_prefill, 1 <= L <= 8 to tfa_decode; a softcap > 0 or
+    sinks (fp32 [Hq] on the device) go to tfa_attention_ex.  key_mask: optional
     fp32 [B,S] (1 keep / 0 drop).  Raises TfaError on a nonzero status."""
     import torch
 
@@ -221,6 +231,19 @@ def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=No
             float(scale), int(bool(causal)), int(window),
             ctypes.c_void_p(key_mask.data_ptr()) if key_mask is not None else None,
             _stream_handle(stream))
+    if softcap or sinks is not None:
+        if debug_flags:
+            raise ValueError("debug flags apply to tfa_prefill_debug only")
+        if sinks is not None:
+            _check(sinks, "sinks", torch.float32, 1)
+            if sinks.shape[0] != Hq:
+                raise ValueError("sinks must hold one logit per query head")
+        rc = tfa_attention_ex(*args[:14], float(softcap),
+                              ctypes.c_void_p(sinks.data_ptr()) if sinks is not None else None,
+                              args[14])
+        if rc != TFA_OK:
+            raise TfaError(rc, "tfa_attention_ex")
+        return out
     if L <= MAX_DECODE_ROWS:
         if debug_flags:
             raise ValueError("debug flags apply to the prefill path only (L >= 9)")

@@ -37,7 +37,7 @@ struct DeviceState {
     bool init = false;
     int sm_count = 0;
     unsigned *status = nullptr;  // device status word (TFA_DEVICE_TIMEOUT bits)
-    bool smem_attr[4] = {false, false, false, false};
+    bool smem_attr[8] = {};  // per kernel variant: D, key mask, softcap
     std::unordered_map<cudaStream_t, SplitScratch> split;
     // staging buffers of tfa_prefill_host
     void *h_buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
@@ -74,12 +74,14 @@ int get_encode_fn() {
 
 // Shared-memory opt-in and the register check for one kernel variant, done
 // once per device at first use (never lazily, so a captured call needs neither).
-template <int D, bool KM>
+constexpr int variant_index(int D, bool km, bool sc) { return (D == 128 ? 4 : 0) + (sc ? 2 : 0) + (km ? 1 : 0); }
+
+template <int D, bool KM, bool SC>
 int prepare_kernel(DeviceState &st) {
     using C = tfa::Cfg<D>;
-    auto kern = tfa::tfa_prefill_kernel<D, KM>;
+    auto kern = tfa::tfa_prefill_kernel<D, KM, SC>;
     const int smem = KM ? C::kSmemBytesKeyMask : C::kSmemBytes;
-    const int which = (D == 128 ? 2 : 0) + (KM ? 1 : 0);
+    const int which = variant_index(D, KM, SC);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
     cudaFuncAttributes fa;
@@ -95,6 +97,18 @@ int prepare_kernel(DeviceState &st) {
     }
     st.smem_attr[which] = true;
     return TFA_OK;
+}
+
+int prepare_all_kernels(DeviceState &st) {
+    int rc = prepare_kernel<64, false, false>(st);
+    if (!rc) rc = prepare_kernel<64, true, false>(st);
+    if (!rc) rc = prepare_kernel<64, false, true>(st);
+    if (!rc) rc = prepare_kernel<64, true, true>(st);
+    if (!rc) rc = prepare_kernel<128, false, false>(st);
+    if (!rc) rc = prepare_kernel<128, true, false>(st);
+    if (!rc) rc = prepare_kernel<128, false, true>(st);
+    if (!rc) rc = prepare_kernel<128, true, true>(st);
+    return rc;
 }
 
 // First use allocates; that cannot happen inside a CUDA graph capture, so a
@@ -126,11 +140,7 @@ int device_state(cudaStream_t stream, DeviceState **out) {
         if ((e = cudaMemsetAsync(st.status, 0, 256, stream)) != cudaSuccess)
             return cuda_fail("cudaMemsetAsync(status)", e);
         if (int rc = get_encode_fn()) return rc;
-        int rc = prepare_kernel<64, false>(st);
-        if (!rc) rc = prepare_kernel<64, true>(st);
-        if (!rc) rc = prepare_kernel<128, false>(st);
-        if (!rc) rc = prepare_kernel<128, true>(st);
-        if (rc) return rc;
+        if (int rc = prepare_all_kernels(st)) return rc;
         st.init = true;
     }
     *out = &st;
@@ -206,7 +216,7 @@ template <int D>
 int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o, int B, int Hq,
            int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
            cudaStream_t stream, unsigned flags, SplitScratch *ss, bool force_split = false,
-           bool packed = false) {
+           bool packed = false, float softcap = 0.f, const float *sinks = nullptr) {
     using C = tfa::Cfg<D>;
     // Short queries: a tile packs pack_heads query heads of one KV group, all L
     // rows of each (pack_heads * L <= 128), loaded as one {64, L, pack_heads} box.
@@ -218,10 +228,13 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
         encode_map(&mk, k, S, B * Hkv, D) || encode_map(&mv, v, S, B * Hkv, D))
         return TFA_ERR_CUDA;
     // separate instantiations with and without a key mask (the mask costs an
-    // extra MMA per score tile and extra shared memory; unmasked calls carry neither)
-    auto kern = key_mask ? tfa::tfa_prefill_kernel<D, true> : tfa::tfa_prefill_kernel<D, false>;
+    // extra MMA per score tile and extra shared memory) and a softcap (extra
+    // work per score); plain calls carry neither
+    const bool sc = softcap > 0.f;
+    auto kern = key_mask ? (sc ? tfa::tfa_prefill_kernel<D, true, true> : tfa::tfa_prefill_kernel<D, true, false>)
+                         : (sc ? tfa::tfa_prefill_kernel<D, false, true> : tfa::tfa_prefill_kernel<D, false, false>);
     const int smem = key_mask ? C::kSmemBytesKeyMask : C::kSmemBytes;
-    const int which = (D == 128 ? 2 : 0) + (key_mask ? 1 : 0);
+    const int which = variant_index(D, key_mask != nullptr, sc);
     if (!st.smem_attr[which]) return drv_fail("kernel not prepared", which);
     tfa::Params p;
     p.o = static_cast<__nv_bfloat16 *>(o);
@@ -237,6 +250,11 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.window = (causal && window > 0) ? window : 0;
     p.flags = flags;
     p.scale_log2 = scale * 1.4426950408889634f;
+    // softcap: y = b (1 - 2 / (2^(a x) + 1)) with a = 2 scale log2(e) / cap, b = cap / scale
+    p.softcap_a = sc ? 2.f * scale * 1.4426950408889634f / softcap : 0.f;
+    p.softcap_b = sc ? softcap / scale : 0.f;
+    p.softcap_u = sc ? scale / softcap : 0.f;
+    p.sinks = sinks;
     p.packed = packed ? 1 : 0;
     p.pack_heads = pack_heads;
     p.pack_chunks = pack_chunks;
@@ -330,6 +348,26 @@ extern "C" int tfa_decode(const void *q, const void *k, const void *v, void *o, 
                                    key_mask, s, 0u, ss, false, true);
 }
 
+extern "C" int tfa_attention_ex(const void *q, const void *k, const void *v, void *o, int B,
+                                int Hq, int Hkv, int L, int S, int D, float scale, int causal,
+                                int window, const float *key_mask, float softcap,
+                                const float *sinks, tfa_stream_t stream) {
+    const bool decode = L >= 1 && L <= TFA_MAX_DECODE_ROWS;
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true, decode);
+    if (rc) return rc;
+    if (!std::isfinite(softcap) || softcap < 0.f || (softcap > 0.f && scale == 0.f)) return TFA_ERR_SOFTCAP;
+    if (sinks && (reinterpret_cast<uintptr_t>(sinks) & 3u)) return TFA_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    SplitScratch *ss = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st)) || (rc = split_scratch(*st, s, &ss))) return rc;
+    return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                    key_mask, s, 0u, ss, false, decode, softcap, sinks)
+                      : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
+                                   key_mask, s, 0u, ss, false, decode, softcap, sinks);
+}
+
 extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o, int B,
                                  int Hq, int Hkv, int L, int S, int D, float scale, int causal,
                                  int window, const float *key_mask, tfa_stream_t stream,
@@ -413,11 +451,7 @@ int noalloc_state(cudaStream_t stream, DeviceState **out) {
         if ((e = cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
             return cuda_fail("cudaDeviceGetAttribute", e);
         if (int rc = get_encode_fn()) return rc;
-        int rc = prepare_kernel<64, false>(st);
-        if (!rc) rc = prepare_kernel<64, true>(st);
-        if (!rc) rc = prepare_kernel<128, false>(st);
-        if (!rc) rc = prepare_kernel<128, true>(st);
-        if (rc) return rc;
+        if (int rc = prepare_all_kernels(st)) return rc;
         st.status = static_cast<unsigned *>(ptr);
         st.init = true;
     }
@@ -503,6 +537,7 @@ extern "C" const char *tfa_status_string(int status) {
         case TFA_ERR_TIMEOUT: return "a kernel wait timed out; the output is invalid";
         case TFA_ERR_SCALE: return "scale must be finite";
         case TFA_ERR_CAPTURE: return "first use of a device or stream inside a CUDA graph capture";
+        case TFA_ERR_SOFTCAP: return "softcap must be finite and >= 0 (and needs a nonzero scale)";
         case TFA_ERR_FLAGS: return "unknown debug flags";
         default: return "unknown status";
     }

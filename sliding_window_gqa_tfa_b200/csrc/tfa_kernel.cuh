@@ -128,6 +128,12 @@ struct Params {
     unsigned *status;
     float *partial;    // split schedule: per (CTA, tile) partial m, l, accumulator
     unsigned *ready;   // split schedule: per (CTA, tile) flag, == the launch's epoch when published
+    // logit softcap (kernels instantiated with SC): a raw score x becomes
+    // (cap/scale) tanh(u), u = x scale/cap = x * softcap_u, evaluated as
+    // softcap_b * (1 - 2 / (2^(x * softcap_a) + 1)) for |u| >= 1/4 and by the
+    // odd Taylor series of tanh through u^7 below (no cancellation near 0)
+    float softcap_a, softcap_b, softcap_u;
+    const float *sinks;  // fp32 [Hq] sink logits, or nullptr
     // split schedule: ctl[0] counts finished launches (the epoch of a launch is
     // ctl[0] + 1, read from device memory so a captured graph replays correctly),
     // ctl[1] counts the CTAs of the running launch that have finished
@@ -443,7 +449,16 @@ out:
 }
 
 // ---------------------------------------------------- softmax and epilogue
-template <int D>
+constexpr float kLog2e = 1.4426950408889634f;
+
+// The row sum with the attention sink's term (a logit with no value row) for
+// output head `head`, against reference maximum m (raw-score units).
+__device__ __forceinline__ float add_sink(const Params &p, float l, float m, float c, int head) {
+    if (p.sinks == nullptr || m == -CUDART_INF_F) return l;  // an empty row stays 0
+    return l + ex2(fmaf(__ldg(p.sinks + head), kLog2e, -m * c));
+}
+
+template <int D, bool KM, bool SC>
 __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint32_t tmem,
                                           const Bars &bar, volatile int *abort_flag) {
     using C = Cfg<D>;
@@ -495,6 +510,23 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             uint32_t s[128];
             tmem_ld128(tS, s);
             if (r == 0) TFA_TR(t, trace_step, 2);
+            if constexpr (SC) {
+                // Gemma-2 logit softcap (brotensor flash_attention.h): the scaled
+                // score t becomes cap * tanh(t / cap), before masks and softmax;
+                // kept in raw-score units so the exponent below is unchanged.
+                const float a = p.softcap_a, b = p.softcap_b, us = p.softcap_u, nb2 = -2.f * p.softcap_b;
+#pragma unroll
+                for (int i = 0; i < 128; ++i) {
+                    const float x = __uint_as_float(s[i]);
+                    const float far = fmaf(nb2, rcp_approx(ex2(x * a) + 1.f), b);
+                    const float u = x * us, u2 = u * u;
+                    // tanh u = u - u^3/3 + 2u^5/15 - 17u^7/315 + O(u^9)
+                    const float series = u * fmaf(u2, fmaf(u2, fmaf(u2, -17.f / 315.f, 2.f / 15.f), -1.f / 3.f), 1.f);
+                    float y = fabsf(u) < 0.25f ? series * b : far;
+                    if (KM) y = (x == -CUDART_INF_F) ? x : y;  // a key-masked score stays -inf
+                    s[i] = __float_as_uint(y);
+                }
+            }
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 0);
 
             if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, 0, q_tile0, j, p.flags)) {
@@ -683,6 +715,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         // Final FP32 normalisation, then BF16 (a row with no allowed key has
         // l == 0 and is written as zeros).
         if (!warp_live) continue;
+        if (row_live) l = add_sink(p, l, m_star, c, out_head);  // m_star == m_ref for a whole tile
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16 *orow = row_valid
             ? p.o + (static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row) * static_cast<size_t>(D)
@@ -728,7 +761,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, bool KM>
+template <int D, bool KM, bool SC>
 __global__ void __launch_bounds__(kThreads, 1)
     tfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -794,7 +827,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         reg_alloc<kRegsSoftmax>();
-        softmax_role<D>(p, warp >> 2, tmem, bar, abort_flag);
+        softmax_role<D, KM, SC>(p, warp >> 2, tmem, bar, abort_flag);
     } else {
         reg_dealloc<kRegsOther>();
         if (warp == 8 && (lane == 0 || KM))

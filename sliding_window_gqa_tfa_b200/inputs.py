@@ -70,11 +70,19 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     Workload("long_chunk_2048x32768_d64", B=1, Hq=32, Hkv=8, L=2048, S=32768, D=64, k_scale=4.0),
     Workload("bidirectional_4096", B=1, Hq=32, Hkv=8, L=4096, S=4096, D=128, causal=False,
              k_scale=4.0),
+    # Score variants on the Llama chunk: a Gemma-2 style logit softcap (50, with K
+    # scaled x4 so that the cap bends the scores) and per-head attention sinks.
+    Workload("llama_gqa_chunk_2048x8192_softcap50", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
+             k_scale=4.0, softcap=50.0),
+    Workload("llama_gqa_chunk_2048x8192_sinks", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
+             sink_scale=2.0),
     # Short queries (1 <= L <= 8): token-by-token decoding over a long cache,
     # batched Qwen3-shaped decoding, and an 8-row chunk (e.g. draft verification).
     Workload("llama_gqa_decode_1x32768", B=1, Hq=56, Hkv=8, L=1, S=32768, D=128),
     Workload("qwen3_decode_b16_8192", B=16, Hq=16, Hkv=8, L=1, S=8192, D=128),
     Workload("llama_gqa_chunk_8x8192_b4", B=4, Hq=56, Hkv=8, L=8, S=8192, D=128),
+    Workload("llama_gqa_decode_1x32768_sinks_softcap", B=1, Hq=56, Hkv=8, L=1, S=32768, D=128,
+             softcap=30.0, sink_scale=2.0),
 ]}
 
 # The workload the throughput figure is quoted on.

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from sliding_window_gqa_tfa_b200 import binding as tb
-from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_inputs, shaped
+from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_inputs, make_sinks, shaped
 
 pytestmark = pytest.mark.gpu
 
@@ -28,10 +28,12 @@ def _cuda():
 
 def _run(w, seed=0, flags=0, inputs=None):
     q, k, v, km = inputs if inputs is not None else make_inputs(w, seed)
+    sinks = make_sinks(w, seed)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     dkm = km.cuda() if km is not None else None
     o = tb.prefill(dq, dk, dv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                   key_mask=dkm, debug_flags=flags)
+                   key_mask=dkm, debug_flags=flags, softcap=w.softcap,
+                   sinks=sinks.cuda() if sinks is not None else None)
     tb.check_status()
     return o, (q, k, v, km)
 
@@ -192,7 +194,7 @@ def test_parity_full_size_sampled(name):
     n_per_head = 12 if w.S >= 16384 else 24
     rows = _sample_rows(w, n_per_head=n_per_head)
     ref = oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                           key_mask=km, rows=rows)
+                           key_mask=km, softcap=w.softcap, sinks=make_sinks(w, 0), rows=rows)
     got = o.reshape(-1, w.D)[torch.as_tensor(rows, device=o.device)]
     err = _assert_close(got, ref, name)
     # properties that hold for every row at any size

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(13):
+    for code in range(14):
         s = tb.status_string(code)
         assert s and s != "unknown status"
     assert tb.status_string(99) == "unknown status"
@@ -62,6 +62,29 @@ def _call(**over):
 ])
 def test_rejections_happen_before_launch(over, code):
     assert _call(**over) == code
+
+
+def _call_ex(**over):
+    a = dict(q=A16, k=A16, v=A16, o=A16, B=1, Hq=8, Hkv=2, L=33, S=47, D=128, scale=0.088,
+             causal=1, window=0, key_mask=None, softcap=0.0, sinks=None, stream=None)
+    a.update(over)
+    return tb.tfa_attention_ex(**a)
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(softcap=-1.0), tb.TFA_ERR_SOFTCAP),
+    (dict(softcap=float("nan")), tb.TFA_ERR_SOFTCAP),
+    (dict(softcap=float("inf")), tb.TFA_ERR_SOFTCAP),
+    (dict(softcap=30.0, scale=0.0), tb.TFA_ERR_SOFTCAP),
+    (dict(sinks=ctypes.c_void_p(0x10002)), tb.TFA_ERR_ALIGN),
+    (dict(L=0, S=47), tb.TFA_ERR_SHORT_QUERY),
+    (dict(L=1, S=0), tb.TFA_ERR_SHAPE),
+    (dict(Hq=7, Hkv=2, softcap=30.0), tb.TFA_ERR_HEADS),
+    (dict(causal=0, window=4, L=3), tb.TFA_ERR_WINDOW),
+    (dict(D=80, L=1), tb.TFA_ERR_HEAD_DIM),
+])
+def test_score_variant_rejections_happen_before_launch(over, code):
+    assert _call_ex(**over) == code
 
 
 def test_debug_rejects_unknown_flags_before_launch():
