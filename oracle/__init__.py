@@ -37,6 +37,9 @@ MUTATIONS = {
     "sink_scaled": 9,
     "sink_in_numerator": 10,
 }
+# Planted mistakes of the rotating-cache and packed variable-length entry points.
+RING_MUTATIONS = {"ring_slot_shifted": 11}
+VARLEN_MUTATIONS = {"varlen_packed_causal": 12, "head_modulo": 3, "no_prefix_offset": 4}
 
 
 def build(force: bool = False) -> str:
@@ -63,8 +66,18 @@ def _load():
             lib.oracle_attention_ex.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                 i32, i32, P, f64, P, P, i64, i32]
             lib.oracle_attention_ex.restype = i32
-            lib.oracle_attention_mutant.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32,
+            lng = ctypes.c_long
+            lib.oracle_attention_mutant.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, lng, i32,
                                                     f64, i32, i32, P, f64, P, i32]
+            lib.oracle_attention_ring.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, lng, i32,
+                                                  f64, i32, f64, P, P, i64, i32]
+            lib.oracle_attention_ring.restype = i32
+            lib.oracle_attention_varlen.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, f64,
+                                                    i32, i32, f64, P, i32]
+            lib.oracle_attention_varlen.restype = i32
+            lib.oracle_attention_varlen_mutant.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32,
+                                                           f64, i32, i32, i32]
+            lib.oracle_attention_varlen_mutant.restype = i32
             lib.oracle_attention_mutant.restype = i32
             lib.oracle_softmax_weights.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                    i32, i32, P, i32, i32, i32]
@@ -156,10 +169,75 @@ def attention_mutant(q, k, v, *, scale, causal, window=0, key_mask=None, softcap
     out = np.empty((B, Hq, L, D), dtype=np.float64)
     code = MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
     rc = _load().oracle_attention_mutant(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L,
-                                         S, D, float(scale), int(bool(causal)), int(window),
+                                         S, 0, D, float(scale), int(bool(causal)), int(window),
                                          _ptr(km), float(softcap), _ptr(sk), code)
     if rc:
         raise ValueError(f"oracle_attention_mutant rejected its arguments (code {rc})")
+    return out
+
+
+def attention_ring(q, k_ring, v_ring, *, S, scale, window, softcap=0.0, sinks=None, rows=None,
+                   threads=0, mutation=0):
+    """Rotating cache: k/v [B,Hkv,R,D], key position j (0 <= j < S) in row j mod R;
+    causal with a window, R >= window - 1 + L.  Returns [B,Hq,L,D] (or rows x D)."""
+    qb, kb, vb = _bits(q), _bits(k_ring), _bits(v_ring)
+    B, Hq, L, D = qb.shape
+    Bk, Hkv, R, Dk = kb.shape
+    if Bk != B or Dk != D:
+        raise ValueError("q/k shapes disagree")
+    sk = _sinks(sinks, Hq)
+    code = RING_MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
+    if code:
+        if rows is not None:
+            raise ValueError("mutants compute every row")
+        out = np.empty((B, Hq, L, D), dtype=np.float64)
+        rc = _load().oracle_attention_mutant(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv,
+                                             L, int(S), int(R), D, float(scale), 1, int(window),
+                                             None, float(softcap), _ptr(sk), code)
+    else:
+        if rows is None:
+            out = np.empty((B, Hq, L, D), dtype=np.float64)
+            r_ptr, nr = None, 0
+        else:
+            r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+            out = np.empty((r.size, D), dtype=np.float64)
+            r_ptr, nr = r.ctypes.data_as(ctypes.c_void_p), r.size
+        rc = _load().oracle_attention_ring(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), B, Hq, Hkv, L,
+                                           int(S), int(R), D, float(scale), int(window),
+                                           float(softcap), _ptr(sk), r_ptr, nr, int(threads))
+    if rc:
+        raise ValueError(f"oracle_attention_ring rejected its arguments (code {rc})")
+    return out
+
+
+def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale, causal, window=0,
+                     softcap=0.0, sinks=None, threads=0, mutation=0):
+    """Packed variable-length attention: q [Tq,Hq,D], k/v [Tk,Hkv,D], int32 prefix sums
+    cu_seqlens_* [B+1].  Returns [Tq,Hq,D] float64."""
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    Tq, Hq, D = qb.shape
+    Tk, Hkv, Dk = kb.shape
+    if Dk != D or vb.shape != kb.shape:
+        raise ValueError("q/k/v shapes disagree")
+    cq = np.ascontiguousarray(np.asarray(cu_seqlens_q, dtype=np.int32))
+    ck = np.ascontiguousarray(np.asarray(cu_seqlens_k, dtype=np.int32))
+    B = cq.size - 1
+    if ck.size != B + 1 or cq[-1] != Tq or ck[-1] != Tk:
+        raise ValueError("cu_seqlens must be [B+1] prefix sums ending at the packed lengths")
+    sk = _sinks(sinks, Hq)
+    out = np.empty((Tq, Hq, D), dtype=np.float64)
+    code = VARLEN_MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
+    if code:
+        rc = _load().oracle_attention_varlen_mutant(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out),
+                                                    _ptr(cq), _ptr(ck), B, Hq, Hkv, D, float(scale),
+                                                    int(bool(causal)), int(window), code)
+    else:
+        rc = _load().oracle_attention_varlen(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(out), _ptr(cq),
+                                             _ptr(ck), B, Hq, Hkv, D, float(scale),
+                                             int(bool(causal)), int(window), float(softcap),
+                                             _ptr(sk), int(threads))
+    if rc:
+        raise ValueError(f"oracle_attention_varlen rejected its arguments (code {rc})")
     return out
 
 

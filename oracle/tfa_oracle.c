@@ -78,6 +78,8 @@ enum {
     MUT_SOFTCAP_BEFORE_SCALE = 8,/* c * tanh(raw / c) * scale                */
     MUT_SINK_SCALED = 9,         /* sink logit multiplied by the scale       */
     MUT_SINK_IN_NUMERATOR = 10,  /* sink weight also added to every output   */
+    MUT_RING_SLOT_SHIFTED = 11,  /* key j read from ring row (j + 1) mod R   */
+    MUT_VARLEN_PACKED_CAUSAL = 12,/* causal test on packed token indices      */
 };
 
 static double bf16_bits_to_f64(uint16_t bits)
@@ -138,34 +140,43 @@ static int check_args(const void *q, const void *k, const void *v, const void *o
     return 0;
 }
 
-/* One output row, two passes, exact softmax, no tiling. */
-static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
-                    int B, int Hq, int Hkv, int L, int S, int D, double scale,
-                    int causal, int window, const float *key_mask, double softcap,
-                    const float *sinks, int mutation, long row, double *s_buf)
-{
-    long i = row % L;
-    long bh = row / L;
-    int h = (int)(bh % Hq);
-    int b = (int)(bh / Hq);
-    int g = kv_head_impl(h, Hq, Hkv, mutation);
-    (void)B;
-    const uint16_t *qr = q + ((size_t)bh * L + i) * D;
-    const uint16_t *kb = k + ((size_t)b * Hkv + g) * (size_t)S * D;
-    const uint16_t *vb = v + ((size_t)b * Hkv + g) * (size_t)S * D;
-    const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
-    double sc = (mutation == MUT_DROP_SCALE) ? 1.0 : scale;
+/* Where one output row reads its operands: its query vector, and the K and V
+ * rows of its KV head -- key j at row slot(j) of kb / vb, rows kv_stride
+ * elements apart.  slot(j) = j, or j mod ring for a rotating cache
+ * (TensorFold PR 3269: "the ring slot of a key and value row"). */
+typedef struct {
+    const uint16_t *qr, *kb, *vb;
+    size_t kv_stride;
+    long ring;          /* 0: no ring */
+    const float *mrow;  /* key-mask row, or NULL */
+    int has_sink;
+    double sigma;       /* sink logit when has_sink */
+    long causal_shift;  /* 0; nonzero only in a planted mistake */
+} RowOperands;
 
+static long key_slot(const RowOperands *op, long j, int mutation)
+{
+    if (!op->ring) return j;
+    if (mutation == MUT_RING_SLOT_SHIFTED) return (j + 1) % op->ring;
+    return j % op->ring;
+}
+
+/* One output row, two passes, exact softmax, no tiling. */
+static void row_core(const RowOperands *op, double *out, long L, long S, long i, int D,
+                     double scale, int causal, int window, double softcap, int mutation,
+                     double *s_buf)
+{
+    double sc = (mutation == MUT_DROP_SCALE) ? 1.0 : scale;
     double m = -INFINITY;
     int any = 0;
     for (long j = 0; j < S; ++j) {
-        if (!allowed_impl(L, S, i, j, causal, window, mrow, mutation)) {
+        if (!allowed_impl(L, S, i + op->causal_shift, j, causal, window, op->mrow, mutation)) {
             s_buf[j] = -INFINITY;
             continue;
         }
         double acc = 0.0;
-        const uint16_t *kr = kb + (size_t)j * D;
-        for (int d = 0; d < D; ++d) acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kr[d]);
+        const uint16_t *kr = op->kb + (size_t)key_slot(op, j, mutation) * op->kv_stride;
+        for (int d = 0; d < D; ++d) acc += bf16_bits_to_f64(op->qr[d]) * bf16_bits_to_f64(kr[d]);
         s_buf[j] = sc * acc;
         if (softcap > 0.0) {
             /* brotensor flash_attention.h, Gemma-2 extensions: cap after the scale */
@@ -181,15 +192,17 @@ static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
     if (!any) {
         /* tiny-llm Week 2 Day 5, Task 2: no probability mass -> finite zeros. */
         if (mutation == MUT_EMPTY_ROW_UNIFORM) {
-            for (long j = 0; j < S; ++j)
-                for (int d = 0; d < D; ++d) out[d] += bf16_bits_to_f64(vb[(size_t)j * D + d]) / (double)S;
+            for (long j = 0; j < S; ++j) {
+                const uint16_t *vr = op->vb + (size_t)key_slot(op, j, mutation) * op->kv_stride;
+                for (int d = 0; d < D; ++d) out[d] += bf16_bits_to_f64(vr[d]) / (double)S;
+            }
         }
         return;
     }
     /* attention sink: one more logit in the denominator, with no value row */
     double sigma = -INFINITY;
-    if (sinks) {
-        sigma = (double)sinks[h];
+    if (op->has_sink) {
+        sigma = op->sigma;
         if (mutation == MUT_SINK_SCALED) sigma *= scale;
         if (sigma > m) m = sigma;
     }
@@ -198,10 +211,10 @@ static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
         if (s_buf[j] == -INFINITY) continue;
         double w = exp(s_buf[j] - m);
         denom += w;
-        const uint16_t *vr = vb + (size_t)j * D;
+        const uint16_t *vr = op->vb + (size_t)key_slot(op, j, mutation) * op->kv_stride;
         for (int d = 0; d < D; ++d) out[d] += w * bf16_bits_to_f64(vr[d]);
     }
-    if (sinks) {
+    if (op->has_sink) {
         double ws = exp(sigma - m);
         denom += ws;
         if (mutation == MUT_SINK_IN_NUMERATOR)
@@ -210,8 +223,34 @@ static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, dou
     for (int d = 0; d < D; ++d) out[d] /= denom;
 }
 
+/* Row (b, h, i) of the dense layout: q/o [B,Hq,L,D], k/v [B,Hkv,rows,D] with
+ * rows = S, or rows = ring for a rotating cache. */
+static void one_row(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *out,
+                    int Hq, int Hkv, int L, int S, long ring, int D, double scale,
+                    int causal, int window, const float *key_mask, double softcap,
+                    const float *sinks, int mutation, long row, double *s_buf)
+{
+    long i = row % L;
+    long bh = row / L;
+    int h = (int)(bh % Hq);
+    int b = (int)(bh / Hq);
+    int g = kv_head_impl(h, Hq, Hkv, mutation);
+    size_t rows = ring ? (size_t)ring : (size_t)S;
+    RowOperands op;
+    op.qr = q + ((size_t)bh * L + i) * D;
+    op.kb = k + ((size_t)b * Hkv + g) * rows * D;
+    op.vb = v + ((size_t)b * Hkv + g) * rows * D;
+    op.kv_stride = (size_t)D;
+    op.ring = ring;
+    op.mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+    op.has_sink = sinks != NULL;
+    op.sigma = sinks ? (double)sinks[h] : 0.0;
+    op.causal_shift = 0;
+    row_core(&op, out, L, S, i, D, scale, causal, window, softcap, mutation, s_buf);
+}
+
 static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
-                          int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                          int B, int Hq, int Hkv, int L, int S, long ring, int D, double scale,
                           int causal, int window, const float *key_mask, double softcap,
                           const float *sinks, const int64_t *rows, int64_t nrows, int nthreads,
                           int mutation)
@@ -219,6 +258,10 @@ static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *
     int rc = check_args(q, k, v, o, B, Hq, Hkv, L, S, D);
     if (rc) return rc;
     if (!(softcap >= 0.0) || isinf(softcap)) return 6;
+    /* a rotating cache keeps the last `ring` positions: every key a row may
+     * see must still be there, so causal, a window, and ring >= W - 1 + L */
+    if (ring < 0 || (ring > 0 && (!causal || window <= 0 || ring < (long)window - 1 + L)))
+        return 7;
     int64_t total = rows ? nrows : (int64_t)B * Hq * L;
     if (rows) {
         for (int64_t r = 0; r < nrows; ++r)
@@ -241,7 +284,7 @@ static int attention_impl(const uint16_t *q, const uint16_t *k, const uint16_t *
         for (int64_t r = 0; r < total; ++r) {
             if (!s_buf) continue;
             long row = rows ? (long)rows[r] : (long)r;
-            one_row(q, k, v, o + (size_t)r * D, B, Hq, Hkv, L, S, D, scale, causal, window,
+            one_row(q, k, v, o + (size_t)r * D, Hq, Hkv, L, S, ring, D, scale, causal, window,
                     key_mask, softcap, sinks, mutation, row, s_buf);
         }
         free(s_buf);
@@ -257,7 +300,7 @@ int oracle_attention(const uint16_t *q, const uint16_t *k, const uint16_t *v, do
                      int causal, int window, const float *key_mask,
                      const int64_t *rows, int64_t nrows, int nthreads)
 {
-    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, 0, D, scale, causal, window, key_mask,
                           0.0, NULL, rows, nrows, nthreads, MUT_NONE);
 }
 
@@ -268,18 +311,116 @@ int oracle_attention_ex(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int causal, int window, const float *key_mask, double softcap,
                         const float *sinks, const int64_t *rows, int64_t nrows, int nthreads)
 {
-    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, 0, D, scale, causal, window, key_mask,
+                          softcap, sinks, rows, nrows, nthreads, MUT_NONE);
+}
+
+/* Rotating cache (TensorFold PR 3269, WINDOW and RING): k/v are
+ * [B,Hkv,ring,D] and key position j (0 <= j < S, S = prefix + L) lives in row
+ * j mod ring.  Causal with a window; ring >= window - 1 + L, so every key a
+ * row may see is still in the ring (else returns 7). */
+int oracle_attention_ring(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                          int B, int Hq, int Hkv, int L, int S, long ring, int D, double scale,
+                          int window, double softcap, const float *sinks, const int64_t *rows,
+                          int64_t nrows, int nthreads)
+{
+    if (ring <= 0) return 7;
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, ring, D, scale, 1, window, NULL,
                           softcap, sinks, rows, nrows, nthreads, MUT_NONE);
 }
 
 /* The same definition with one planted mistake; for mutation tests only. */
 int oracle_attention_mutant(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
-                            int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                            int B, int Hq, int Hkv, int L, int S, long ring, int D, double scale,
                             int causal, int window, const float *key_mask, double softcap,
                             const float *sinks, int mutation)
 {
-    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
+    return attention_impl(q, k, v, o, B, Hq, Hkv, L, S, ring, D, scale, causal, window, key_mask,
                           softcap, sinks, NULL, 0, 1, mutation);
+}
+
+/* Packed variable-length attention (brotensor flash_attention.h,
+ * flash_attention_varlen_forward comment): sequence b owns query rows
+ * [cu_q[b], cu_q[b+1]) and key/value rows [cu_k[b], cu_k[b+1]) of
+ * q/o [Tq, Hq, D] and k/v [Tk, Hkv, D]; nothing crosses sequences.  Within a
+ * sequence the definition above holds with L = its query count and S = its
+ * key count, so the causal offset is S - L (brotensor's rule
+ * k - cu_k[b] <= q - cu_q[b] when the two counts match).  A causal sequence
+ * needs S >= L (else returns 8). */
+static int varlen_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                       const int32_t *cu_q, const int32_t *cu_k, int B, int Hq, int Hkv, int D,
+                       double scale, int causal, int window, double softcap, const float *sinks,
+                       int nthreads, int mutation)
+{
+    if (!q || !k || !v || !o || !cu_q || !cu_k) return 1;
+    if (B < 1 || Hq < 1 || Hkv < 1 || D < 1) return 2;
+    if (Hq % Hkv != 0) return 3;
+    if (!(softcap >= 0.0) || isinf(softcap)) return 6;
+    if (cu_q[0] != 0 || cu_k[0] != 0) return 8;
+    long max_s = 1;
+    for (int b = 0; b < B; ++b) {
+        long Lb = cu_q[b + 1] - cu_q[b], Sb = cu_k[b + 1] - cu_k[b];
+        if (Lb < 0 || Sb < 0 || (causal && Sb < Lb)) return 8;
+        if (Sb > max_s) max_s = Sb;
+    }
+    long total = (long)cu_q[B] * Hq;  /* rows, in packed order (t, h) */
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s_buf = (double *)malloc(sizeof(double) * (size_t)max_s);
+        if (!s_buf) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (long r = 0; r < total; ++r) {
+            if (!s_buf) continue;
+            long t = r / Hq;
+            int h = (int)(r % Hq);
+            int b = 0;
+            while (cu_q[b + 1] <= t) ++b;
+            long i = t - cu_q[b];
+            long Lb = cu_q[b + 1] - cu_q[b], Sb = cu_k[b + 1] - cu_k[b];
+            int g = kv_head_impl(h, Hq, Hkv, mutation);
+            RowOperands op;
+            op.qr = q + ((size_t)t * Hq + h) * D;
+            op.kb = k + ((size_t)cu_k[b] * Hkv + g) * D;
+            op.vb = v + ((size_t)cu_k[b] * Hkv + g) * D;
+            op.kv_stride = (size_t)Hkv * D;
+            op.ring = 0;
+            op.mrow = NULL;
+            op.has_sink = sinks != NULL;
+            op.sigma = sinks ? (double)sinks[h] : 0.0;
+            op.causal_shift = (mutation == MUT_VARLEN_PACKED_CAUSAL) ? (long)cu_q[b] - cu_k[b] : 0;
+            row_core(&op, o + ((size_t)t * Hq + h) * D, Lb, Sb, i, D, scale, causal, window,
+                     softcap, mutation, s_buf);
+        }
+        free(s_buf);
+    }
+    return failed ? 5 : 0;
+}
+
+int oracle_attention_varlen(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,
+                            const int32_t *cu_q, const int32_t *cu_k, int B, int Hq, int Hkv,
+                            int D, double scale, int causal, int window, double softcap,
+                            const float *sinks, int nthreads)
+{
+    return varlen_impl(q, k, v, o, cu_q, cu_k, B, Hq, Hkv, D, scale, causal, window, softcap,
+                       sinks, nthreads, MUT_NONE);
+}
+
+int oracle_attention_varlen_mutant(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                   double *o, const int32_t *cu_q, const int32_t *cu_k, int B,
+                                   int Hq, int Hkv, int D, double scale, int causal, int window,
+                                   int mutation)
+{
+    return varlen_impl(q, k, v, o, cu_q, cu_k, B, Hq, Hkv, D, scale, causal, window, 0.0, NULL,
+                       1, mutation);
 }
 
 /* Row-normalised softmax weights of one (b, h): W is L x S, zero where the
