@@ -75,7 +75,12 @@ typedef enum {
     TFA_ERR_FLAGS = 11,      /* unknown debug flag bits                                  */
     TFA_ERR_CAPTURE = 12,    /* first call on a device or stream made inside a CUDA graph
                                 capture (it would allocate); call once outside capture   */
-    TFA_ERR_SOFTCAP = 13     /* softcap not finite, negative, or > 0 with scale == 0     */
+    TFA_ERR_SOFTCAP = 13,    /* softcap not finite, negative, or > 0 with scale == 0     */
+    TFA_ERR_SEQLENS = 14,    /* (tfa_check_status) a variable-length call met an
+                                inconsistent cu_seqlens entry; that call's output is
+                                invalid                                                  */
+    TFA_ERR_RING = 15        /* ring cache without a window, ring_rows not a positive
+                                multiple of 64, or ring_rows < window - 1 + L            */
 } tfa_status;
 
 /* Minimum query length accepted by the tiled operator (tiny-llm Week 2 Day 5,
@@ -143,6 +148,51 @@ int tfa_attention_ex(const void *q, const void *k, const void *v, void *o,
                      int causal, int window, const float *key_mask, float softcap,
                      const float *sinks, tfa_stream_t stream);
 
+/* Longest batch of tfa_prefill_varlen. */
+#define TFA_MAX_VARLEN_SEQS 1024
+
+/* tfa_prefill_ring -- the same attention over a rotating (ring) K/V cache
+ * (TensorFold PR 3269's sliding layer: WINDOW and RING, the ring slot of a
+ * key and value row; mlx-lm's RotatingKVCache).  k and v hold the last
+ * ring_rows positions: [B, Hkv, ring_rows, D] bf16, where the key at absolute
+ * position j (0 <= j < S, S = prefix + L) lives in row j mod ring_rows.
+ * q/o are [B, Hq, L, D] as for tfa_prefill (any L >= 1; L <= 8 takes the
+ * packed short-query path).  Causal with a sliding window, always:
+ * window > 0, ring_rows a positive multiple of 64, and
+ * ring_rows >= window - 1 + L (every key a new row may see is still in the
+ * ring), else TFA_ERR_RING.  No key mask.  softcap and sinks as for
+ * tfa_attention_ex.  Other arguments, ownership and errors as tfa_prefill. */
+int tfa_prefill_ring(const void *q, const void *k, const void *v, void *o,
+                     int B, int Hq, int Hkv, int L, int S, int ring_rows, int D, float scale,
+                     int window, float softcap, const float *sinks, tfa_stream_t stream);
+
+/* tfa_prefill_varlen -- packed variable-length batches (brotensor
+ * flash_attention.h, flash_attention_varlen_forward; flash_attn_varlen_func
+ * semantics, here with GQA).  q and o are [total_q, Hq, D] bf16, k and v
+ * [total_k, Hkv, D] bf16, all caller-owned device memory, 16-byte aligned.
+ * cu_seqlens_q / cu_seqlens_k: caller-owned DEVICE int32 [B + 1] prefix sums
+ * (4-byte aligned), 1 <= B <= TFA_MAX_VARLEN_SEQS: sequence b owns query rows
+ * [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key/value rows
+ * [cu_seqlens_k[b], cu_seqlens_k[b+1]); nothing crosses sequences.
+ * max_seqlen_q bounds every sequence's query count (tiles are enumerated up
+ * to it).  Within sequence b the definition of tfa_prefill holds with
+ * L_b = its query count and S_b = its key count: causal rows are aligned to
+ * the end of the sequence's keys (prefix S_b - L_b; for L_b == S_b this is
+ * brotensor's (k - cu_k[b]) <= (q - cu_q[b])), and a causal sequence needs
+ * S_b >= L_b.  Any L_b >= 0 (no short-query minimum).  window, softcap and
+ * sinks as for tfa_attention_ex; no key mask.
+ * The lengths live in device memory, so they are checked by the kernel: a
+ * sequence whose entries are inconsistent (decreasing, past total_q/total_k,
+ * L_b > max_seqlen_q, or causal with S_b < L_b) is skipped, its rows are not
+ * written, and tfa_check_status() returns TFA_ERR_SEQLENS.  total_q == 0:
+ * nothing to do, TFA_OK without a launch (no pointer is examined); with
+ * queries, max_seqlen_q == 0 or total_k == 0 return TFA_ERR_SHAPE. */
+int tfa_prefill_varlen(const void *q, const void *k, const void *v, void *o,
+                       const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int Hq, int Hkv,
+                       int total_q, int total_k, int max_seqlen_q, int D, float scale,
+                       int causal, int window, float softcap, const float *sinks,
+                       tfa_stream_t stream);
+
 /* Debug flags for tfa_prefill_debug. */
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
 #define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */
@@ -198,7 +248,8 @@ int tfa_prefill_noalloc(const void *q, const void *k, const void *v, void *o,
 /* tfa_check_status -- synchronizes `stream`, then reads and clears the current
  * device's status words (tfa_prefill's and, once set up, tfa_prefill_noalloc's).
  * Returns TFA_OK, TFA_ERR_TIMEOUT if a kernel launched since the last check
- * recorded a wait that gave up, or TFA_ERR_CUDA. */
+ * recorded a wait that gave up, TFA_ERR_SEQLENS if a tfa_prefill_varlen call
+ * met inconsistent cu_seqlens (and no wait gave up), or TFA_ERR_CUDA. */
 int tfa_check_status(tfa_stream_t stream);
 
 /* tfa_last_error -- for the calling host thread, a description of the last CUDA

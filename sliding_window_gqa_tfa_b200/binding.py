@@ -33,6 +33,9 @@ TFA_ERR_SCALE = 10
 TFA_ERR_FLAGS = 11
 TFA_ERR_CAPTURE = 12
 TFA_ERR_SOFTCAP = 13
+TFA_ERR_SEQLENS = 14
+TFA_ERR_RING = 15
+MAX_VARLEN_SEQS = 1024
 
 TFA_DEBUG_NO_TILE_SKIP = 1
 TFA_DEBUG_MASK_ALL = 2
@@ -79,6 +82,10 @@ def lib():
             L.tfa_decode.restype = i32
             L.tfa_attention_ex.argtypes = common[:14] + [f32, P, P]
             L.tfa_attention_ex.restype = i32
+            L.tfa_prefill_ring.argtypes = [P, P, P, P] + [i32] * 7 + [f32, i32, f32, P, P]
+            L.tfa_prefill_ring.restype = i32
+            L.tfa_prefill_varlen.argtypes = [P] * 6 + [i32] * 7 + [f32, i32, i32, f32, P, P]
+            L.tfa_prefill_varlen.restype = i32
             L.tfa_check_status.argtypes = [P]
             L.tfa_check_status.restype = i32
             L.tfa_last_error.argtypes = []
@@ -114,6 +121,18 @@ def tfa_attention_ex(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key
                      sinks, stream) -> int:
     return lib().tfa_attention_ex(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask,
                                   softcap, sinks, stream)
+
+
+def tfa_prefill_ring(q, k, v, o, B, Hq, Hkv, L, S, ring_rows, D, scale, window, softcap, sinks,
+                     stream) -> int:
+    return lib().tfa_prefill_ring(q, k, v, o, B, Hq, Hkv, L, S, ring_rows, D, scale, window,
+                                  softcap, sinks, stream)
+
+
+def tfa_prefill_varlen(q, k, v, o, cu_q, cu_k, B, Hq, Hkv, total_q, total_k, max_seqlen_q, D,
+                       scale, causal, window, softcap, sinks, stream) -> int:
+    return lib().tfa_prefill_varlen(q, k, v, o, cu_q, cu_k, B, Hq, Hkv, total_q, total_k,
+                                    max_seqlen_q, D, scale, causal, window, softcap, sinks, stream)
 
 
 def tfa_prefill(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, stream) -> int:
@@ -254,6 +273,72 @@ def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=No
     rc = tfa_prefill_debug(*args, debug_flags) if debug_flags else tfa_prefill(*args)
     if rc != TFA_OK:
         raise TfaError(rc)
+    return out
+
+
+def _ptr_or_none(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def prefill_ring(q, k_ring, v_ring, *, S, window, scale=None, softcap=0.0, sinks=None, out=None,
+                 stream=None):
+    """Attention over a rotating K/V cache: k_ring/v_ring [B,Hkv,R,D] bf16 hold the
+    last R positions, position j in row j mod R; q [B,Hq,L,D] are the newest L
+    positions of S.  Causal with a window (R >= window - 1 + L, R a multiple of 64)."""
+    import torch
+
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k_ring, "k_ring", torch.bfloat16, 4)
+    _check(v_ring, "v_ring", torch.bfloat16, 4)
+    B, Hq, L, D = q.shape
+    Bk, Hkv, R, Dk = k_ring.shape
+    if tuple(v_ring.shape) != tuple(k_ring.shape) or Bk != B or Dk != D:
+        raise ValueError("q, k_ring and v_ring disagree")
+    if sinks is not None:
+        _check(sinks, "sinks", torch.float32, 1)
+    out = torch.empty_like(q) if out is None else out
+    _check(out, "out", torch.bfloat16, 4)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = tfa_prefill_ring(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k_ring.data_ptr()),
+                          ctypes.c_void_p(v_ring.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                          B, Hq, Hkv, L, int(S), R, D, float(scale), int(window), float(softcap),
+                          _ptr_or_none(sinks), _stream_handle(stream))
+    if rc != TFA_OK:
+        raise TfaError(rc, "tfa_prefill_ring")
+    return out
+
+
+def prefill_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, max_seqlen_q, scale=None, causal=True,
+                   window=0, softcap=0.0, sinks=None, out=None, stream=None):
+    """Packed variable-length attention: q [Tq,Hq,D], k/v [Tk,Hkv,D] bf16, int32 device
+    prefix sums cu_seqlens_* [B+1].  Returns out [Tq,Hq,D]."""
+    import torch
+
+    _check(q, "q", torch.bfloat16, 3)
+    _check(k, "k", torch.bfloat16, 3)
+    _check(v, "v", torch.bfloat16, 3)
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1)
+    Tq, Hq, D = q.shape
+    Tk, Hkv, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Dk != D:
+        raise ValueError("q, k and v disagree")
+    B = cu_seqlens_q.shape[0] - 1
+    if cu_seqlens_k.shape[0] != B + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    if sinks is not None:
+        _check(sinks, "sinks", torch.float32, 1)
+    out = torch.empty_like(q) if out is None else out
+    _check(out, "out", torch.bfloat16, 3)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    rc = tfa_prefill_varlen(ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+                            ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                            ctypes.c_void_p(cu_seqlens_q.data_ptr()),
+                            ctypes.c_void_p(cu_seqlens_k.data_ptr()), B, Hq, Hkv, Tq, Tk,
+                            int(max_seqlen_q), D, float(scale), int(bool(causal)), int(window),
+                            float(softcap), _ptr_or_none(sinks), _stream_handle(stream))
+    if rc != TFA_OK:
+        raise TfaError(rc, "tfa_prefill_varlen")
     return out
 
 

@@ -80,7 +80,8 @@ template <int D, bool KM, bool SC>
 int prepare_kernel(DeviceState &st) {
     using C = tfa::Cfg<D>;
     auto kern = tfa::tfa_prefill_kernel<D, KM, SC>;
-    const int smem = KM ? C::kSmemBytesKeyMask : C::kSmemBytes;
+    // the largest launch of this variant: with a key mask, or a varlen table
+    const int smem = KM ? C::kSmemBytesKeyMask : C::kSmemBytesVarlen;
     const int which = variant_index(D, KM, SC);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
@@ -198,12 +199,15 @@ int validate(const void *q, const void *k, const void *v, const void *o, int B, 
 
 // 3-D view [planes][rows][D] of a contiguous bf16 tensor, boxes of 128 rows x
 // 64 columns (128 bytes) with 128-byte swizzle; rows past the end read as 0.
+// token_major: the tensor is [rows][planes][D] (packed variable-length
+// layout), viewed with the same [plane][row][D] coordinates.
 int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D,
-               int box_rows = tfa::kBlockQ, int box_planes = 1) {
+               int box_rows = tfa::kBlockQ, int box_planes = 1, bool token_major = false) {
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                           static_cast<cuuint64_t>(planes)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2,
-                             static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(D) * 2};
+    const cuuint64_t row_bytes = static_cast<cuuint64_t>(D) * 2;
+    cuuint64_t strides[2] = {token_major ? row_bytes * static_cast<cuuint64_t>(planes) : row_bytes,
+                             token_major ? row_bytes : static_cast<cuuint64_t>(rows) * row_bytes};
     cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_planes)};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
@@ -212,28 +216,46 @@ int encode_map(CUtensorMap *m, const void *ptr, int rows, int planes, int D,
     return r == CUDA_SUCCESS ? TFA_OK : drv_fail("cuTensorMapEncodeTiled", static_cast<int>(r));
 }
 
+// How K/V (and Q/O) rows are addressed beyond the dense [B, H, len, D] layout.
+struct Addressing {
+    int ring_rows = 0;  // rotating cache: K/V [B, Hkv, ring_rows, D], key j in row j mod ring_rows
+    const int *cu_q = nullptr, *cu_k = nullptr;  // packed variable-length batch (device, [B+1])
+    int total_q = 0, total_k = 0;
+};
+
 template <int D>
 int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o, int B, int Hq,
            int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
            cudaStream_t stream, unsigned flags, SplitScratch *ss, bool force_split = false,
-           bool packed = false, float softcap = 0.f, const float *sinks = nullptr) {
+           bool packed = false, float softcap = 0.f, const float *sinks = nullptr,
+           const Addressing &ad = Addressing{}) {
     using C = tfa::Cfg<D>;
     // Short queries: a tile packs pack_heads query heads of one KV group, all L
     // rows of each (pack_heads * L <= 128), loaded as one {64, L, pack_heads} box.
     const int G = Hq / Hkv;
     const int pack_heads = packed ? (G < tfa::kBlockQ / L ? G : tfa::kBlockQ / L) : 0;
     const int pack_chunks = packed ? (G + pack_heads - 1) / pack_heads : 0;
+    const bool varlen = ad.cu_q != nullptr;
     CUtensorMap mq, mk, mv;
-    if ((packed ? encode_map(&mq, q, L, B * Hq, D, L, pack_heads) : encode_map(&mq, q, L, B * Hq, D)) ||
-        encode_map(&mk, k, S, B * Hkv, D) || encode_map(&mv, v, S, B * Hkv, D))
-        return TFA_ERR_CUDA;
+    int rc = 0;
+    if (varlen)  // packed [total, H, D]: rows are tokens, planes are heads
+        rc = encode_map(&mq, q, ad.total_q, Hq, D, tfa::kBlockQ, 1, true) ||
+             encode_map(&mk, k, ad.total_k, Hkv, D, tfa::kBlockK, 1, true) ||
+             encode_map(&mv, v, ad.total_k, Hkv, D, tfa::kBlockK, 1, true);
+    else if (ad.ring_rows)  // K/V tiles arrive as two 64-row boxes (a box never wraps)
+        rc = (packed ? encode_map(&mq, q, L, B * Hq, D, L, pack_heads) : encode_map(&mq, q, L, B * Hq, D)) ||
+             encode_map(&mk, k, ad.ring_rows, B * Hkv, D, 64) || encode_map(&mv, v, ad.ring_rows, B * Hkv, D, 64);
+    else
+        rc = (packed ? encode_map(&mq, q, L, B * Hq, D, L, pack_heads) : encode_map(&mq, q, L, B * Hq, D)) ||
+             encode_map(&mk, k, S, B * Hkv, D) || encode_map(&mv, v, S, B * Hkv, D);
+    if (rc) return TFA_ERR_CUDA;
     // separate instantiations with and without a key mask (the mask costs an
     // extra MMA per score tile and extra shared memory) and a softcap (extra
     // work per score); plain calls carry neither
     const bool sc = softcap > 0.f;
     auto kern = key_mask ? (sc ? tfa::tfa_prefill_kernel<D, true, true> : tfa::tfa_prefill_kernel<D, true, false>)
                          : (sc ? tfa::tfa_prefill_kernel<D, false, true> : tfa::tfa_prefill_kernel<D, false, false>);
-    const int smem = key_mask ? C::kSmemBytesKeyMask : C::kSmemBytes;
+    const int smem = key_mask ? C::kSmemBytesKeyMask : varlen ? C::kSmemBytesVarlen : C::kSmemBytes;
     const int which = variant_index(D, key_mask != nullptr, sc);
     if (!st.smem_attr[which]) return drv_fail("kernel not prepared", which);
     tfa::Params p;
@@ -255,6 +277,12 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.softcap_b = sc ? softcap / scale : 0.f;
     p.softcap_u = sc ? scale / softcap : 0.f;
     p.sinks = sinks;
+    p.ring_rows = ad.ring_rows;
+    p.varlen = varlen ? 1 : 0;
+    p.total_q = ad.total_q;
+    p.total_k = ad.total_k;
+    p.cu_q = ad.cu_q;
+    p.cu_k = ad.cu_k;
     p.packed = packed ? 1 : 0;
     p.pack_heads = pack_heads;
     p.pack_chunks = pack_chunks;
@@ -268,11 +296,12 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     sh.flags = flags;
     sh.n_qp = tfa::shape_n_qp(L);
     const long long n_items = static_cast<long long>(B) * sh.Hq * sh.n_qp;
-    p.W = tfa::total_steps(sh);
+    p.W = varlen ? 0 : tfa::total_steps(sh);  // varlen: per-sequence lengths live on the device
     // whole-item schedule, and the split one when scratch exists and the
     // estimate says it finishes sooner (few, large items per CTA)
     sh.split = 0;
     sh.grid = n_items < st.sm_count ? static_cast<int>(n_items) : st.sm_count;
+    if (varlen) ss = nullptr;  // whole items only (the host does not know the lengths)
     if (ss != nullptr && (n_items <= (1 << 16) || force_split)) {
         tfa::Shape sp = sh;
         sp.split = 1;
@@ -366,6 +395,71 @@ extern "C" int tfa_attention_ex(const void *q, const void *k, const void *v, voi
                                     key_mask, s, 0u, ss, false, decode, softcap, sinks)
                       : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
                                    key_mask, s, 0u, ss, false, decode, softcap, sinks);
+}
+
+extern "C" int tfa_prefill_ring(const void *q, const void *k, const void *v, void *o, int B,
+                                int Hq, int Hkv, int L, int S, int ring_rows, int D, float scale,
+                                int window, float softcap, const float *sinks, tfa_stream_t stream) {
+    const bool decode = L >= 1 && L <= TFA_MAX_DECODE_ROWS;
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, 1, window, nullptr, true, decode);
+    if (rc) return rc;
+    if (window <= 0 || ring_rows < 64 || ring_rows % 64 != 0 ||
+        static_cast<long long>(ring_rows) < static_cast<long long>(window) - 1 + L ||
+        static_cast<long long>(B) * Hkv * ring_rows > (1ll << 31) - 1)
+        return TFA_ERR_RING;
+    if (!std::isfinite(softcap) || softcap < 0.f || (softcap > 0.f && scale == 0.f)) return TFA_ERR_SOFTCAP;
+    if (sinks && (reinterpret_cast<uintptr_t>(sinks) & 3u)) return TFA_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    SplitScratch *ss = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st)) || (rc = split_scratch(*st, s, &ss))) return rc;
+    Addressing ad;
+    ad.ring_rows = ring_rows;
+    return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, 1, window, nullptr, s, 0u,
+                                    ss, false, decode, softcap, sinks, ad)
+                      : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, 1, window, nullptr, s, 0u,
+                                   ss, false, decode, softcap, sinks, ad);
+}
+
+extern "C" int tfa_prefill_varlen(const void *q, const void *k, const void *v, void *o,
+                                  const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int Hq,
+                                  int Hkv, int total_q, int total_k, int max_seqlen_q, int D,
+                                  float scale, int causal, int window, float softcap,
+                                  const float *sinks, tfa_stream_t stream) {
+    if (total_q == 0) return TFA_OK;  // no query row: nothing is read or written
+    if (!q || !k || !v || !o || !cu_seqlens_q || !cu_seqlens_k) return TFA_ERR_NULL;
+    if (Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return TFA_ERR_HEADS;
+    if (B < 1 || B > tfa::kMaxVarlenSeqs || total_q < 0 || total_k < 0 || max_seqlen_q < 0 ||
+        max_seqlen_q > (1 << 30) || static_cast<long long>(total_q) * Hq > (1ll << 31) - 1 ||
+        static_cast<long long>(total_k) * Hkv > (1ll << 31) - 1)
+        return TFA_ERR_SHAPE;
+    if (D != 64 && D != 128) return TFA_ERR_HEAD_DIM;
+    if (window > 0 && !causal) return TFA_ERR_WINDOW;
+    auto mis = [](const void *p, unsigned a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; };
+    if (mis(q, 16) || mis(k, 16) || mis(v, 16) || mis(o, 16) || mis(cu_seqlens_q, 4) ||
+        mis(cu_seqlens_k, 4) || (sinks && mis(sinks, 4)))
+        return TFA_ERR_ALIGN;
+    if (!std::isfinite(scale)) return TFA_ERR_SCALE;
+    if (!std::isfinite(softcap) || softcap < 0.f || (softcap > 0.f && scale == 0.f)) return TFA_ERR_SOFTCAP;
+    if (max_seqlen_q == 0) return TFA_ERR_SHAPE;  // query rows exist, so some sequence has one
+    if (total_k == 0) return TFA_ERR_SHAPE;  // keys are read through a map over k: it needs rows
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    int rc = device_state(s, &st);
+    if (rc) return rc;
+    Addressing ad;
+    ad.cu_q = cu_seqlens_q;
+    ad.cu_k = cu_seqlens_k;
+    ad.total_q = total_q;
+    ad.total_k = total_k;
+    return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, max_seqlen_q, max_seqlen_q, scale,
+                                    causal, window, nullptr, s, 0u, nullptr, false, false, softcap,
+                                    sinks, ad)
+                      : launch<64>(*st, q, k, v, o, B, Hq, Hkv, max_seqlen_q, max_seqlen_q, scale,
+                                   causal, window, nullptr, s, 0u, nullptr, false, false, softcap,
+                                   sinks, ad);
 }
 
 extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o, int B,
@@ -467,7 +561,7 @@ int take_status_word(unsigned *status) {
     if (word == 0) return TFA_OK;
     if (cudaMemset(status, 0, sizeof word) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess)
         return TFA_ERR_CUDA;
-    return TFA_ERR_TIMEOUT;
+    return (word & tfa::TFA_DEVICE_TIMEOUT) ? TFA_ERR_TIMEOUT : TFA_ERR_SEQLENS;
 }
 }  // namespace
 
@@ -538,6 +632,8 @@ extern "C" const char *tfa_status_string(int status) {
         case TFA_ERR_SCALE: return "scale must be finite";
         case TFA_ERR_CAPTURE: return "first use of a device or stream inside a CUDA graph capture";
         case TFA_ERR_SOFTCAP: return "softcap must be finite and >= 0 (and needs a nonzero scale)";
+        case TFA_ERR_SEQLENS: return "inconsistent cu_seqlens in a variable-length call; its output is invalid";
+        case TFA_ERR_RING: return "ring cache needs a window, ring_rows a multiple of 64 and >= window - 1 + L";
         case TFA_ERR_FLAGS: return "unknown debug flags";
         default: return "unknown status";
     }

@@ -93,6 +93,8 @@ constexpr int kPolyPeriod = TFA_POLY_PERIOD;
 constexpr int kPartKeys = 96;
 static_assert(kPartKeys % 32 == 0 && kPartKeys % 16 == 0 && kPartKeys < 128, "P split");
 
+constexpr int kMaxVarlenSeqs = 1024;  // sequences per packed variable-length call
+
 template <int D>
 struct Cfg {
     static_assert(D == 64 || D == 128, "head dim");
@@ -116,6 +118,11 @@ struct Cfg {
     static constexpr int kBiasOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
     static constexpr int kOnesOff = kBiasOff + kSlots * kBiasBytes;
     static constexpr int kSmemBytesKeyMask = kOnesOff + kBiasBytes + 1024;
+    // Packed variable-length calls: per sequence q_start, q_len, k_start,
+    // k_len (validated copies of cu_seqlens), in place of the key-mask blocks
+    // (the two never meet).
+    static constexpr int kTableOff = kBiasOff;
+    static constexpr int kSmemBytesVarlen = kTableOff + 16 * kMaxVarlenSeqs + 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kTmemS = 0;                 // S_t at kTmemS + 128 t
     static constexpr uint32_t kTmemO = 256;               // O_t at kTmemO + D t
@@ -134,6 +141,14 @@ struct Params {
     // odd Taylor series of tanh through u^7 below (no cancellation near 0)
     float softcap_a, softcap_b, softcap_u;
     const float *sinks;  // fp32 [Hq] sink logits, or nullptr
+    // rotating cache: K/V hold ring_rows rows and key position j sits in row
+    // j mod ring_rows (0: K/V hold all S keys in order)
+    int ring_rows;
+    // packed variable-length batch: q/o [total_q, Hq, D], k/v [total_k, Hkv, D],
+    // sequence b = rows [cu_q[b], cu_q[b+1]) / [cu_k[b], cu_k[b+1]); shape.L is
+    // the longest query (max_seqlen_q)
+    int varlen, total_q, total_k;
+    const int *cu_q, *cu_k;
     // split schedule: ctl[0] counts finished launches (the epoch of a launch is
     // ctl[0] + 1, read from device memory so a captured graph replays correctly),
     // ctl[1] counts the CTAs of the running launch that have finished
@@ -182,8 +197,30 @@ __device__ __forceinline__ unsigned launch_epoch(const unsigned *ctl) {
     return e == 0u ? 1u : e;
 }
 
+// The CTA's dynamic shared memory, 1 KB aligned (the same base the kernel uses).
+__device__ __forceinline__ uint8_t *smem_base() {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    return smem_raw + (((raw + 1023u) & ~1023u) - raw);
+}
+
+// Start the CTA's piece iterator (with the validated sequence table for a
+// packed variable-length call).
+template <int D>
+__device__ __forceinline__ void iter_init(SegIter &it, const Params &p) {
+    it.init(p.shape, p.W, blockIdx.x);
+    if (p.varlen) {
+        const int *tab = reinterpret_cast<const int *>(smem_base() + Cfg<D>::kTableOff);
+        it.seq.q_start = tab;
+        it.seq.q_len = tab + kMaxVarlenSeqs;
+        it.seq.k_start = tab + 2 * kMaxVarlenSeqs;
+        it.seq.k_len = tab + 3 * kMaxVarlenSeqs;
+    }
+}
+
 struct ItemPlan {
     int b, h, g;
+    int q_row0, k_row0;  // varlen: the sequence's first packed query / key row
     int q0[2];
     bool present[2];
     int lo[2], hi[2];
@@ -198,7 +235,9 @@ __device__ __forceinline__ ItemPlan plan_piece(const Params &p, const Segment &s
     ip.g = p.packed ? seg.h / p.pack_chunks : seg.h / p.G;
     ip.jl = seg.jb;
     ip.jh = seg.je;
-    const ItemSpan sp = item_span(p.shape, seg.qp);
+    ip.q_row0 = seg.q_base;
+    ip.k_row0 = seg.k_base;
+    const ItemSpan sp = seg_span(p.shape, seg);
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const TileRole tr = tile_role(p.shape, seg, sp, t);
@@ -245,7 +284,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
     uint32_t kv_prod = 0;
     uint32_t q_use[2] = {0, 0};
     SegIter it;
-    it.init(p.shape, p.W, blockIdx.x);
+    iter_init<D>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
         const ItemPlan ip = plan_piece(p, seg);
@@ -262,11 +301,12 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
                                     tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0);
-                } else {
+                } else {  // dense: plane b*Hq + h; varlen: packed rows, plane h
                     mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
+                    const int plane = p.varlen ? ip.h : ip.b * p.Hq + ip.h;
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
-                                    tm_q, bar.q_full(t), cb * 64, ip.q0[t], ip.b * p.Hq + ip.h);
+                                    tm_q, bar.q_full(t), cb * 64, ip.q_row0 + ip.q0[t], plane);
                 }
             }
             ++q_use[t];
@@ -294,10 +334,22 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                 }
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bar.kv_full(s), C::kTileBytes);
-                    for (int cb = 0; cb < C::kColBlocks; ++cb)
-                        tma_load_3d(sbase + C::kKVOff + s * C::kTileBytes + cb * C::kColBlockBytes,
-                                    which ? tm_v : tm_k, bar.kv_full(s), cb * 64, j * kBlockK,
-                                    ip.b * p.Hkv + ip.g);
+                    const uint32_t dst = sbase + C::kKVOff + s * C::kTileBytes;
+                    if (p.ring_rows) {
+                        // rotating cache: two 64-row boxes, each contiguous in
+                        // the ring (ring_rows is a multiple of 64)
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int row = (j * kBlockK + 64 * hf) % p.ring_rows;
+                            for (int cb = 0; cb < C::kColBlocks; ++cb)
+                                tma_load_3d(dst + cb * C::kColBlockBytes + hf * 64 * 128, which ? tm_v : tm_k,
+                                            bar.kv_full(s), cb * 64, row, ip.b * p.Hkv + ip.g);
+                        }
+                    } else {
+                        const int plane = p.varlen ? ip.g : ip.b * p.Hkv + ip.g;
+                        for (int cb = 0; cb < C::kColBlocks; ++cb)
+                            tma_load_3d(dst + cb * C::kColBlockBytes, which ? tm_v : tm_k, bar.kv_full(s),
+                                        cb * 64, ip.k_row0 + j * kBlockK, plane);
+                    }
                 }
                 ++kv_prod;
             }
@@ -372,7 +424,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     int trace_step = 0;
     (void)trace_step;
     SegIter it;
-    it.init(p.shape, p.W, blockIdx.x);
+    iter_init<D>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
         const ItemPlan ip = plan_piece(p, seg);
@@ -475,16 +527,16 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     (void)trace_step;
 
     SegIter it;
-    it.init(p.shape, p.W, blockIdx.x);
+    iter_init<D>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
-        const ItemSpan sp = item_span(p.shape, seg.qp);
+        const ItemSpan sp = seg_span(p.shape, seg);
         const TileRole ip = tile_role(p.shape, seg, sp, t);
         if (!ip.active) continue;
         // query row of this thread (its head too, for a packed tile)
         int row = seg.qp * 2 * kBlockQ + t * kBlockQ + r;
         int out_head = seg.h;
-        bool row_valid = row < p.L;
+        bool row_valid = row < seg.L;
         const int q_tile0 = row - r;  // first row of the tile, for the tile-level mask test
         if (p.packed) {
             const PackedRows pr = packed_rows(p, seg.h);
@@ -492,8 +544,8 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             out_head = pr.h0 + r / p.L;
             row_valid = r < pr.heads * p.L;
         }
-        const int pos = (p.S - p.L) + row;  // absolute position of this query row
-        const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
+        const int pos = (seg.S - seg.L) + row;  // absolute position of this query row
+        const int hi_abs = p.causal ? imin(pos, seg.S - 1) : seg.S - 1;
         const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
         float m_ref = -CUDART_INF_F;  // row maximum the exponentials are taken against
         float l = 0.f;
@@ -529,7 +581,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             }
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 0);
 
-            if (key_tile_needs_mask(p.L, p.S, p.causal, p.window, 0, q_tile0, j, p.flags)) {
+            if (key_tile_needs_mask(seg.L, seg.S, p.causal, p.window, 0, q_tile0, j, p.flags)) {
                 const int k0 = j * kBlockK;
                 const int lo_c = lo_abs - k0;
                 const int hi_c = hi_abs - k0;
@@ -641,7 +693,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 
         // Rows of this tile that hold a query row: a packed tile fills
         // heads * L of its 128 rows, a prefill tile ends at row L.
-        const int n_valid = p.packed ? packed_rows(p, seg.h).heads * p.L : imin(kBlockQ, p.L - q_tile0);
+        const int n_valid = p.packed ? packed_rows(p, seg.h).heads * p.L : imin(kBlockQ, seg.L - q_tile0);
         const bool warp_live = (r & ~31) < n_valid;  // warp-uniform: tcgen05.ld is warp-collective
         const bool row_live = r < n_valid;
 
@@ -717,9 +769,11 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         if (!warp_live) continue;
         if (row_live) l = add_sink(p, l, m_star, c, out_head);  // m_star == m_ref for a whole tile
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        __nv_bfloat16 *orow = row_valid
-            ? p.o + (static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row) * static_cast<size_t>(D)
-            : nullptr;
+        __nv_bfloat16 *orow = nullptr;
+        if (row_valid)  // dense [B,Hq,L,D]; varlen packed [total_q, Hq, D]
+            orow = p.o + (p.varlen ? static_cast<size_t>(seg.q_base + row) * p.Hq + out_head
+                                   : static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row) *
+                             static_cast<size_t>(D);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
@@ -811,6 +865,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = lane; n < 128; n += 32)
             *reinterpret_cast<uint16_t *>(gbase + C::kOnesOff + bias_offset(n, 0)) = 0x3F80u;
         fence_proxy_async_smem();
+    }
+    if (p.varlen && warp < 8) {
+        // validated copy of cu_seqlens; a bad sequence is skipped and reported
+        int *tab = reinterpret_cast<int *>(gbase + C::kTableOff);
+        for (int b = threadIdx.x; b < p.B; b += 256) {
+            const int q0 = __ldg(p.cu_q + b), q1 = __ldg(p.cu_q + b + 1);
+            const int k0 = __ldg(p.cu_k + b), k1 = __ldg(p.cu_k + b + 1);
+            const bool ok = q0 >= 0 && q1 >= q0 && q1 <= p.total_q && k0 >= 0 && k1 >= k0 &&
+                            k1 <= p.total_k && q1 - q0 <= p.shape.L && (!p.causal || k1 - k0 >= q1 - q0);
+            tab[b] = q0;
+            tab[kMaxVarlenSeqs + b] = ok ? q1 - q0 : 0;
+            tab[2 * kMaxVarlenSeqs + b] = k0;
+            tab[3 * kMaxVarlenSeqs + b] = k1 - k0;
+            if (!ok && blockIdx.x == 0) atomicOr(p.status, TFA_DEVICE_BAD_SEQLENS);
+        }
     }
     if (warp == 8 && lane == 0) {
         prefetch_tensormap(&tm_q);

@@ -14,6 +14,10 @@ namespace tfa {
 
 constexpr long long TFA_WAIT_LIMIT_CYCLES = 8ll << 30;  // ~4 s at 2 GHz
 constexpr unsigned TFA_DEVICE_TIMEOUT = 1u;
+// A packed variable-length call met a sequence whose cu_seqlens entries are
+// inconsistent (decreasing, past the packed length, longer than max_seqlen_q,
+// or a causal sequence with fewer keys than queries); its rows are not written.
+constexpr unsigned TFA_DEVICE_BAD_SEQLENS = 2u;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
     unsigned long long t;

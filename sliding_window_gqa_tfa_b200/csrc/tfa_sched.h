@@ -27,8 +27,15 @@
 
 namespace tfa {
 
+// Packed variable-length batches: sequence b has q_len[b] query rows from
+// packed row q_start[b] and k_len[b] keys from packed row k_start[b] (a
+// sequence whose lengths failed validation has q_len 0 and is skipped).
+struct SeqTable {
+    const int *q_start, *q_len, *k_start, *k_len;
+};
+
 struct Shape {
-    int B, Hq, L, S, causal, window;
+    int B, Hq, L, S, causal, window;  // varlen: L = longest query, S unused
     unsigned flags;
     int n_qp;   // query-tile pairs per head: ceil(L / 256)
     int grid;   // CTAs
@@ -44,14 +51,14 @@ struct ItemSpan {
     bool present[2];
 };
 
-TFA_HD ItemSpan item_span(const Shape &s, int qp) {
+TFA_HD ItemSpan item_span_ls(const Shape &s, int L, int S, int qp) {
     ItemSpan sp;
     sp.jl = 0x7fffffff;
     sp.jh = -1;
     for (int t = 0; t < 2; ++t) {
         const int q0 = qp * 2 * kBlockQ + t * kBlockQ;
-        sp.present[t] = q0 < s.L;
-        const KeyRange kr = qtile_key_range(s.L, s.S, s.causal, s.window, q0, s.flags);
+        sp.present[t] = q0 < L;
+        const KeyRange kr = qtile_key_range(L, S, s.causal, s.window, q0, s.flags);
         sp.lo[t] = kr.lo;
         sp.hi[t] = sp.present[t] ? kr.hi : -1;
         if (sp.present[t]) {
@@ -61,6 +68,8 @@ TFA_HD ItemSpan item_span(const Shape &s, int qp) {
     }
     return sp;
 }
+
+TFA_HD ItemSpan item_span(const Shape &s, int qp) { return item_span_ls(s, s.L, s.S, qp); }
 
 // Items of group r all have query-tile pair group_qp(r).
 TFA_HD int group_qp(const Shape &s, int r) { return s.causal ? s.n_qp - 1 - r : r; }
@@ -84,7 +93,12 @@ struct Segment {
     int qp, b, h;
     int jb, je;     // key tiles [jb, je] of this piece
     long long x0;   // global index of the item's first step (split schedule)
+    int L, S;       // the item's query rows and keys (the call's, or its sequence's)
+    int q_base, k_base;  // varlen: first packed query / key row of the sequence
 };
+
+// Key-tile ranges of the segment's query-tile pair, for its own lengths.
+TFA_HD ItemSpan seg_span(const Shape &s, const Segment &seg) { return item_span_ls(s, seg.L, seg.S, seg.qp); }
 
 // Per-CTA iterator over its pieces, identical on every role of the CTA.
 struct SegIter {
@@ -92,8 +106,10 @@ struct SegIter {
     long long gstart;     // split: first global step of group r
     int r, gsteps, bh;    // split: current group, steps per item in it, items per group
     int item, stride, n_items;  // whole-item schedule
+    SeqTable seq;  // varlen batches (whole-item schedule only); q_start == nullptr otherwise
 
     TFA_HD void init(const Shape &s, long long W, int c) {
+        seq.q_start = seq.q_len = seq.k_start = seq.k_len = nullptr;
         bh = s.B * s.Hq;
         n_items = s.n_qp * bh;
         item = c;
@@ -114,18 +130,31 @@ struct SegIter {
 
     TFA_HD bool next(const Shape &s, Segment &seg) {
         if (!s.split) {
-            if (item >= n_items) return false;
-            const int rr = item / bh, rem = item - rr * bh;
-            seg.item = item;
-            seg.qp = group_qp(s, rr);
-            seg.b = rem / s.Hq;
-            seg.h = rem - seg.b * s.Hq;
-            const ItemSpan sp = item_span(s, seg.qp);
-            seg.jb = sp.jl;
-            seg.je = sp.jh;
-            seg.x0 = 0;
-            item += stride;
-            return true;
+            for (;;) {
+                if (item >= n_items) return false;
+                const int rr = item / bh, rem = item - rr * bh;
+                seg.item = item;
+                seg.qp = group_qp(s, rr);
+                seg.b = rem / s.Hq;
+                seg.h = rem - seg.b * s.Hq;
+                item += stride;
+                seg.L = s.L;
+                seg.S = s.S;
+                seg.q_base = 0;
+                seg.k_base = 0;
+                if (seq.q_start) {  // varlen: the sequence's own lengths
+                    seg.L = seq.q_len[seg.b];
+                    seg.S = seq.k_len[seg.b];
+                    seg.q_base = seq.q_start[seg.b];
+                    seg.k_base = seq.k_start[seg.b];
+                    if (seg.qp * 2 * kBlockQ >= seg.L) continue;  // no such tile pair
+                }
+                const ItemSpan sp = seg_span(s, seg);
+                seg.jb = sp.jl;
+                seg.je = sp.jh;
+                seg.x0 = 0;
+                return true;
+            }
         }
         if (pos >= end) return false;
         while (pos >= gstart + static_cast<long long>(bh) * gsteps) {
@@ -141,6 +170,10 @@ struct SegIter {
         seg.qp = group_qp(s, r);
         seg.b = rem / s.Hq;
         seg.h = rem - seg.b * s.Hq;
+        seg.L = s.L;
+        seg.S = s.S;
+        seg.q_base = 0;
+        seg.k_base = 0;
         const ItemSpan sp = item_span(s, seg.qp);
         seg.jb = sp.jl + static_cast<int>(pos - x0);
         seg.je = sp.jl + static_cast<int>(stop - x0) - 1;

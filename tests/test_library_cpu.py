@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings():
-    for code in range(14):
+    for code in range(16):
         s = tb.status_string(code)
         assert s and s != "unknown status"
     assert tb.status_string(99) == "unknown status"
@@ -85,6 +85,36 @@ def _call_ex(**over):
 ])
 def test_score_variant_rejections_happen_before_launch(over, code):
     assert _call_ex(**over) == code
+
+
+def test_ring_rejections_happen_before_launch():
+    a = dict(q=A16, k=A16, v=A16, o=A16, B=1, Hq=8, Hkv=2, L=33, S=5000, ring_rows=1088, D=128,
+             scale=0.088, window=1024, softcap=0.0, sinks=None, stream=None)
+    assert tb.tfa_prefill_ring(**{**a, "window": 0}) == tb.TFA_ERR_RING
+    assert tb.tfa_prefill_ring(**{**a, "ring_rows": 1000}) == tb.TFA_ERR_RING   # not a multiple of 64
+    assert tb.tfa_prefill_ring(**{**a, "ring_rows": 1024}) == tb.TFA_ERR_RING   # < 1023 + 33
+    assert tb.tfa_prefill_ring(**{**a, "S": 20}) == tb.TFA_ERR_SHAPE            # S < L
+    assert tb.tfa_prefill_ring(**{**a, "Hq": 7}) == tb.TFA_ERR_HEADS
+    assert tb.tfa_prefill_ring(**{**a, "softcap": -2.0}) == tb.TFA_ERR_SOFTCAP
+    assert tb.tfa_prefill_ring(**{**a, "k": MIS}) == tb.TFA_ERR_ALIGN
+
+
+def test_varlen_rejections_happen_before_launch():
+    a = dict(q=A16, k=A16, v=A16, o=A16, cu_q=A16, cu_k=A16, B=3, Hq=8, Hkv=2, total_q=100,
+             total_k=300, max_seqlen_q=60, D=128, scale=0.088, causal=1, window=0, softcap=0.0,
+             sinks=None, stream=None)
+    assert tb.tfa_prefill_varlen(**{**a, "total_q": 0, "q": None}) == tb.TFA_OK  # nothing to do
+    assert tb.tfa_prefill_varlen(**{**a, "cu_k": None}) == tb.TFA_ERR_NULL
+    assert tb.tfa_prefill_varlen(**{**a, "Hkv": 3}) == tb.TFA_ERR_HEADS
+    assert tb.tfa_prefill_varlen(**{**a, "B": 0}) == tb.TFA_ERR_SHAPE
+    assert tb.tfa_prefill_varlen(**{**a, "B": tb.MAX_VARLEN_SEQS + 1}) == tb.TFA_ERR_SHAPE
+    assert tb.tfa_prefill_varlen(**{**a, "max_seqlen_q": 0}) == tb.TFA_ERR_SHAPE
+    assert tb.tfa_prefill_varlen(**{**a, "total_k": 0}) == tb.TFA_ERR_SHAPE
+    assert tb.tfa_prefill_varlen(**{**a, "D": 96}) == tb.TFA_ERR_HEAD_DIM
+    assert tb.tfa_prefill_varlen(**{**a, "causal": 0, "window": 5}) == tb.TFA_ERR_WINDOW
+    assert tb.tfa_prefill_varlen(**{**a, "cu_q": ctypes.c_void_p(0x10002)}) == tb.TFA_ERR_ALIGN
+    assert tb.tfa_prefill_varlen(**{**a, "scale": float("nan")}) == tb.TFA_ERR_SCALE
+    assert tb.tfa_prefill_varlen(**{**a, "softcap": float("inf")}) == tb.TFA_ERR_SOFTCAP
 
 
 def test_debug_rejects_unknown_flags_before_launch():
