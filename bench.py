@@ -3,8 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one launch (tfa_prefill; tfa_decode when L <= 8) over the whole workload (every query row of
-every head).  Inputs are seeded synthetic bf16 tensors resident in HBM before
+One step = one launch over the whole workload (every query row of every head):
+tfa_prefill (tfa_decode when L <= 8; tfa_attention_ex with a softcap or
+sinks; tfa_prefill_ring for a rotating cache; tfa_prefill_varlen for a packed
+variable-length batch).  Inputs are seeded synthetic bf16 tensors resident in HBM before
 the timed region; L2 is flushed (256 MiB memset) between steps, outside each
 step's CUDA events.  Prints one JSON line on rank 0.
 
@@ -33,8 +35,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sliding_window_gqa_tfa_b200 import binding as tb  # noqa: E402
-from sliding_window_gqa_tfa_b200.flops import algorithmic_bytes, useful_flops  # noqa: E402
-from sliding_window_gqa_tfa_b200.inputs import HEADLINE, WORKLOADS, make_inputs, make_sinks  # noqa: E402
+from sliding_window_gqa_tfa_b200.flops import workload_bytes, workload_flops  # noqa: E402
+from sliding_window_gqa_tfa_b200.inputs import (HEADLINE, WORKLOADS, make_inputs,  # noqa: E402
+                                                make_sinks, varlen_cu)
 
 METRIC = "prefill attention TFLOP/s (unmasked pairs) and % of B200 BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -168,37 +171,76 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
-def oracle_rows_flops(w, rows):
-    """Useful flops of the given flattened rows (host arithmetic, 4*D per allowed key)."""
-    i = rows % w.L
-    P = w.S - w.L
-    if w.causal:
-        last = P + i
-        first = np.maximum(0, last - w.window + 1) if w.window > 0 else np.zeros_like(i)
-        keys = last - first + 1
+def rows_flops(L, S, causal, window, D, i):
+    """Useful flops of query rows i (0 <= i < L) of one head: 4*D per key the row
+    may see under causal/window (a key mask is ignored in the count)."""
+    P = S - L
+    if causal:
+        last = np.minimum(P + i, S - 1)
+        first = np.maximum(0, last - window + 1) if window > 0 else np.zeros_like(i)
+        keys = np.maximum(last - first + 1, 0)
     else:
-        keys = np.full_like(i, w.S)
-    return int(keys.sum()) * 4 * w.D
+        keys = np.full_like(i, S)
+    return int(keys.sum()) * 4 * D
 
 
-def cpu_baseline(w, q, k, v, km, budget_s=12.0):
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "S": w.S, "D": w.D,
+            "causal": w.causal, "window": w.window, "key_mask": w.key_mask_keep is not None,
+            "softcap": w.softcap, "sinks": w.sink_scale is not None, "ring_rows": w.ring_rows,
+            "varlen_tokens": sum(L for L, _ in w.seqlens) if w.seqlens else None}
+
+
+class OracleSampler:
+    """Bounded units of the fp64 oracle's work on a workload: a few random query
+    rows (of a random sequence, for a packed variable-length workload)."""
+
+    def __init__(self, w, seed=0):
+        import oracle
+
+        oracle.build()
+        self.oracle, self.w = oracle, w
+        self.q, self.k, self.v, self.km = make_inputs(w, seed=seed)
+        self.sinks = make_sinks(w, seed=seed)
+        if w.kind == "varlen":
+            self.cq, self.ck = varlen_cu(w)
+            self.live = [b for b, (L, _) in enumerate(w.seqlens) if L > 0]
+        self.n_rows = w.B * w.Hq * w.L
+
+    def unit(self, rng, n):
+        """Run the oracle on n random rows; return their useful flops."""
+        w, o = self.w, self.oracle
+        kw = dict(scale=w.softmax_scale, window=w.window, softcap=w.softcap, sinks=self.sinks)
+        if w.kind == "varlen":
+            # one sequence through the dense oracle (the varlen definition per sequence)
+            b = int(rng.choice(self.live))
+            L, S = w.seqlens[b]
+            qb = self.q[self.cq[b]:self.cq[b + 1]].transpose(0, 1)[None].contiguous()
+            kb = self.k[self.ck[b]:self.ck[b + 1]].transpose(0, 1)[None].contiguous()
+            vb = self.v[self.ck[b]:self.ck[b + 1]].transpose(0, 1)[None].contiguous()
+            rows = np.sort(rng.choice(w.Hq * L, size=min(n, w.Hq * L), replace=False)).astype(np.int64)
+            o.attention(qb, kb, vb, causal=w.causal, rows=rows, **kw)
+            return rows_flops(L, S, w.causal, w.window, w.D, rows % L)
+        rows = np.sort(rng.choice(self.n_rows, size=min(n, self.n_rows), replace=False)).astype(np.int64)
+        if w.kind == "ring":
+            o.attention_ring(self.q, self.k, self.v, S=w.S, rows=rows, **kw)
+        else:
+            o.attention(self.q, self.k, self.v, causal=w.causal, key_mask=self.km, rows=rows, **kw)
+        return rows_flops(w.L, w.S, w.causal, w.window, w.D, rows % w.L)
+
+
+def cpu_baseline(w, budget_s=12.0):
     """The fp64 oracle as it stands, on the host cores, over a bounded row sample."""
-    import oracle
-
-    oracle.build()
+    sampler = OracleSampler(w, seed=0)
     rng = np.random.default_rng(0)
-    n_rows = w.B * w.Hq * w.L
     chunk = 64
     done_rows, flops, t0 = 0, 0, time.perf_counter()
     while time.perf_counter() - t0 < budget_s:
-        rows = np.sort(rng.choice(n_rows, size=chunk, replace=False)).astype(np.int64)
-        oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                         key_mask=km, softcap=w.softcap, sinks=make_sinks(w, 0), rows=rows)
+        flops += sampler.unit(rng, chunk)
         done_rows += chunk
-        flops += oracle_rows_flops(w, rows)
     dt = time.perf_counter() - t0
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"{done_rows} random query rows of {w.name} (of {n_rows}), fp64, "
+            "sample": f"{done_rows} random query rows of {w.name} (of {sampler.n_rows}), fp64, "
                       f"{dt:.1f} s wall; flops counted as 4*D per key the row may see "
                       f"(key mask ignored in the count)"}
 
@@ -208,24 +250,17 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    import oracle
-
-    oracle.build()
-    q, k, v, km = make_inputs(w, seed=0)
-    sinks = make_sinks(w, seed=0)
+    sampler = OracleSampler(w, seed=0)
     rng = np.random.default_rng(1)
-    n_rows = w.B * w.Hq * w.L
     per_step = 32
     times, flops = [], []
     for step in range(args.warmup + args.steps):
-        rows = np.sort(rng.choice(n_rows, size=per_step, replace=False)).astype(np.int64)
         t0 = time.perf_counter()
-        oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                         key_mask=km, softcap=w.softcap, sinks=sinks, rows=rows)
+        f = sampler.unit(rng, per_step)
         dt = time.perf_counter() - t0
         if step >= args.warmup:
             times.append(dt)
-            flops.append(oracle_rows_flops(w, rows))
+            flops.append(f)
     total_t = sum(times)
     value = sum(flops) / total_t / 1e12
     sample = (f"each step: {per_step} random query rows of {w.name} through the fp64 oracle "
@@ -234,10 +269,7 @@ def run_reference(args, w):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total_t / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L,
-                       "S": w.S, "D": w.D, "causal": w.causal, "window": w.window,
-                       "key_mask": w.key_mask_keep is not None, "softcap": w.softcap,
-                       "sinks": w.sink_scale is not None, "sample_rows_per_step": per_step},
+            "config": {**workload_config(w), "sample_rows_per_step": per_step},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -269,18 +301,30 @@ def main():
 
     q, k, v, km = make_inputs(w, seed=rank)
     sinks = make_sinks(w, seed=rank)
-    dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
-    dkm = km.to(dev) if km is not None else None
-    dsinks = sinks.to(dev) if sinks is not None else None
-    variant = w.softcap > 0 or sinks is not None  # score variants: tfa_attention_ex
-    out = torch.empty_like(dq)
-    flops = useful_flops(w.B, w.Hq, w.L, w.S, w.D, causal=w.causal, window=w.window, key_mask=km)
+    cu = tuple(torch.from_numpy(c) for c in varlen_cu(w)) if w.kind == "varlen" else ()
+    host_inputs = [q, k, v, km, sinks, *cu]  # what one call reads (None: absent)
+    dev_inputs = [t.to(dev) if t is not None else None for t in host_inputs]
+    out = torch.empty_like(dev_inputs[0])
+    flops = workload_flops(w, key_mask=km)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    def call(ins, o):
+        """One launch on the current stream: the entry point the workload needs."""
+        dq, dk, dv, dkm, dsinks = ins[:5]
+        if w.kind == "varlen":
+            tb.prefill_varlen(dq, dk, dv, ins[5], ins[6], max_seqlen_q=w.L, scale=w.softmax_scale,
+                              causal=w.causal, window=w.window, softcap=w.softcap, sinks=dsinks,
+                              out=o)
+        elif w.kind == "ring":
+            tb.prefill_ring(dq, dk, dv, S=w.S, window=w.window, scale=w.softmax_scale,
+                            softcap=w.softcap, sinks=dsinks, out=o)
+        else:
+            tb.prefill(dq, dk, dv, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                       key_mask=dkm, out=o, softcap=w.softcap, sinks=dsinks)
+
     def step():
-        tb.prefill(dq, dk, dv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                   key_mask=dkm, out=out, softcap=w.softcap, sinks=dsinks)
+        call(dev_inputs, out)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -309,26 +353,24 @@ def main():
     per_sorted = sorted(per)
 
     # end to end through the C ABI with host buffers (copies inside the timed region)
-    hq, hk, hv = q.pin_memory(), k.pin_memory(), v.pin_memory()
-    hkm = km.pin_memory() if km is not None else None
+    pinned = [t.pin_memory() if t is not None else None for t in host_inputs]
+    hq, hk, hv, hkm = pinned[:4]
     hout = torch.empty_like(hq).pin_memory()
-    hsinks = sinks.pin_memory() if sinks is not None else None
-    if variant:
-        # tfa_attention_ex takes device pointers: the step copies the pinned
-        # inputs in, calls it, and copies the output back, all on `stream`
-        eq, ek, ev = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
-        ekm = torch.empty_like(dkm) if dkm is not None else None
-        esinks = torch.empty_like(dsinks) if dsinks is not None else None
-        eout = torch.empty_like(dq)
+    if w.kind != "dense" or w.softcap > 0 or sinks is not None:
+        # the device entry points: the step copies the pinned inputs in, calls
+        # the entry point, and copies the output back, all on `stream`
+        staged = [torch.empty_like(t) if t is not None else None for t in dev_inputs]
+        eout = torch.empty_like(out)
 
         def e2e_step():
-            for d, h in ((eq, hq), (ek, hk), (ev, hv), (ekm, hkm), (esinks, hsinks)):
+            for d, h in zip(staged, pinned):
                 if d is not None:
                     d.copy_(h, non_blocking=True)
-            tb.prefill(eq, ek, ev, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                       key_mask=ekm, out=eout, softcap=w.softcap, sinks=esinks)
+            call(staged, eout)
             hout.copy_(eout, non_blocking=True)
-        e2e_api = "tfa_attention_ex (pinned host buffers, copies on the stream)"
+        entry = {"varlen": "tfa_prefill_varlen", "ring": "tfa_prefill_ring"}.get(w.kind,
+                                                                                  "tfa_attention_ex")
+        e2e_api = f"{entry} (pinned host buffers, copies on the stream)"
     else:
         def e2e_step():
             tb.prefill_host(hq, hk, hv, scale=w.softmax_scale, causal=w.causal, window=w.window,
@@ -346,12 +388,11 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2 + (hkm.numel() * 4 if hkm is not None else 0) \
-        + (hsinks.numel() * 4 if hsinks is not None else 0)
+    h2d = sum(t.numel() * t.element_size() for t in pinned if t is not None)
     d2h = hout.numel() * 2
 
     peaks, peak_kind = load_peaks()
-    alg_bytes = algorithmic_bytes(w.B, w.Hq, w.Hkv, w.L, w.S, w.D, key_mask=km is not None)
+    alg_bytes = workload_bytes(w)
     if w.L <= tb.MAX_DECODE_ROWS:
         # short queries read every K/V byte for a few flops: bounded by HBM
         bound, roof_unit = "hbm", "GB/s"
@@ -371,10 +412,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L,
-                       "S": w.S, "D": w.D, "causal": w.causal, "window": w.window,
-                       "key_mask": w.key_mask_keep is not None, "softcap": w.softcap,
-                       "sinks": w.sink_scale is not None, "useful_gflop": flops / 1e9,
+            "config": {**workload_config(w), "useful_gflop": flops / 1e9,
                        "l2": "flushed between steps (256 MiB memset outside the step events)",
                        "parallelism": f"weak x{world}" if world > 1 else "single GPU"},
             "ms_p10": per_sorted[len(per) // 10], "ms_p50": per_sorted[len(per) // 2],
@@ -393,7 +431,7 @@ def main():
             "wall_s_timed_region": t_wall,
         }
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline(w, q, k, v, km)
+            line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -37,3 +37,24 @@ def useful_flops(B, Hq, L, S, D, *, causal, window=0, key_mask=None) -> int:
 def algorithmic_bytes(B, Hq, Hkv, L, S, D, *, key_mask=False) -> int:
     """Q read + O written once, K and V read once (bf16); key mask read once."""
     return 2 * D * (2 * B * Hq * L + 2 * B * Hkv * S) + (4 * B * S if key_mask else 0)
+
+
+def workload_flops(w, key_mask=None) -> int:
+    """Useful flops of one call on workload w (dense, rotating cache or packed
+    variable-length): 4*D per allowed pair, summed per sequence for varlen."""
+    if w.seqlens is not None:
+        return sum(useful_flops(1, w.Hq, L, S, w.D, causal=w.causal, window=w.window)
+                   for L, S in w.seqlens)
+    return useful_flops(w.B, w.Hq, w.L, w.S, w.D, causal=w.causal, window=w.window,
+                        key_mask=key_mask)
+
+
+def workload_bytes(w) -> int:
+    """Algorithmic bytes of one call: Q read and O written once, the K/V rows that
+    exist read once (the ring's rows for a rotating cache), the key mask once."""
+    if w.seqlens is not None:
+        Tq = sum(L for L, _ in w.seqlens)
+        Tk = sum(S for _, S in w.seqlens)
+        return 2 * w.D * (2 * Tq * w.Hq + 2 * Tk * w.Hkv)
+    S = min(w.S, w.ring_rows) if w.ring_rows else w.S
+    return algorithmic_bytes(w.B, w.Hq, w.Hkv, w.L, S, w.D, key_mask=w.key_mask_keep is not None)

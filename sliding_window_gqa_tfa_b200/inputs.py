@@ -41,6 +41,15 @@ class Workload:
     scale: float | None = None  # None: 1/sqrt(D)
     softcap: float = 0.0        # 0: none
     sink_scale: float | None = None  # None: no sinks; else sinks ~ sink_scale * N(0, 1)
+    # rotating cache: K/V hold ring_rows rows, position j in row j mod ring_rows
+    ring_rows: int = 0
+    # packed variable-length batch: ((L_b, S_b), ...) per sequence; B = len(seqlens),
+    # L / S = the longest query / key count
+    seqlens: tuple | None = None
+
+    @property
+    def kind(self) -> str:
+        return "varlen" if self.seqlens is not None else "ring" if self.ring_rows else "dense"
 
     @property
     def softmax_scale(self) -> float:
@@ -53,6 +62,10 @@ class Workload:
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
 
+
+# Prompt lengths of the variable-length workload (a fixed draw, uniform in [256, 4096]).
+_VARLEN16 = (3184, 1291, 2869, 417, 3977, 2050, 733, 1504, 256, 3511, 1876, 988, 4096, 2290, 612, 1362)
+_VARLEN16_MAX = max(_VARLEN16)
 
 WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     # 33 query rows over 47 keys (prefix 14): crosses both tile tails.
@@ -76,6 +89,15 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
              k_scale=4.0, softcap=50.0),
     Workload("llama_gqa_chunk_2048x8192_sinks", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
              sink_scale=2.0),
+    # Rotating cache of TensorFold's sliding layer (WINDOW 1024, RING 1088): 16
+    # sequences 32K tokens in, a 64-row chunk each, and 64 sequences decoding.
+    Workload("swa_ring_r1088_chunk64_b16", B=16, Hq=32, Hkv=8, L=64, S=32768, D=128, window=1024,
+             ring_rows=1088),
+    Workload("swa_ring_r1088_decode_b64", B=64, Hq=32, Hkv=8, L=1, S=32768, D=128, window=1024,
+             ring_rows=1088),
+    # Packed variable-length prefill of 16 Qwen3-shaped prompts (256..4096 tokens).
+    Workload("varlen_qwen3_16seqs", B=16, Hq=16, Hkv=8, L=_VARLEN16_MAX, S=_VARLEN16_MAX, D=128,
+             seqlens=tuple((n, n) for n in _VARLEN16)),
     # Short queries (1 <= L <= 8): token-by-token decoding over a long cache,
     # batched Qwen3-shaped decoding, and an 8-row chunk (e.g. draft verification).
     Workload("llama_gqa_decode_1x32768", B=1, Hq=56, Hkv=8, L=1, S=32768, D=128),
@@ -91,9 +113,20 @@ HEADLINE = "llama_gqa_chunk_2048x8192"
 
 def make_inputs(w: Workload, seed: int = 0):
     """Return (q, k, v, key_mask) as CPU tensors: bf16 [B,Hq,L,D], bf16 [B,Hkv,S,D] x2,
-    and fp32 [B,S] (or None).  Sink logits, when the workload has them, come from
-    make_sinks with the same seed."""
+    and fp32 [B,S] (or None).  A rotating-cache workload's k/v are the ring contents
+    [B,Hkv,ring_rows,D]; a variable-length workload's are packed: q [sum L_b, Hq, D],
+    k/v [sum S_b, Hkv, D] (see varlen_cu).  Sink logits, when the workload has
+    them, come from make_sinks with the same seed."""
     return _draw(w, seed)[:4]
+
+
+def varlen_cu(w: Workload):
+    """int32 prefix sums (cu_seqlens_q, cu_seqlens_k) of a variable-length workload."""
+    import numpy as np
+
+    cq = np.concatenate([[0], np.cumsum([L for L, _ in w.seqlens])]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum([S for _, S in w.seqlens])]).astype(np.int32)
+    return cq, ck
 
 
 def make_sinks(w: Workload, seed: int = 0):
@@ -104,9 +137,15 @@ def make_sinks(w: Workload, seed: int = 0):
 
 def _draw(w: Workload, seed: int):
     g = torch.Generator().manual_seed(seed)
-    q = torch.randn(w.B, w.Hq, w.L, w.D, generator=g, dtype=torch.float32)
-    k = torch.randn(w.B, w.Hkv, w.S, w.D, generator=g, dtype=torch.float32)
-    v = torch.randn(w.B, w.Hkv, w.S, w.D, generator=g, dtype=torch.float32)
+    if w.seqlens is not None:
+        q_shape = (sum(L for L, _ in w.seqlens), w.Hq, w.D)
+        kv_shape = (sum(S for _, S in w.seqlens), w.Hkv, w.D)
+    else:
+        q_shape = (w.B, w.Hq, w.L, w.D)
+        kv_shape = (w.B, w.Hkv, w.ring_rows if w.ring_rows else w.S, w.D)
+    q = torch.randn(*q_shape, generator=g, dtype=torch.float32)
+    k = torch.randn(*kv_shape, generator=g, dtype=torch.float32)
+    v = torch.randn(*kv_shape, generator=g, dtype=torch.float32)
     if w.k_scale != 1.0:
         k = k * w.k_scale
     key_mask = None

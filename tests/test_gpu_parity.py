@@ -187,7 +187,8 @@ def _sample_rows(w, n_per_head=24, seed=0):
     return np.array(rows, dtype=np.int64)
 
 
-@pytest.mark.parametrize("name", [n for n in WORKLOADS if n != "witness_33x47"])
+@pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items()
+                                  if n != "witness_33x47" and w.kind == "dense"])
 def test_parity_full_size_sampled(name):
     w = WORKLOADS[name]
     o, (q, k, v, km) = _run(w, seed=0)

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 from sliding_window_gqa_tfa_b200 import binding as tb
-from sliding_window_gqa_tfa_b200.inputs import make_inputs, make_sinks, shaped
+from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_inputs, make_sinks, shaped, varlen_cu
 
 pytestmark = pytest.mark.gpu
 
@@ -157,3 +157,43 @@ def test_varlen_empty_and_rejected_calls():
                           torch.tensor([0, 5], dtype=torch.int32, device="cuda"), max_seqlen_q=3,
                           causal=False, window=4)
     assert e.value.code == tb.TFA_ERR_WINDOW
+
+
+@pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items() if w.kind != "dense"])
+def test_full_size_workloads_sampled(name):
+    """The benchmark's rotating-cache and variable-length workloads, launched as
+    the benchmark launches them, on rows the oracle computes one by one."""
+    w = WORKLOADS[name]
+    q, k, v, _ = make_inputs(w, seed=0)
+    sinks = make_sinks(w, seed=0)
+    rng = np.random.default_rng(5)
+    if w.kind == "ring":
+        o = tb.prefill_ring(q.cuda(), k.cuda(), v.cuda(), S=w.S, window=w.window,
+                            scale=w.softmax_scale, softcap=w.softcap,
+                            sinks=sinks.cuda() if sinks is not None else None)
+        tb.check_status()
+        n = w.B * w.Hq * w.L
+        rows = np.unique(np.concatenate([[0, n - 1], rng.choice(n, size=min(n, 600), replace=False)]))
+        ref = oracle.attention_ring(q, k, v, S=w.S, scale=w.softmax_scale, window=w.window,
+                                    softcap=w.softcap, sinks=sinks, rows=rows)
+        got = o.reshape(-1, w.D)[torch.as_tensor(rows, device=o.device)]
+        _assert_close(got, ref, name)
+        return
+    cq, ck = varlen_cu(w)
+    o = tb.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cq).cuda(),
+                          torch.from_numpy(ck).cuda(), max_seqlen_q=w.L, scale=w.softmax_scale,
+                          causal=w.causal, window=w.window, softcap=w.softcap,
+                          sinks=sinks.cuda() if sinks is not None else None)
+    tb.check_status()
+    for b in [0, 4, 8, 12, len(w.seqlens) - 1]:  # sampled rows of several sequences
+        L, S = w.seqlens[b]
+        qb = q[cq[b]:cq[b + 1]].transpose(0, 1)[None].contiguous()
+        kb = k[ck[b]:ck[b + 1]].transpose(0, 1)[None].contiguous()
+        vb = v[ck[b]:ck[b + 1]].transpose(0, 1)[None].contiguous()
+        i = np.unique(np.concatenate([[0, 127, 128, L - 1], rng.choice(L, size=min(L, 24), replace=False)]))
+        i = i[i < L]
+        rows = (np.arange(w.Hq)[:, None] * L + i[None, :]).reshape(-1)
+        ref = oracle.attention(qb, kb, vb, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                               softcap=w.softcap, sinks=sinks, rows=rows)
+        got = o[cq[b]:cq[b + 1]].transpose(0, 1).reshape(-1, w.D)[torch.as_tensor(rows, device=o.device)]
+        _assert_close(got, ref, f"{name} sequence {b}")
