@@ -40,6 +40,8 @@ MUTATIONS = {
 # Planted mistakes of the rotating-cache and packed variable-length entry points.
 RING_MUTATIONS = {"ring_slot_shifted": 11}
 VARLEN_MUTATIONS = {"varlen_packed_causal": 12, "head_modulo": 3, "no_prefix_offset": 4}
+BACKWARD_MUTATIONS = {"bwd_no_delta": 13, "bwd_dk_no_scale": 14, "bwd_dq_uses_v": 15,
+                      "head_modulo": 3, "causal_sees_next": 1, "keymask_inverted": 6}
 
 
 def build(force: bool = False) -> str:
@@ -78,6 +80,11 @@ def _load():
             lib.oracle_attention_varlen_mutant.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32,
                                                            f64, i32, i32, i32]
             lib.oracle_attention_varlen_mutant.restype = i32
+            lib.oracle_attention_backward.argtypes = [P] * 7 + [i32] * 6 + [f64, i32, i32, P, i32]
+            lib.oracle_attention_backward.restype = i32
+            lib.oracle_attention_backward_mutant.argtypes = [P] * 7 + [i32] * 6 + [f64, i32, i32, P,
+                                                                                 i32]
+            lib.oracle_attention_backward_mutant.restype = i32
             lib.oracle_attention_mutant.restype = i32
             lib.oracle_softmax_weights.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                    i32, i32, P, i32, i32, i32]
@@ -239,6 +246,28 @@ def attention_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale, causal, wind
     if rc:
         raise ValueError(f"oracle_attention_varlen rejected its arguments (code {rc})")
     return out
+
+
+def attention_backward(q, k, v, dout, *, scale, causal, window=0, key_mask=None, threads=0,
+                       mutation=0):
+    """Gradients (dq [B,Hq,L,D], dk, dv [B,Hkv,S,D], float64) of the plain definition
+    for the upstream gradient dout [B,Hq,L,D] (bf16)."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    if db.shape != qb.shape or vb.shape != kb.shape:
+        raise ValueError("dout must match q, v must match k")
+    km = _mask(key_mask)
+    dq = np.empty(qb.shape, dtype=np.float64)
+    dk = np.empty(kb.shape, dtype=np.float64)
+    dv = np.empty(kb.shape, dtype=np.float64)
+    code = BACKWARD_MUTATIONS[mutation] if isinstance(mutation, str) else int(mutation)
+    args = (_ptr(qb), _ptr(kb), _ptr(vb), _ptr(db), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, L, S,
+            D, float(scale), int(bool(causal)), int(window), _ptr(km))
+    rc = (_load().oracle_attention_backward_mutant(*args, code) if code
+          else _load().oracle_attention_backward(*args, int(threads)))
+    if rc:
+        raise ValueError(f"oracle_attention_backward rejected its arguments (code {rc})")
+    return dq, dk, dv
 
 
 def attention_blockwise(q, k, v, *, scale, causal, window=0, key_mask=None, bq=128, bk=128,

@@ -80,6 +80,9 @@ enum {
     MUT_SINK_IN_NUMERATOR = 10,  /* sink weight also added to every output   */
     MUT_RING_SLOT_SHIFTED = 11,  /* key j read from ring row (j + 1) mod R   */
     MUT_VARLEN_PACKED_CAUSAL = 12,/* causal test on packed token indices      */
+    MUT_BWD_NO_DELTA = 13,       /* dS = P dP, without the row term          */
+    MUT_BWD_DK_NO_SCALE = 14,    /* dK without the softmax scale             */
+    MUT_BWD_DQ_USES_V = 15,      /* dQ accumulates dS V instead of dS K      */
 };
 
 static double bf16_bits_to_f64(uint16_t bits)
@@ -459,6 +462,124 @@ int oracle_softmax_weights(const uint16_t *q, const uint16_t *k, double *W,
             for (long j = 0; j < S; ++j) wr[j] /= denom;
     }
     return 0;
+}
+
+/* Gradients of the plain definition with respect to q, k and v, for an
+ * upstream gradient dout of the output (brotensor flash_attention.h,
+ * flash_attention_backward and flash_attention_varlen_backward comments: the
+ * backward of the bare attention core, recompute-based; causal- and
+ * mask-excluded positions contribute nothing to any gradient).  With
+ * s = scale q.k over the allowed keys, P the softmax of each row (a row with
+ * no allowed key has P = 0 and output 0) and O = P V:
+ *   dV[b,g,j]   = sum over the group's heads h and rows i of P[h,i,j] dout[h,i]
+ *   dP[h,i,j]   = dout[h,i] . v[g,j]
+ *   dS[h,i,j]   = P[h,i,j] (dP[h,i,j] - sum_j' P[h,i,j'] dP[h,i,j'])
+ *   dQ[b,h,i]   = scale sum_j dS[h,i,j] k[g,j]
+ *   dK[b,g,j]   = scale sum over h, i of dS[h,i,j] q[h,i]
+ * (the softmax Jacobian: d softmax_j / d s_j' = P_j (delta_jj' - P_j')).
+ * Inputs bf16 bits, upcast exactly; dout likewise; outputs fp64 in the input
+ * layouts.  Parallel over (b, g): one thread owns a KV head's dK/dV. */
+static int backward_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                         const uint16_t *dout, double *dq, double *dk, double *dv, int B, int Hq,
+                         int Hkv, int L, int S, int D, double scale, int causal, int window,
+                         const float *key_mask, int nthreads, int mutation)
+{
+    int rc = check_args(q, k, v, dq, B, Hq, Hkv, L, S, D);
+    if (rc) return rc;
+    if (!dout || !dk || !dv) return 1;
+    memset(dq, 0, sizeof(double) * (size_t)B * Hq * L * D);
+    memset(dk, 0, sizeof(double) * (size_t)B * Hkv * S * D);
+    memset(dv, 0, sizeof(double) * (size_t)B * Hkv * S * D);
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)S);
+        double *dP = (double *)malloc(sizeof(double) * (size_t)S);
+        if (!P || !dP) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+            if (!P || !dP) continue;
+            const int b = (int)(bg / Hkv), g = (int)(bg % Hkv);
+            const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+            const uint16_t *kb = k + ((size_t)b * Hkv + g) * (size_t)S * D;
+            const uint16_t *vb = v + ((size_t)b * Hkv + g) * (size_t)S * D;
+            double *dkb = dk + ((size_t)b * Hkv + g) * (size_t)S * D;
+            double *dvb = dv + ((size_t)b * Hkv + g) * (size_t)S * D;
+            for (int h = 0; h < Hq; ++h) {
+                if (kv_head_impl(h, Hq, Hkv, mutation) != g) continue;
+                for (long i = 0; i < L; ++i) {
+                    const size_t row = (((size_t)b * Hq + h) * L + i) * D;
+                    const uint16_t *qr = q + row, *dor = dout + row;
+                    double m = -INFINITY;
+                    for (long j = 0; j < S; ++j) {
+                        P[j] = -INFINITY;
+                        if (!allowed_impl(L, S, i, j, causal, window, mrow, mutation)) continue;
+                        double acc = 0.0;
+                        for (int d = 0; d < D; ++d)
+                            acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kb[(size_t)j * D + d]);
+                        P[j] = scale * acc;
+                        if (P[j] > m) m = P[j];
+                    }
+                    if (m == -INFINITY) continue;  /* no allowed key: no gradient */
+                    double denom = 0.0;
+                    for (long j = 0; j < S; ++j) {
+                        P[j] = (P[j] == -INFINITY) ? 0.0 : exp(P[j] - m);
+                        denom += P[j];
+                    }
+                    double delta = 0.0;  /* sum_j P_j dP_j */
+                    for (long j = 0; j < S; ++j) {
+                        P[j] /= denom;
+                        dP[j] = 0.0;
+                        if (P[j] == 0.0) continue;
+                        for (int d = 0; d < D; ++d)
+                            dP[j] += bf16_bits_to_f64(dor[d]) * bf16_bits_to_f64(vb[(size_t)j * D + d]);
+                        delta += P[j] * dP[j];
+                    }
+                    if (mutation == MUT_BWD_NO_DELTA) delta = 0.0;
+                    const double ks = (mutation == MUT_BWD_DK_NO_SCALE) ? 1.0 : scale;
+                    const uint16_t *qsrc = (mutation == MUT_BWD_DQ_USES_V) ? vb : kb;
+                    for (long j = 0; j < S; ++j) {
+                        if (P[j] == 0.0) continue;
+                        const double ds = P[j] * (dP[j] - delta);
+                        for (int d = 0; d < D; ++d) {
+                            dvb[(size_t)j * D + d] += P[j] * bf16_bits_to_f64(dor[d]);
+                            dkb[(size_t)j * D + d] += ks * ds * bf16_bits_to_f64(qr[d]);
+                            dq[row + d] += scale * ds * bf16_bits_to_f64(qsrc[(size_t)j * D + d]);
+                        }
+                    }
+                }
+            }
+        }
+        free(P);
+        free(dP);
+    }
+    return failed ? 5 : 0;
+}
+
+int oracle_attention_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                              const uint16_t *dout, double *dq, double *dk, double *dv, int B,
+                              int Hq, int Hkv, int L, int S, int D, double scale, int causal,
+                              int window, const float *key_mask, int nthreads)
+{
+    return backward_impl(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, D, scale, causal, window,
+                         key_mask, nthreads, MUT_NONE);
+}
+
+int oracle_attention_backward_mutant(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                     const uint16_t *dout, double *dq, double *dk, double *dv,
+                                     int B, int Hq, int Hkv, int L, int S, int D, double scale,
+                                     int causal, int window, const float *key_mask, int mutation)
+{
+    return backward_impl(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, D, scale, causal, window,
+                         key_mask, 1, mutation);
 }
 
 /* Brute-force count of allowed (b, h, i, j) quadruples: the "unmasked pairs"

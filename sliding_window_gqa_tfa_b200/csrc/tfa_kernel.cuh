@@ -661,6 +661,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             // keys [0, kPartKeys): publish, then the rest
 #pragma unroll
             for (int i = 0; i < kPartKeys / 2; ++i) TFA_EXP_PAIR(i);
+            if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 3);
 #pragma unroll
             for (int c32 = 0; c32 < kPartKeys / 64; ++c32) tmem_st32(tP + 32 * c32, pk + 32 * c32);
             if ((kPartKeys / 2) % 32) tmem_st16(tP + (kPartKeys / 64) * 32, pk + (kPartKeys / 64) * 32);
@@ -668,8 +669,10 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.p_part(t));
+            if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 4);
 #pragma unroll
             for (int i = kPartKeys / 2; i < 64; ++i) TFA_EXP_PAIR(i);
+            if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 5);
 #undef TFA_EXP_PAIR
 #undef TFA_F
             const float2 acc = add2(acc0, acc1);
