@@ -193,6 +193,27 @@ int tfa_prefill_varlen(const void *q, const void *k, const void *v, void *o,
                        int causal, int window, float softcap, const float *sinks,
                        tfa_stream_t stream);
 
+/* tfa_prefill_backward -- gradients of the attention core (brotensor
+ * flash_attention.h, flash_attention_backward: the backward of the bare
+ * core, recompute-based, consuming no forward caches; causal- and
+ * mask-excluded positions contribute nothing to any gradient).
+ *   q, k, v, key_mask, sizes, scale, causal, window: as for tfa_prefill
+ *            (any L >= 1; L <= 8 recomputes through tfa_decode's path)
+ *   dout     upstream gradient of the output, bf16 [B, Hq, L, D]
+ *   dq       bf16 [B, Hq, L, D]; dk, dv bf16 [B, Hkv, S, D] -- overwritten
+ *            (dk, dv summed over the query heads of each KV group)
+ * All caller-owned device memory, 16-byte aligned (else TFA_ERR_ALIGN;
+ * TFA_ERR_NULL for a NULL gradient pointer).  With P the softmax weights and
+ * dP = dout V^T: dS = P (dP - rowsum(dout o O)), dq = scale dS K,
+ * dk = scale dS^T Q, dv = P^T dout.  The call re-runs the forward (its output
+ * and per-row log-sum-exp go to a per-stream workspace of 2 B Hq L (D + 4)
+ * bytes, grown on demand; growth during graph capture returns
+ * TFA_ERR_CAPTURE), then three kernels, all asynchronous on `stream`. */
+int tfa_prefill_backward(const void *q, const void *k, const void *v, const void *dout,
+                         void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int L, int S,
+                         int D, float scale, int causal, int window, const float *key_mask,
+                         tfa_stream_t stream);
+
 /* Debug flags for tfa_prefill_debug. */
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
 #define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */
@@ -271,6 +292,14 @@ const char *tfa_status_string(int status);
  * error for the sizes.  No device work. */
 int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_mask, int qtile,
                    int *kt_lo, int *kt_hi, unsigned char *needs_mask, int needs_mask_len);
+
+/* tfa_plan_ktile -- host view of the backward pass's enumeration for one
+ * 128-key tile (keys [128*ktile, min(128*ktile+128, S))): the first and last
+ * 128-row query tile holding a row that may see one of its keys under the
+ * causal mask and the window (*qt_hi < *qt_lo: no row sees the tile, and its
+ * key and value gradients are zero).  Returns TFA_OK, TFA_ERR_SHAPE for an
+ * out-of-range tile, or a validation error for the sizes.  No device work. */
+int tfa_plan_ktile(int L, int S, int causal, int window, int ktile, int *qt_lo, int *qt_hi);
 
 /* tfa_plan_pieces -- host view of the work one CTA of a grid of `grid` CTAs
  * performs (no device work).  The work of (batch, query head, pair of 128-row

@@ -82,6 +82,8 @@ def lib():
             L.tfa_decode.restype = i32
             L.tfa_attention_ex.argtypes = common[:14] + [f32, P, P]
             L.tfa_attention_ex.restype = i32
+            L.tfa_prefill_backward.argtypes = [P] * 7 + [i32] * 6 + [f32, i32, i32, P, P]
+            L.tfa_prefill_backward.restype = i32
             L.tfa_prefill_ring.argtypes = [P, P, P, P] + [i32] * 7 + [f32, i32, f32, P, P]
             L.tfa_prefill_ring.restype = i32
             L.tfa_prefill_varlen.argtypes = [P] * 6 + [i32] * 7 + [f32, i32, i32, f32, P, P]
@@ -95,6 +97,8 @@ def lib():
             L.tfa_plan_qtile.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.POINTER(i32),
                                          ctypes.POINTER(i32), P, i32]
             L.tfa_plan_qtile.restype = i32
+            L.tfa_plan_ktile.argtypes = [i32] * 5 + [ctypes.POINTER(i32), ctypes.POINTER(i32)]
+            L.tfa_plan_ktile.restype = i32
             L.tfa_plan_pieces.argtypes = [i32] * 9 + [P, i32, ctypes.POINTER(i32),
                                                       ctypes.POINTER(ctypes.c_longlong)]
             L.tfa_plan_pieces.restype = i32
@@ -177,6 +181,13 @@ def tfa_plan_qtile(L, S, causal, window, has_key_mask, qtile):
     if rc:
         return rc, None, None, None
     return rc, lo.value, hi.value, [bool(buf[i]) for i in range(hi.value - lo.value + 1)]
+
+
+def tfa_plan_ktile(L, S, causal, window, ktile):
+    """(status, first query tile, last query tile) that see key tile `ktile`."""
+    lo, hi = ctypes.c_int(0), ctypes.c_int(0)
+    rc = lib().tfa_plan_ktile(L, S, int(bool(causal)), window, ktile, ctypes.byref(lo), ctypes.byref(hi))
+    return rc, lo.value, hi.value
 
 
 def tfa_plan_pieces(B, Hq, L, S, causal, window, grid, split, cta, max_pieces=4096):
@@ -274,6 +285,35 @@ def prefill(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=No
     if rc != TFA_OK:
         raise TfaError(rc)
     return out
+
+
+def tfa_prefill_backward(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, D, scale, causal, window,
+                         key_mask, stream) -> int:
+    return lib().tfa_prefill_backward(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, D, scale, causal,
+                                      window, key_mask, stream)
+
+
+def backward(q, k, v, dout, *, scale=None, causal=True, window=0, key_mask=None, stream=None):
+    """(dq, dk, dv) bf16 of the attention core for the upstream gradient dout
+    [B,Hq,L,D] (recompute-based: the forward is re-run inside)."""
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
+        _check(t, n, torch.bfloat16, 4)
+    B, Hq, L, D = q.shape
+    Bk, Hkv, S, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or tuple(dout.shape) != tuple(q.shape) or Bk != B or Dk != D:
+        raise ValueError("q, k, v and dout disagree")
+    if key_mask is not None:
+        _check(key_mask, "key_mask", torch.float32, 2)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc = tfa_prefill_backward(*(ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, dout, dq, dk, dv)),
+                              B, Hq, Hkv, L, S, D, float(scale), int(bool(causal)), int(window),
+                              _ptr_or_none(key_mask), _stream_handle(stream))
+    if rc != TFA_OK:
+        raise TfaError(rc, "tfa_prefill_backward")
+    return dq, dk, dv
 
 
 def _ptr_or_none(t):

@@ -18,6 +18,7 @@
 #include <cudaTypedefs.h>
 
 #include "../../include/tfa.h"
+#include "tfa_bwd.cuh"
 #include "tfa_kernel.cuh"
 
 namespace {
@@ -33,12 +34,22 @@ struct SplitScratch {
     unsigned *ctl = nullptr;
 };
 
+// Workspace of the backward pass, per (device, stream), grown on demand: the
+// recomputed forward output and per-row log-sum-exp, and delta = rowsum(dO o O).
+struct BwdScratch {
+    void *o = nullptr;
+    float *lse = nullptr, *delta = nullptr;
+    size_t rows = 0, o_bytes = 0;
+};
+
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
     unsigned *status = nullptr;  // device status word (TFA_DEVICE_TIMEOUT bits)
     bool smem_attr[8] = {};  // per kernel variant: D, key mask, softcap
     std::unordered_map<cudaStream_t, SplitScratch> split;
+    std::unordered_map<cudaStream_t, BwdScratch> bwd;
+    bool bwd_attr[4] = {};  // backward kernels prepared, per (D, key mask)
     // staging buffers of tfa_prefill_host
     void *h_buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
     size_t h_cap[5] = {0, 0, 0, 0, 0};
@@ -100,6 +111,17 @@ int prepare_kernel(DeviceState &st) {
     return TFA_OK;
 }
 
+template <int D, bool KM>
+int prepare_bwd_kernels(DeviceState &st) {
+    const int smem = tfa::bwd::Cfg<D>::kSmemBytes;
+    cudaError_t e = cudaFuncSetAttribute(tfa::bwd::dq_kernel<D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tfa::bwd::dkv_kernel<D, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(backward smem)", e);
+    st.bwd_attr[(D == 128 ? 2 : 0) + (KM ? 1 : 0)] = true;
+    return TFA_OK;
+}
+
 int prepare_all_kernels(DeviceState &st) {
     int rc = prepare_kernel<64, false, false>(st);
     if (!rc) rc = prepare_kernel<64, true, false>(st);
@@ -109,6 +131,10 @@ int prepare_all_kernels(DeviceState &st) {
     if (!rc) rc = prepare_kernel<128, true, false>(st);
     if (!rc) rc = prepare_kernel<128, false, true>(st);
     if (!rc) rc = prepare_kernel<128, true, true>(st);
+    if (!rc) rc = prepare_bwd_kernels<64, false>(st);
+    if (!rc) rc = prepare_bwd_kernels<64, true>(st);
+    if (!rc) rc = prepare_bwd_kernels<128, false>(st);
+    if (!rc) rc = prepare_bwd_kernels<128, true>(st);
     return rc;
 }
 
@@ -172,6 +198,33 @@ int split_scratch(DeviceState &st, cudaStream_t stream, SplitScratch **out) {
     return TFA_OK;
 }
 
+// The backward workspace for `stream`, at least `rows` rows of D columns.
+int bwd_scratch(DeviceState &st, cudaStream_t stream, size_t rows, int D, BwdScratch **out) {
+    BwdScratch &bs = st.bwd[stream];
+    const size_t o_bytes = rows * static_cast<size_t>(D) * 2;
+    if (bs.rows < rows || bs.o_bytes < o_bytes) {
+        if (int rc = refuse_under_capture(stream, "a larger backward workspace")) return rc;
+        cudaFree(bs.o);
+        cudaFree(bs.lse);
+        cudaFree(bs.delta);
+        bs = BwdScratch{};
+        cudaError_t e = cudaMalloc(&bs.o, o_bytes);
+        if (e == cudaSuccess) e = cudaMalloc(&bs.lse, rows * sizeof(float));
+        if (e == cudaSuccess) e = cudaMalloc(&bs.delta, rows * sizeof(float));
+        if (e != cudaSuccess) {
+            cudaFree(bs.o);
+            cudaFree(bs.lse);
+            cudaFree(bs.delta);
+            bs = BwdScratch{};
+            return cuda_fail("cudaMalloc(backward workspace)", e);
+        }
+        bs.rows = rows;
+        bs.o_bytes = o_bytes;
+    }
+    *out = &bs;
+    return TFA_OK;
+}
+
 int validate(const void *q, const void *k, const void *v, const void *o, int B, int Hq, int Hkv,
              int L, int S, int D, float scale, int causal, int window, const float *key_mask,
              bool check_pointers, bool decode = false) {
@@ -221,6 +274,7 @@ struct Addressing {
     int ring_rows = 0;  // rotating cache: K/V [B, Hkv, ring_rows, D], key j in row j mod ring_rows
     const int *cu_q = nullptr, *cu_k = nullptr;  // packed variable-length batch (device, [B+1])
     int total_q = 0, total_k = 0;
+    float *lse = nullptr;  // optional per-row log-sum-exp output (dense layout only)
 };
 
 template <int D>
@@ -283,6 +337,7 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.total_k = ad.total_k;
     p.cu_q = ad.cu_q;
     p.cu_k = ad.cu_k;
+    p.lse = ad.lse;
     p.packed = packed ? 1 : 0;
     p.pack_heads = pack_heads;
     p.pack_chunks = pack_chunks;
@@ -462,6 +517,91 @@ extern "C" int tfa_prefill_varlen(const void *q, const void *k, const void *v, v
                                    sinks, ad);
 }
 
+namespace {
+// Backward: a forward recompute (output and log-sum-exp into the workspace),
+// delta = rowsum(dO o O), then the dQ and the dK/dV kernels, all on `stream`.
+template <int D>
+int backward_impl(DeviceState &st, SplitScratch *ss, BwdScratch &bs, const void *q, const void *k,
+                  const void *v, const void *dout, void *dq, void *dk, void *dv, int B, int Hq,
+                  int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
+                  cudaStream_t stream) {
+    namespace bw = tfa::bwd;
+    const bool decode = L <= TFA_MAX_DECODE_ROWS;
+    Addressing ad;
+    ad.lse = bs.lse;
+    int rc = launch<D>(st, q, k, v, bs.o, B, Hq, Hkv, L, S, scale, causal, window, key_mask, stream, 0u,
+                       ss, false, decode, 0.f, nullptr, ad);
+    if (rc) return rc;
+    const long long rows = static_cast<long long>(B) * Hq * L;
+    const long long threads = rows * 32;
+    bw::delta_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(bs.o), static_cast<const __nv_bfloat16 *>(dout), bs.delta, rows);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("delta kernel launch", e);
+    CUtensorMap mq, mdo, mk, mv;
+    if (encode_map(&mq, q, L, B * Hq, D) || encode_map(&mdo, dout, L, B * Hq, D) ||
+        encode_map(&mk, k, S, B * Hkv, D) || encode_map(&mv, v, S, B * Hkv, D))
+        return TFA_ERR_CUDA;
+    if (!st.bwd_attr[(D == 128 ? 2 : 0) + (key_mask ? 1 : 0)]) return drv_fail("backward kernel not prepared", D);
+    bw::BwdParams p;
+    p.dq = static_cast<__nv_bfloat16 *>(dq);
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.lse = bs.lse;
+    p.delta = bs.delta;
+    p.key_mask = key_mask;
+    p.status = st.status;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.L = L;
+    p.S = S;
+    p.G = Hq / Hkv;
+    p.causal = causal ? 1 : 0;
+    p.window = (causal && window > 0) ? window : 0;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const int smem = bw::Cfg<D>::kSmemBytes;
+    const long long nq_items = static_cast<long long>(B) * Hq * ((L + tfa::kBlockQ - 1) / tfa::kBlockQ);
+    p.n_items = static_cast<int>(nq_items);
+    auto dq_kern = key_mask ? bw::dq_kernel<D, true> : bw::dq_kernel<D, false>;
+    dq_kern<<<static_cast<int>(nq_items < st.sm_count ? nq_items : st.sm_count), bw::kThreads, smem, stream>>>(
+        mq, mdo, mk, mv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail("dQ kernel launch", e);
+    const long long nk_items = static_cast<long long>(B) * Hkv * ((S + tfa::kBlockK - 1) / tfa::kBlockK);
+    p.n_items = static_cast<int>(nk_items);
+    auto dkv_kern = key_mask ? bw::dkv_kernel<D, true> : bw::dkv_kernel<D, false>;
+    dkv_kern<<<static_cast<int>(nk_items < st.sm_count ? nk_items : st.sm_count), bw::kThreads, smem, stream>>>(
+        mq, mdo, mk, mv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail("dK/dV kernel launch", e);
+    return TFA_OK;
+}
+}  // namespace
+
+extern "C" int tfa_prefill_backward(const void *q, const void *k, const void *v, const void *dout,
+                                    void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int L,
+                                    int S, int D, float scale, int causal, int window,
+                                    const float *key_mask, tfa_stream_t stream) {
+    const bool decode = L >= 1 && L <= TFA_MAX_DECODE_ROWS;
+    int rc = validate(q, k, v, dout, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true, decode);
+    if (rc) return rc;
+    if (!dq || !dk || !dv) return TFA_ERR_NULL;
+    auto mis16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+    if (mis16(dq) || mis16(dk) || mis16(dv)) return TFA_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    SplitScratch *ss = nullptr;
+    BwdScratch *bs = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st)) || (rc = split_scratch(*st, s, &ss)) ||
+        (rc = bwd_scratch(*st, s, static_cast<size_t>(B) * Hq * L, D, &bs)))
+        return rc;
+    return (D == 128) ? backward_impl<128>(*st, ss, *bs, q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, scale,
+                                           causal, window, key_mask, s)
+                      : backward_impl<64>(*st, ss, *bs, q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, scale,
+                                          causal, window, key_mask, s);
+}
+
 extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o, int B,
                                  int Hq, int Hkv, int L, int S, int D, float scale, int causal,
                                  int window, const float *key_mask, tfa_stream_t stream,
@@ -637,6 +777,19 @@ extern "C" const char *tfa_status_string(int status) {
         case TFA_ERR_FLAGS: return "unknown debug flags";
         default: return "unknown status";
     }
+}
+
+extern "C" int tfa_plan_ktile(int L, int S, int causal, int window, int ktile, int *qt_lo,
+                              int *qt_hi) {
+    int rc = validate(nullptr, nullptr, nullptr, nullptr, 1, 1, 1, L, S, 128, 1.0f, causal, window,
+                      nullptr, false, L < TFA_MIN_QUERY_ROWS);
+    if (rc) return rc;
+    if (!qt_lo || !qt_hi) return TFA_ERR_NULL;
+    if (ktile < 0 || ktile * tfa::kBlockK >= S) return TFA_ERR_SHAPE;
+    const tfa::KeyRange r = tfa::ktile_query_range(L, S, causal, causal ? window : 0, ktile);
+    *qt_lo = r.lo;
+    *qt_hi = r.hi;
+    return TFA_OK;
 }
 
 extern "C" int tfa_plan_qtile(int L, int S, int causal, int window, int has_key_mask, int qtile,

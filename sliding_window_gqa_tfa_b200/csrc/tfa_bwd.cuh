@@ -1,0 +1,629 @@
+// tfa_bwd.cuh -- backward pass of tiled GQA prefill attention on sm_100a:
+// dQ, dK and dV of the bare attention core, recompute-based (brotensor
+// "include/brotensor/ops/flash_attention.h", flash_attention_backward: no
+// forward caches are consumed; causal- and mask-excluded positions contribute
+// nothing to any gradient).  With s = q.k (raw), c = scale * log2(e),
+// lse the per-row base-2 log-sum-exp of s*c (from a forward recompute) and
+// delta_i = sum_d dO[i,d] O[i,d]:
+//   P[i,j]  = 2^(s[i,j] c - lse_i)                (0 where (i, j) is excluded)
+//   dP[i,j] = dO[i] . V[j]
+//   dS[i,j] = P[i,j] (dP[i,j] - delta_i)
+//   dQ[i]   = scale sum_j dS[i,j] K[j]
+//   dK[j]   = scale sum_i dS[i,j] Q[i]      (summed over the GQA group's heads)
+//   dV[j]   =       sum_i P[i,j] dO[i]      (likewise)
+// (delta_i = sum_j P[i,j] dP[i,j], the softmax Jacobian's row term.)
+//
+// Two kernels share the forward's machinery (TMA tiles with 128-byte swizzle,
+// tcgen05 MMAs with fp32 accumulators in tensor memory, one thread per
+// 128-lane row for the elementwise work), each with 192 threads: warps 0-3 do
+// the elementwise work and the epilogue, warp 4 is the TMA producer, warp 5
+// issues the MMAs.
+//   dQ kernel:  work item (b, h, 128-row query tile), walking the key tiles
+//               the tile sees: S = Q K^T and dP = dO V^T into tensor memory,
+//               dS (bf16) written over dP, then dQ += dS K.
+//   dKV kernel: work item (b, KV head, 128-key tile), walking the query tiles
+//               of every head of the group that see it: S^T = K Q^T and
+//               dP^T = V dO^T, P^T and dS^T (bf16) written over them, then
+//               dV += P^T dO and dK += dS^T Q.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "tfa_plan.h"
+#include "tfa_ptx.cuh"
+
+namespace tfa {
+namespace bwd {
+
+constexpr int kThreads = 192;
+
+template <int D>
+struct Cfg {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kTileBytes = 128 * D * 2;
+    static constexpr int kColBlocks = D / 64;
+    static constexpr int kColBlockBytes = 128 * 128;
+    static constexpr int kSlots = (D == 128) ? 4 : 8;  // ring of streamed tiles
+    static constexpr int kFixOff = 0;                  // two tiles fixed per item
+    static constexpr int kRingOff = 2 * kTileBytes;
+    static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
+    static constexpr int kNumBars = 2 * kSlots + 8;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kTmemA = 0;    // S (dQ kernel) / S^T (dKV kernel), 128 columns
+    static constexpr uint32_t kTmemB = 128;  // dP / dP^T, 128 columns
+    static constexpr uint32_t kTmemC = 256;  // dQ accumulator / dV accumulator, D columns
+    static constexpr uint32_t kTmemD = 256 + D;  // dK accumulator (dKV kernel), D columns
+};
+
+struct BwdParams {
+    __nv_bfloat16 *dq, *dk, *dv;  // outputs: [B,Hq,L,D], [B,Hkv,S,D] x2
+    const float *lse, *delta;     // [B,Hq,L]
+    const float *key_mask;        // [B,S] or nullptr
+    unsigned *status;
+    int B, Hq, Hkv, L, S, G, causal, window;
+    float scale, scale_log2;
+    int n_items;
+};
+
+// Barriers: fixed tiles full/empty, ring full/empty, the two score matrices
+// ready, the bf16 operands written, accumulators ready / read, teardown.
+struct Bars {
+    uint32_t base;
+    int slots;
+    __device__ __forceinline__ uint32_t fix_full() const { return base; }
+    __device__ __forceinline__ uint32_t fix_empty() const { return base + 8; }
+    __device__ __forceinline__ uint32_t ring_full(int s) const { return base + 8 * (2 + s); }
+    __device__ __forceinline__ uint32_t ring_empty(int s) const { return base + 8 * (2 + slots + s); }
+    __device__ __forceinline__ uint32_t mm_full() const { return base + 8 * (2 + 2 * slots); }
+    __device__ __forceinline__ uint32_t op_full() const { return base + 8 * (3 + 2 * slots); }
+    __device__ __forceinline__ uint32_t acc_full() const { return base + 8 * (4 + 2 * slots); }
+    __device__ __forceinline__ uint32_t acc_empty() const { return base + 8 * (5 + 2 * slots); }
+    __device__ __forceinline__ uint32_t done() const { return base + 8 * (6 + 2 * slots); }
+};
+
+// delta_i = sum_d dO[i,d] O[i,d] (fp32), one warp per row.
+template <int D>
+__global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16 *o, const __nv_bfloat16 *dout,
+                                                    float *delta, long long rows) {
+    const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    constexpr int kPer = D / 32;  // elements per lane: 4 (D = 128) or 2 (D = 64)
+    const __nv_bfloat16 *po = o + row * D + lane * kPer;
+    const __nv_bfloat16 *pd = dout + row * D + lane * kPer;
+    float acc = 0.f;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(po + e));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(pd + e));
+        acc = fmaf(a.x, b.x, fmaf(a.y, b.y, acc));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (lane == 0) delta[row] = acc;
+}
+
+// Item enumeration shared by the roles of one CTA (round-robin over the grid).
+// dQ kernel: item = (qt, b, h), query tiles in descending order when causal
+// (longest key ranges first).  dKV kernel: item = (kt, b, g).
+struct QItem {
+    int b, h, qt, lo, hi;  // key tiles [lo, hi]
+};
+__device__ __forceinline__ QItem q_item(const BwdParams &p, int item) {
+    const int nqt = (p.L + kBlockQ - 1) / kBlockQ;
+    const int bh = p.B * p.Hq;
+    const int r = item / bh, rem = item - r * bh;
+    QItem it;
+    it.qt = p.causal ? nqt - 1 - r : r;
+    it.b = rem / p.Hq;
+    it.h = rem - it.b * p.Hq;
+    const KeyRange kr = qtile_key_range(p.L, p.S, p.causal, p.window, it.qt * kBlockQ, 0u);
+    it.lo = kr.lo;
+    it.hi = kr.hi;
+    return it;
+}
+struct KItem {
+    int b, g, kt, qlo, qhi, nq, steps;  // per head of the group: query tiles [qlo, qhi]
+};
+__device__ __forceinline__ KItem k_item(const BwdParams &p, int item) {
+    const int bg = p.B * p.Hkv;
+    const int kt = item / bg, rem = item - kt * bg;
+    KItem it;
+    it.kt = kt;
+    it.b = rem / p.Hkv;
+    it.g = rem - it.b * p.Hkv;
+    const KeyRange qr = ktile_query_range(p.L, p.S, p.causal, p.window, kt);
+    it.qlo = qr.lo;
+    it.qhi = qr.hi;
+    it.nq = qr.hi >= qr.lo ? qr.hi - qr.lo + 1 : 0;
+    it.steps = it.nq * p.G;
+    return it;
+}
+
+// Common set-up of both kernels: barriers, tensor memory, the abort flag.
+template <int D>
+struct Setup {
+    uint32_t sbase, tmem;
+    uint8_t *gbase;
+    Bars bar;
+    volatile int *abort_flag;
+};
+
+template <int D>
+__device__ __forceinline__ Setup<D> setup(const CUtensorMap *m0, const CUtensorMap *m1,
+                                          const CUtensorMap *m2, const CUtensorMap *m3) {
+    using C = Cfg<D>;
+    extern __shared__ uint8_t smem_raw[];
+    Setup<D> st;
+    const uint32_t raw = smem_addr(smem_raw);
+    st.sbase = (raw + 1023u) & ~1023u;
+    st.gbase = smem_raw + (st.sbase - raw);
+    st.bar = Bars{st.sbase + C::kBarOff, C::kSlots};
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(st.gbase + C::kMiscOff);
+    st.abort_flag = reinterpret_cast<volatile int *>(st.gbase + C::kMiscOff + 4);
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+        mbar_init(st.bar.fix_full(), 1);
+        mbar_init(st.bar.fix_empty(), 1);
+        for (int s = 0; s < C::kSlots; ++s) {
+            mbar_init(st.bar.ring_full(s), 1);
+            mbar_init(st.bar.ring_empty(s), 1);
+        }
+        mbar_init(st.bar.mm_full(), 1);
+        mbar_init(st.bar.op_full(), 4);
+        mbar_init(st.bar.acc_full(), 1);
+        mbar_init(st.bar.acc_empty(), 4);
+        mbar_init(st.bar.done(), 1);
+        *st.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
+        tmem_relinquish();
+    }
+    if (warp == 4 && (threadIdx.x & 31) == 0) {
+        prefetch_tensormap(m0);
+        prefetch_tensormap(m1);
+        prefetch_tensormap(m2);
+        prefetch_tensormap(m3);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    st.tmem = *tmem_slot;
+    return st;
+}
+
+template <int D>
+__device__ __forceinline__ void teardown(const Setup<D> &st) {
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) {
+        tc_fence_after();
+        tmem_dealloc(st.tmem, Cfg<D>::kTmemCols);
+    }
+}
+
+// The producer's exit: every copy it started must land before the CTA leaves.
+template <int D>
+__device__ __forceinline__ void drain_copies(const Bars &bar, uint32_t prod, uint32_t fix_use) {
+    using C = Cfg<D>;
+    for (uint32_t s = 0; s < (uint32_t)C::kSlots; ++s) {
+        if (prod > s) {
+            const uint32_t armed = (prod - s - 1) / C::kSlots + 1;
+            mbar_drain(bar.ring_full(s), (armed - 1) & 1);
+        }
+    }
+    if (fix_use > 0) mbar_drain(bar.fix_full(), (fix_use - 1) & 1);
+}
+
+// Load two [128 rows][D] tiles (64-column boxes) onto one barrier.
+template <int D>
+__device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap *map, uint32_t bar, int row,
+                                          int plane) {
+    using C = Cfg<D>;
+    for (int cb = 0; cb < C::kColBlocks; ++cb)
+        tma_load_3d(dst + cb * C::kColBlockBytes, map, bar, cb * 64, row, plane);
+}
+
+// K-step offset (>> 4) inside a K-major 128-byte-swizzled [128][D] tile.
+template <int D>
+__device__ __forceinline__ uint32_t kstep_off(int kk) {
+    return static_cast<uint32_t>(((kk >> 2) * Cfg<D>::kColBlockBytes + (kk & 3) * 32) >> 4);
+}
+
+// ------------------------------------------------------------------ dQ kernel
+template <int D, bool KM>
+__global__ void __launch_bounds__(kThreads, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+              const BwdParams p) {
+    using C = Cfg<D>;
+    const Setup<D> st = setup<D>(&tm_q, &tm_do, &tm_k, &tm_v);
+    const Bars &bar = st.bar;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t kTileStep = C::kTileBytes >> 4;
+
+    if (warp == 4) {
+        // ---- producer: Q and dO once per item, then K_j, V_j per key tile
+        if (lane == 0) {
+            uint32_t prod = 0, fix_use = 0;
+            for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+                const QItem it = q_item(p, item);
+                if (fix_use > 0 && !mbar_wait(bar.fix_empty(), (fix_use - 1) & 1, st.abort_flag, p.status))
+                    break;
+                mbar_arrive_expect_tx(bar.fix_full(), 2 * C::kTileBytes);
+                load_tile<D>(st.sbase + C::kFixOff, &tm_q, bar.fix_full(), it.qt * kBlockQ, it.b * p.Hq + it.h);
+                load_tile<D>(st.sbase + C::kFixOff + C::kTileBytes, &tm_do, bar.fix_full(), it.qt * kBlockQ,
+                             it.b * p.Hq + it.h);
+                ++fix_use;
+                bool stop = false;
+                for (int j = it.lo; j <= it.hi && !stop; ++j) {
+                    for (int which = 0; which < 2; ++which) {
+                        const uint32_t s = prod % C::kSlots, round = prod / C::kSlots;
+                        if (round > 0 && !mbar_wait(bar.ring_empty(s), (round - 1) & 1, st.abort_flag, p.status)) {
+                            stop = true;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bar.ring_full(s), C::kTileBytes);
+                        load_tile<D>(st.sbase + C::kRingOff + s * C::kTileBytes, which ? &tm_v : &tm_k,
+                                     bar.ring_full(s), j * kBlockK, it.b * p.Hkv + it.h / p.G);
+                        ++prod;
+                    }
+                }
+                if (stop) break;
+            }
+            drain_copies<D>(bar, prod, fix_use);
+        }
+    } else if (warp == 5) {
+        // ---- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_bf16_f32(128, kBlockK, 0);  // both operands K-major
+            constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, 1);       // B = K tile, MN-major
+            const uint64_t d_q = smem_desc_sw128(st.sbase + C::kFixOff, 16, 1024);
+            const uint64_t d_do = d_q + kTileStep;
+            const uint64_t d_ring = smem_desc_sw128(st.sbase + C::kRingOff, 16, 1024);
+            const uint64_t d_ring_mn = smem_desc_sw128(st.sbase + C::kRingOff, C::kColBlockBytes, 1024);
+            uint32_t cons = 0, fix_use = 0, op_cnt = 0, acc_use = 0;
+            for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+                const QItem it = q_item(p, item);
+                if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
+                ++fix_use;
+                for (int j = it.lo; j <= it.hi; ++j) {
+                    const uint32_t sk = cons % C::kSlots;
+                    if (!mbar_wait(bar.ring_full(sk), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++cons;
+                    const uint32_t sv = cons % C::kSlots;
+                    if (!mbar_wait(bar.ring_full(sv), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++cons;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemA, d_q + kstep_off<D>(kk), d_ring + sk * kTileStep + kstep_off<D>(kk),
+                                kIdescS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemB, d_do + kstep_off<D>(kk), d_ring + sv * kTileStep + kstep_off<D>(kk),
+                                kIdescS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar.mm_full());
+                    umma_commit(bar.ring_empty(sv));
+                    if (j == it.hi) umma_commit(bar.fix_empty());
+                    // dQ += dS K, dS (bf16) in the first 64 columns of the dP region
+                    if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++op_cnt;
+                    // the previous item's dQ must have been read before it is overwritten
+                    if (j == it.lo && acc_use > 0 &&
+                        !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
+                        goto mma_out;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kBlockK / 16; ++kk)
+                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemB + kk * 8,
+                                d_ring_mn + sk * kTileStep + kk * ((16 * 128) >> 4), kIdescDQ,
+                                (j > it.lo || kk > 0) ? 1u : 0u);
+                    umma_commit(bar.ring_empty(sk));
+                }
+                umma_commit(bar.acc_full());
+                ++acc_use;
+            }
+        mma_out:
+            umma_commit(bar.done());
+            mbar_drain(bar.done(), 0);
+        }
+    } else {
+        // ---- elementwise (warps 0-3): P, dS per key tile; dQ epilogue per item
+        const int r = threadIdx.x;  // query row inside the tile = tensor-memory lane
+        const uint32_t lane_base = (static_cast<uint32_t>(warp) * 32u) << 16;
+        const uint32_t tA = st.tmem + C::kTmemA + lane_base;
+        const uint32_t tB = st.tmem + C::kTmemB + lane_base;
+        const uint32_t tC = st.tmem + C::kTmemC + lane_base;
+        const float c = p.scale_log2;
+        uint32_t mm_cnt = 0, acc_cnt = 0;
+        for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+            const QItem it = q_item(p, item);
+            const int q0 = it.qt * kBlockQ;
+            const int row = q0 + r;
+            const bool valid = row < p.L;
+            const size_t idx = static_cast<size_t>(it.b * p.Hq + it.h) * p.L + row;
+            const float lse_r = valid ? __ldg(p.lse + idx) : CUDART_INF_F;
+            const float dl_r = valid ? __ldg(p.delta + idx) : 0.f;
+            const int pos = (p.S - p.L) + row;
+            const int hi_abs = p.causal ? imin(pos, p.S - 1) : p.S - 1;
+            const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
+            const float *km_row = KM ? p.key_mask + static_cast<size_t>(it.b) * p.S : nullptr;
+            for (int j = it.lo; j <= it.hi; ++j) {
+                if (!__all_sync(0xffffffffu, mbar_wait(bar.mm_full(), mm_cnt & 1, st.abort_flag, p.status)))
+                    goto ew_out;
+                ++mm_cnt;
+                tc_fence_after();
+                const bool needs = key_tile_needs_mask(p.L, p.S, p.causal, p.window, KM ? 1 : 0, q0, j, 0u);
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t sv[32], dv[32], w[16];
+                    tmem_ld32(tA + 32 * ch, sv);
+                    tmem_ld32(tB + 32 * ch, dv);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -lse_r));
+                        float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -lse_r));
+                        if (needs) {
+                            const int k = j * kBlockK + 32 * ch + 2 * e;
+                            const bool a0 = k >= lo_abs && k <= hi_abs && (!KM || __ldg(km_row + k) > 0.5f);
+                            const bool a1 = k + 1 >= lo_abs && k + 1 <= hi_abs && (!KM || __ldg(km_row + k + 1) > 0.5f);
+                            p0 = a0 ? p0 : 0.f;
+                            p1 = a1 ? p1 : 0.f;
+                        }
+                        w[e] = pack_bf16(p0 * (__uint_as_float(dv[2 * e]) - dl_r),
+                                         p1 * (__uint_as_float(dv[2 * e + 1]) - dl_r));
+                    }
+                    tmem_st16(tB + 16 * ch, w);  // over dP columns already read
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.op_full());
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.acc_full(), acc_cnt & 1, st.abort_flag, p.status)))
+                goto ew_out;
+            ++acc_cnt;
+            tc_fence_after();
+            {
+                __nv_bfloat16 *orow = valid ? p.dq + idx * D : nullptr;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32(tC + 32 * cc, o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16(__uint_as_float(o[2 * i]) * p.scale, __uint_as_float(o[2 * i + 1]) * p.scale);
+                    if (orow) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.acc_empty());
+        }
+    ew_out:;
+    }
+    teardown<D>(st);
+}
+
+// ----------------------------------------------------------------- dKV kernel
+template <int D, bool KM>
+__global__ void __launch_bounds__(kThreads, 1)
+    dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+               const BwdParams p) {
+    using C = Cfg<D>;
+    const Setup<D> st = setup<D>(&tm_q, &tm_do, &tm_k, &tm_v);
+    const Bars &bar = st.bar;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t kTileStep = C::kTileBytes >> 4;
+
+    if (warp == 4) {
+        // ---- producer: K and V once per item, then Q_i, dO_i per (head, query tile)
+        if (lane == 0) {
+            uint32_t prod = 0, fix_use = 0;
+            bool stop = false;
+            for (int item = blockIdx.x; item < p.n_items && !stop; item += gridDim.x) {
+                const KItem it = k_item(p, item);
+                if (it.steps == 0) continue;
+                if (fix_use > 0 && !mbar_wait(bar.fix_empty(), (fix_use - 1) & 1, st.abort_flag, p.status))
+                    break;
+                mbar_arrive_expect_tx(bar.fix_full(), 2 * C::kTileBytes);
+                load_tile<D>(st.sbase + C::kFixOff, &tm_k, bar.fix_full(), it.kt * kBlockK, it.b * p.Hkv + it.g);
+                load_tile<D>(st.sbase + C::kFixOff + C::kTileBytes, &tm_v, bar.fix_full(), it.kt * kBlockK,
+                             it.b * p.Hkv + it.g);
+                ++fix_use;
+                for (int step = 0; step < it.steps && !stop; ++step) {
+                    const int h = it.g * p.G + step / it.nq;
+                    const int qt = it.qlo + step % it.nq;
+                    for (int which = 0; which < 2; ++which) {  // Q_i then dO_i
+                        const uint32_t s = prod % C::kSlots, round = prod / C::kSlots;
+                        if (round > 0 && !mbar_wait(bar.ring_empty(s), (round - 1) & 1, st.abort_flag, p.status)) {
+                            stop = true;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(bar.ring_full(s), C::kTileBytes);
+                        load_tile<D>(st.sbase + C::kRingOff + s * C::kTileBytes, which ? &tm_do : &tm_q,
+                                     bar.ring_full(s), qt * kBlockQ, it.b * p.Hq + h);
+                        ++prod;
+                    }
+                }
+            }
+            drain_copies<D>(bar, prod, fix_use);
+        }
+    } else if (warp == 5) {
+        // ---- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_bf16_f32(128, kBlockQ, 0);  // both operands K-major
+            constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, 1);      // B = dO / Q tile, MN-major
+            const uint64_t d_k = smem_desc_sw128(st.sbase + C::kFixOff, 16, 1024);
+            const uint64_t d_v = d_k + kTileStep;
+            const uint64_t d_ring = smem_desc_sw128(st.sbase + C::kRingOff, 16, 1024);
+            const uint64_t d_ring_mn = smem_desc_sw128(st.sbase + C::kRingOff, C::kColBlockBytes, 1024);
+            uint32_t cons = 0, fix_use = 0, op_cnt = 0, acc_use = 0;
+            for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+                const KItem it = k_item(p, item);
+                if (it.steps == 0) continue;
+                if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
+                ++fix_use;
+                for (int step = 0; step < it.steps; ++step) {
+                    const uint32_t sq = cons % C::kSlots;
+                    if (!mbar_wait(bar.ring_full(sq), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++cons;
+                    const uint32_t sd = cons % C::kSlots;
+                    if (!mbar_wait(bar.ring_full(sd), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++cons;
+                    tc_fence_after();
+                    // S^T = K Q^T, dP^T = V dO^T
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk), d_ring + sq * kTileStep + kstep_off<D>(kk),
+                                kIdescS, kk > 0 ? 1u : 0u);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk), d_ring + sd * kTileStep + kstep_off<D>(kk),
+                                kIdescS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar.mm_full());
+                    if (step == it.steps - 1) umma_commit(bar.fix_empty());
+                    if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++op_cnt;
+                    if (step == 0 && acc_use > 0 &&
+                        !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
+                        goto mma_out;
+                    tc_fence_after();
+                    // dV += P^T dO (P^T in the first 64 columns of the S^T region),
+                    // dK += dS^T Q (dS^T in the first 64 columns of the dP^T region)
+#pragma unroll
+                    for (int kk = 0; kk < kBlockQ / 16; ++kk) {
+                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemA + kk * 8,
+                                d_ring_mn + sd * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
+                                (step > 0 || kk > 0) ? 1u : 0u);
+                        umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + kk * 8,
+                                d_ring_mn + sq * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
+                                (step > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    umma_commit(bar.ring_empty(sq));
+                    umma_commit(bar.ring_empty(sd));
+                }
+                umma_commit(bar.acc_full());
+                ++acc_use;
+            }
+        mma_out:
+            umma_commit(bar.done());
+            mbar_drain(bar.done(), 0);
+        }
+    } else {
+        // ---- elementwise (warps 0-3): P^T, dS^T per step; dK, dV epilogue per item
+        const int r = threadIdx.x;  // key row inside the tile = tensor-memory lane
+        const uint32_t lane_base = (static_cast<uint32_t>(warp) * 32u) << 16;
+        const uint32_t tA = st.tmem + C::kTmemA + lane_base;
+        const uint32_t tB = st.tmem + C::kTmemB + lane_base;
+        const uint32_t tC = st.tmem + C::kTmemC + lane_base;
+        const uint32_t tD = st.tmem + C::kTmemD + lane_base;
+        const float c = p.scale_log2;
+        const int P = p.S - p.L;
+        uint32_t mm_cnt = 0, acc_cnt = 0;
+        for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+            const KItem it = k_item(p, item);
+            const int key = it.kt * kBlockK + r;
+            const bool kvalid = key < p.S;
+            const bool kept = kvalid && (!KM || __ldg(p.key_mask + static_cast<size_t>(it.b) * p.S + key) > 0.5f);
+            const size_t oidx = (static_cast<size_t>(it.b * p.Hkv + it.g) * p.S + key) * D;
+            if (it.steps == 0) {  // no row sees this key tile: zero gradients
+                if (kvalid) {
+                    uint4 *dk4 = reinterpret_cast<uint4 *>(p.dk + oidx);
+                    uint4 *dv4 = reinterpret_cast<uint4 *>(p.dv + oidx);
+                    for (int v4 = 0; v4 < D / 8; ++v4) {
+                        dk4[v4] = make_uint4(0u, 0u, 0u, 0u);
+                        dv4[v4] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+                continue;
+            }
+            for (int step = 0; step < it.steps; ++step) {
+                const int h = it.g * p.G + step / it.nq;
+                const int q0 = (it.qlo + step % it.nq) * kBlockQ;
+                const float *lse_h = p.lse + static_cast<size_t>(it.b * p.Hq + h) * p.L;
+                const float *dl_h = p.delta + static_cast<size_t>(it.b * p.Hq + h) * p.L;
+                if (!__all_sync(0xffffffffu, mbar_wait(bar.mm_full(), mm_cnt & 1, st.abort_flag, p.status)))
+                    goto ew_out;
+                ++mm_cnt;
+                tc_fence_after();
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t sv[32], dv[32], wp[16], wd[16];
+                    tmem_ld32(tA + 32 * ch, sv);
+                    tmem_ld32(tB + 32 * ch, dv);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const int q = q0 + 32 * ch + e;
+                        const bool qv = q < p.L;
+                        const float lse_q = qv ? __ldg(lse_h + q) : CUDART_INF_F;
+                        const float dl_q = qv ? __ldg(dl_h + q) : 0.f;
+                        const bool allowed = kept && qv &&
+                                             (!p.causal || (key <= P + q && (p.window <= 0 || key > P + q - p.window)));
+                        const float pv = allowed ? ex2(fmaf(__uint_as_float(sv[e]), c, -lse_q)) : 0.f;
+                        const float ds = pv * (__uint_as_float(dv[e]) - dl_q);
+                        // pack in pairs as they complete
+                        if (e & 1) {
+                            wp[e >> 1] = pack_bf16(__uint_as_float(sv[e - 1]), pv);
+                            wd[e >> 1] = pack_bf16(__uint_as_float(dv[e - 1]), ds);
+                        } else {
+                            sv[e] = __float_as_uint(pv);  // keep the even element until its pair is done
+                            dv[e] = __float_as_uint(ds);
+                        }
+                    }
+                    tmem_st16(tA + 16 * ch, wp);  // over S^T columns already read
+                    tmem_st16(tB + 16 * ch, wd);  // over dP^T columns already read
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.op_full());
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.acc_full(), acc_cnt & 1, st.abort_flag, p.status)))
+                goto ew_out;
+            ++acc_cnt;
+            tc_fence_after();
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
+                __nv_bfloat16 *orow = kvalid ? (which ? p.dk : p.dv) + oidx : nullptr;
+                const float f = which ? p.scale : 1.f;
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t o[32];
+                    tmem_ld32((which ? tD : tC) + 32 * cc, o);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16(__uint_as_float(o[2 * i]) * f, __uint_as_float(o[2 * i + 1]) * f);
+                    if (orow) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+#pragma unroll
+                        for (int v4 = 0; v4 < 4; ++v4)
+                            dst[v4] = make_uint4(w[4 * v4], w[4 * v4 + 1], w[4 * v4 + 2], w[4 * v4 + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.acc_empty());
+        }
+    ew_out:;
+    }
+    teardown<D>(st);
+}
+
+}  // namespace bwd
+}  // namespace tfa

@@ -149,6 +149,10 @@ struct Params {
     // the longest query (max_seqlen_q)
     int varlen, total_q, total_k;
     const int *cu_q, *cu_k;
+    // optional per-row log-sum-exp in base 2 of the scaled scores,
+    // log2(sum_j 2^(s_j * scale_log2)) (+inf for a row with no allowed key),
+    // [B, Hq, L] fp32: what a backward pass needs to rebuild P from S
+    float *lse;
     // split schedule: ctl[0] counts finished launches (the epoch of a launch is
     // ctl[0] + 1, read from device memory so a captured graph replays correctly),
     // ctl[1] counts the CTAs of the running launch that have finished
@@ -771,6 +775,9 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         // l == 0 and is written as zeros).
         if (!warp_live) continue;
         if (row_live) l = add_sink(p, l, m_star, c, out_head);  // m_star == m_ref for a whole tile
+        if (p.lse && row_valid)
+            p.lse[static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row] =
+                l > 0.f ? fmaf(m_star, c, __log2f(l)) : CUDART_INF_F;
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16 *orow = nullptr;
         if (row_valid)  // dense [B,Hq,L,D]; varlen packed [total_q, Hq, D]

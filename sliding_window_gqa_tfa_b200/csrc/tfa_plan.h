@@ -61,4 +61,37 @@ TFA_HD bool key_tile_needs_mask(int L, int S, int causal, int window, int has_ke
     return false;
 }
 
+// The query tiles that hold a row seeing some key of 128-key tile kt (the
+// transpose of qtile_key_range, for the backward pass that walks key tiles):
+// a row i sees key j iff (causal => j <= P + i) and (window => j > P + i - W).
+// Returns lo > hi when no row sees the tile.
+TFA_HD KeyRange ktile_query_range(int L, int S, int causal, int window, int kt) {
+    const int P = S - L;
+    const int k0 = kt * kBlockK;
+    const int k1 = imin(k0 + kBlockK - 1, S - 1);
+    const int nqt = (L + kBlockQ - 1) / kBlockQ;
+    KeyRange r;
+    r.lo = 0;
+    r.hi = nqt - 1;
+    if (causal) {
+        const int first_row = k0 - P;  // the first row that sees key k0
+        if (first_row > L - 1) {
+            r.lo = 1;
+            r.hi = 0;
+            return r;
+        }
+        r.lo = first_row > 0 ? first_row / kBlockQ : 0;
+        if (window > 0) {
+            const int last_row = k1 - P + window - 1;  // the last row that sees key k1
+            if (last_row < 0) {
+                r.lo = 1;
+                r.hi = 0;
+                return r;
+            }
+            r.hi = imin(last_row, L - 1) / kBlockQ;
+        }
+    }
+    return r;
+}
+
 }  // namespace tfa

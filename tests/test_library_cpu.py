@@ -222,3 +222,29 @@ def test_decode_validates_like_prefill():
                          None) == tb.TFA_ERR_SHAPE
     assert tb.tfa_decode(A16, A16, A16, A16, 1, 8, 2, 1, 100, 128, 0.1, 0, 16, None,
                          None) == tb.TFA_ERR_WINDOW
+
+
+@pytest.mark.parametrize("case", _plan_cases(), ids=lambda c: c[0])
+def test_key_tile_enumeration_is_exact(case):
+    """The backward pass's view: every allowed (row, key) pair has its row's
+    query tile inside the range of its key's tile, and the first and last
+    query tiles of each range hold an allowed pair."""
+    _, L, S, causal, window, _ = case
+    P = S - L
+    nkt = (S + 127) // 128
+    rows = np.arange(L)[:, None]
+    keys = np.arange(S)[None, :]
+    allowed = np.ones((L, S), dtype=bool)
+    if causal:
+        allowed &= keys <= P + rows
+        if window > 0:
+            allowed &= keys > P + rows - window
+    for kt in range(nkt):
+        rc, lo, hi = tb.tfa_plan_ktile(L, S, causal, window, kt)
+        assert rc == 0
+        blk = allowed[:, kt * 128:(kt + 1) * 128].any(axis=1)
+        qts = sorted(set(np.nonzero(blk)[0] // 128))
+        if not qts:
+            assert hi < lo
+        else:
+            assert (lo, hi) == (qts[0], qts[-1]), (kt, lo, hi, qts[0], qts[-1])
