@@ -36,8 +36,8 @@ sys.path.insert(0, ROOT)
 
 from sliding_window_gqa_tfa_b200 import binding as tb  # noqa: E402
 from sliding_window_gqa_tfa_b200.flops import workload_bytes, workload_flops  # noqa: E402
-from sliding_window_gqa_tfa_b200.inputs import (HEADLINE, WORKLOADS, make_inputs,  # noqa: E402
-                                                make_sinks, varlen_cu)
+from sliding_window_gqa_tfa_b200.inputs import (HEADLINE, WORKLOADS, make_dout,  # noqa: E402
+                                                make_inputs, make_sinks, varlen_cu)
 
 METRIC = "prefill attention TFLOP/s (unmasked pairs) and % of B200 BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -206,11 +206,33 @@ class OracleSampler:
             self.cq, self.ck = varlen_cu(w)
             self.live = [b for b, (L, _) in enumerate(w.seqlens) if L > 0]
         self.n_rows = w.B * w.Hq * w.L
+        if w.kind == "backward":
+            self.dout = make_dout(w, seed=seed)
 
     def unit(self, rng, n):
         """Run the oracle on n random rows; return their useful flops."""
         w, o = self.w, self.oracle
         kw = dict(scale=w.softmax_scale, window=w.window, softcap=w.softcap, sinks=self.sinks)
+        if w.kind == "backward":
+            # the gradients of n query rows of one KV group (all heads of the
+            # group), over the keys those rows reach: a sub-problem of the same
+            # shape family (prefix S - L kept), rows starting at a random tile
+            G = w.Hq // w.Hkv
+            P = w.S - w.L
+            r0 = int(rng.integers(0, max(1, w.L - n + 1)))
+            rows = slice(r0, r0 + n)
+            g = int(rng.integers(0, w.Hkv))
+            heads = slice(g * G, (g + 1) * G)
+            S_sub = P + r0 + n
+            q = self.q[:1, heads, rows].contiguous()
+            do = self.dout[:1, heads, rows].contiguous()
+            k = self.k[:1, g:g + 1, :S_sub].contiguous()
+            v = self.v[:1, g:g + 1, :S_sub].contiguous()
+            # rows r0..r0+n-1 of the full problem are rows 0..n-1 here with prefix P + r0
+            o.attention_backward(q, k, v, do, scale=w.softmax_scale, causal=w.causal, window=w.window)
+            return 10 * w.D * G * int(sum(min(P + r0 + i, S_sub - 1) + 1 -
+                                          (max(0, P + r0 + i - w.window + 1) if w.window > 0 else 0)
+                                          for i in range(n)) if w.causal else n * S_sub * G * 10 * w.D)
         if w.kind == "varlen":
             # one sequence through the dense oracle (the varlen definition per sequence)
             b = int(rng.choice(self.live))
@@ -252,7 +274,7 @@ def run_reference(args, w):
         return 0
     sampler = OracleSampler(w, seed=0)
     rng = np.random.default_rng(1)
-    per_step = 32
+    per_step = 8 if w.kind == "backward" else 32  # the backward oracle runs one KV group per thread
     times, flops = [], []
     for step in range(args.warmup + args.steps):
         t0 = time.perf_counter()
@@ -301,10 +323,18 @@ def main():
 
     q, k, v, km = make_inputs(w, seed=rank)
     sinks = make_sinks(w, seed=rank)
-    cu = tuple(torch.from_numpy(c) for c in varlen_cu(w)) if w.kind == "varlen" else ()
-    host_inputs = [q, k, v, km, sinks, *cu]  # what one call reads (None: absent)
+    if w.kind == "varlen":
+        extra = tuple(torch.from_numpy(c) for c in varlen_cu(w))
+    elif w.kind == "backward":
+        extra = (make_dout(w, seed=rank),)
+    else:
+        extra = ()
+    host_inputs = [q, k, v, km, sinks, *extra]  # what one call reads (None: absent)
     dev_inputs = [t.to(dev) if t is not None else None for t in host_inputs]
-    out = torch.empty_like(dev_inputs[0])
+    if w.kind == "backward":  # (dq, dk, dv)
+        out = tuple(torch.empty_like(t) for t in dev_inputs[:3])
+    else:
+        out = torch.empty_like(dev_inputs[0])
     flops = workload_flops(w, key_mask=km)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -312,7 +342,10 @@ def main():
     def call(ins, o):
         """One launch on the current stream: the entry point the workload needs."""
         dq, dk, dv, dkm, dsinks = ins[:5]
-        if w.kind == "varlen":
+        if w.kind == "backward":
+            tb.backward(dq, dk, dv, ins[5], scale=w.softmax_scale, causal=w.causal, window=w.window,
+                        key_mask=dkm, out=o)
+        elif w.kind == "varlen":
             tb.prefill_varlen(dq, dk, dv, ins[5], ins[6], max_seqlen_q=w.L, scale=w.softmax_scale,
                               causal=w.causal, window=w.window, softcap=w.softcap, sinks=dsinks,
                               out=o)
@@ -355,21 +388,25 @@ def main():
     # end to end through the C ABI with host buffers (copies inside the timed region)
     pinned = [t.pin_memory() if t is not None else None for t in host_inputs]
     hq, hk, hv, hkm = pinned[:4]
-    hout = torch.empty_like(hq).pin_memory()
+    if w.kind == "backward":
+        hout = tuple(torch.empty_like(t).pin_memory() for t in (hq, hk, hv))
+    else:
+        hout = torch.empty_like(hq).pin_memory()
     if w.kind != "dense" or w.softcap > 0 or sinks is not None:
         # the device entry points: the step copies the pinned inputs in, calls
         # the entry point, and copies the output back, all on `stream`
         staged = [torch.empty_like(t) if t is not None else None for t in dev_inputs]
-        eout = torch.empty_like(out)
+        eout = tuple(torch.empty_like(t) for t in out) if w.kind == "backward" else torch.empty_like(out)
 
         def e2e_step():
             for d, h in zip(staged, pinned):
                 if d is not None:
                     d.copy_(h, non_blocking=True)
             call(staged, eout)
-            hout.copy_(eout, non_blocking=True)
-        entry = {"varlen": "tfa_prefill_varlen", "ring": "tfa_prefill_ring"}.get(w.kind,
-                                                                                  "tfa_attention_ex")
+            for h, d in (zip(hout, eout) if w.kind == "backward" else [(hout, eout)]):
+                h.copy_(d, non_blocking=True)
+        entry = {"varlen": "tfa_prefill_varlen", "ring": "tfa_prefill_ring",
+                 "backward": "tfa_prefill_backward"}.get(w.kind, "tfa_attention_ex")
         e2e_api = f"{entry} (pinned host buffers, copies on the stream)"
     else:
         def e2e_step():
@@ -389,7 +426,7 @@ def main():
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
     h2d = sum(t.numel() * t.element_size() for t in pinned if t is not None)
-    d2h = hout.numel() * 2
+    d2h = sum(t.numel() * 2 for t in hout) if w.kind == "backward" else hout.numel() * 2
 
     peaks, peak_kind = load_peaks()
     alg_bytes = workload_bytes(w)
@@ -426,7 +463,9 @@ def main():
             "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "api": e2e_api},
-            "gpu_launches": args.steps,
+            # kernels per step: one, or four for the backward (forward recompute,
+            # delta, dQ, dK/dV)
+            "gpu_launches": args.steps * (4 if w.kind == "backward" else 1),
             "clocks": clocks,
             "wall_s_timed_region": t_wall,
         }

@@ -293,7 +293,8 @@ def tfa_prefill_backward(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, D, scale, 
                                       window, key_mask, stream)
 
 
-def backward(q, k, v, dout, *, scale=None, causal=True, window=0, key_mask=None, stream=None):
+def backward(q, k, v, dout, *, scale=None, causal=True, window=0, key_mask=None, out=None,
+             stream=None):
     """(dq, dk, dv) bf16 of the attention core for the upstream gradient dout
     [B,Hq,L,D] (recompute-based: the forward is re-run inside)."""
     import torch
@@ -307,7 +308,13 @@ def backward(q, k, v, dout, *, scale=None, causal=True, window=0, key_mask=None,
     if key_mask is not None:
         _check(key_mask, "key_mask", torch.float32, 2)
     scale = 1.0 / math.sqrt(D) if scale is None else scale
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    if out is None:
+        out = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = out
+    for t, ref, n in ((dq, q, "dq"), (dk, k, "dk"), (dv, v, "dv")):
+        _check(t, n, torch.bfloat16, 4)
+        if tuple(t.shape) != tuple(ref.shape):
+            raise ValueError(f"{n} has the wrong shape")
     rc = tfa_prefill_backward(*(ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, dout, dq, dk, dv)),
                               B, Hq, Hkv, L, S, D, float(scale), int(bool(causal)), int(window),
                               _ptr_or_none(key_mask), _stream_handle(stream))

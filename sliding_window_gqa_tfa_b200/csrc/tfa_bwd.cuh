@@ -50,7 +50,9 @@ struct Cfg {
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
     static constexpr int kNumBars = 2 * kSlots + 8;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-    static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
+    // dKV kernel: per elementwise warp, the step's 128 values of -lse and delta
+    static constexpr int kStageOff = kMiscOff + 16;
+    static constexpr int kSmemBytes = kStageOff + 4 * 256 * 4 + 1024;  // + slack to align the base
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kTmemA = 0;    // S (dQ kernel) / S^T (dKV kernel), 128 columns
     static constexpr uint32_t kTmemB = 128;  // dP / dP^T, 128 columns
@@ -533,12 +535,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tD = st.tmem + C::kTmemD + lane_base;
         const float c = p.scale_log2;
         const int P = p.S - p.L;
+        float *stage = reinterpret_cast<float *>(st.gbase + C::kStageOff) + warp * 256;
         uint32_t mm_cnt = 0, acc_cnt = 0;
         for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
             const KItem it = k_item(p, item);
             const int key = it.kt * kBlockK + r;
             const bool kvalid = key < p.S;
             const bool kept = kvalid && (!KM || __ldg(p.key_mask + static_cast<size_t>(it.b) * p.S + key) > 0.5f);
+            // the query rows that see this key: [q_lo, q_hi] (empty when not kept)
+            int q_lo = p.causal ? imax(0, key - P) : 0;
+            int q_hi = (p.causal && p.window > 0) ? imin(p.L - 1, key - P + p.window - 1) : p.L - 1;
+            if (!kept) q_hi = q_lo - 1;
             const size_t oidx = (static_cast<size_t>(it.b * p.Hkv + it.g) * p.S + key) * D;
             if (it.steps == 0) {  // no row sees this key tile: zero gradients
                 if (kvalid) {
@@ -556,6 +563,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int q0 = (it.qlo + step % it.nq) * kBlockQ;
                 const float *lse_h = p.lse + static_cast<size_t>(it.b * p.Hq + h) * p.L;
                 const float *dl_h = p.delta + static_cast<size_t>(it.b * p.Hq + h) * p.L;
+                // -lse and delta of the tile's 128 query columns, loaded once per
+                // warp (lane e: columns e, 32 + e, ...) into the warp's stage and
+                // read back as shared-memory broadcasts
+                __syncwarp();  // every lane is done with the previous step's stage
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    const int q = q0 + 32 * ch + lane;
+                    stage[32 * ch + lane] = q < p.L ? -__ldg(lse_h + q) : -CUDART_INF_F;
+                    stage[128 + 32 * ch + lane] = q < p.L ? __ldg(dl_h + q) : 0.f;
+                }
+                __syncwarp();
                 if (!__all_sync(0xffffffffu, mbar_wait(bar.mm_full(), mm_cnt & 1, st.abort_flag, p.status)))
                     goto ew_out;
                 ++mm_cnt;
@@ -565,15 +583,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t sv[32], dv[32], wp[16], wd[16];
                     tmem_ld32(tA + 32 * ch, sv);
                     tmem_ld32(tB + 32 * ch, dv);
+                    const int qc = q0 + 32 * ch;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const int q = q0 + 32 * ch + e;
-                        const bool qv = q < p.L;
-                        const float lse_q = qv ? __ldg(lse_h + q) : CUDART_INF_F;
-                        const float dl_q = qv ? __ldg(dl_h + q) : 0.f;
-                        const bool allowed = kept && qv &&
-                                             (!p.causal || (key <= P + q && (p.window <= 0 || key > P + q - p.window)));
-                        const float pv = allowed ? ex2(fmaf(__uint_as_float(sv[e]), c, -lse_q)) : 0.f;
+                        const float nlse_q = stage[32 * ch + e];
+                        const float dl_q = stage[128 + 32 * ch + e];
+                        const bool allowed = (qc + e >= q_lo) & (qc + e <= q_hi);
+                        const float ev = ex2(fmaf(__uint_as_float(sv[e]), c, nlse_q));
+                        const float pv = allowed ? ev : 0.f;
                         const float ds = pv * (__uint_as_float(dv[e]) - dl_q);
                         // pack in pairs as they complete
                         if (e & 1) {

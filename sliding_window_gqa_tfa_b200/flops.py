@@ -45,8 +45,10 @@ def workload_flops(w, key_mask=None) -> int:
     if w.seqlens is not None:
         return sum(useful_flops(1, w.Hq, L, S, w.D, causal=w.causal, window=w.window)
                    for L, S in w.seqlens)
-    return useful_flops(w.B, w.Hq, w.L, w.S, w.D, causal=w.causal, window=w.window,
-                        key_mask=key_mask)
+    f = useful_flops(w.B, w.Hq, w.L, w.S, w.D, causal=w.causal, window=w.window, key_mask=key_mask)
+    # backward: five products of 2*D per allowed pair (S = Q K^T, dP = dO V^T,
+    # dV = P^T dO, dQ = dS K, dK = dS^T Q) against the forward's two
+    return f * 5 // 2 if w.backward else f
 
 
 def workload_bytes(w) -> int:
@@ -57,4 +59,7 @@ def workload_bytes(w) -> int:
         Tk = sum(S for _, S in w.seqlens)
         return 2 * w.D * (2 * Tq * w.Hq + 2 * Tk * w.Hkv)
     S = min(w.S, w.ring_rows) if w.ring_rows else w.S
-    return algorithmic_bytes(w.B, w.Hq, w.Hkv, w.L, S, w.D, key_mask=w.key_mask_keep is not None)
+    fwd = algorithmic_bytes(w.B, w.Hq, w.Hkv, w.L, S, w.D, key_mask=w.key_mask_keep is not None)
+    if w.backward:  # + dO read and dQ written, dK and dV written
+        return fwd + 2 * w.D * (2 * w.B * w.Hq * w.L + 2 * w.B * w.Hkv * S)
+    return fwd

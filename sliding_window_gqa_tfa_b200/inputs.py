@@ -8,8 +8,9 @@ Recipe: a CPU ``torch.Generator`` seeded with ``seed``; fp32 ``randn`` drawn in
 the order Q, K, V (K multiplied by ``k_scale`` before the cast), then, when the
 workload has a key mask, ``rand(B, S) >= 1 - keep`` as the 1/0 fp32 key mask,
 then, when it has attention sinks, ``sink_scale * randn(Hq)`` fp32 sink logits;
-Q/K/V are cast to bf16 (round to nearest even).  A logit softcap is a plain
-number of the workload (Gemma-2 uses 50).  The shapes are the model
+then, for a backward workload, ``randn`` of q's shape as the upstream gradient
+dO (bf16); Q/K/V are cast to bf16 (round to nearest even).  A logit softcap
+is a plain number of the workload (Gemma-2 uses 50).  The shapes are the model
 shapes the pages use: Qwen3-0.6B (16 query heads, 8 KV heads, head dim 128,
 tiny-llm "Week 2 Day 5"), the Llama geometry of TensorFold PR 3269 (56 query
 heads, 8 KV heads, group 7, head dim 128), the 1024-key sliding window of the
@@ -46,9 +47,13 @@ class Workload:
     # packed variable-length batch: ((L_b, S_b), ...) per sequence; B = len(seqlens),
     # L / S = the longest query / key count
     seqlens: tuple | None = None
+    # the backward pass (gradients of q, k, v for an upstream gradient of the output)
+    backward: bool = False
 
     @property
     def kind(self) -> str:
+        if self.backward:
+            return "backward"
         return "varlen" if self.seqlens is not None else "ring" if self.ring_rows else "dense"
 
     @property
@@ -98,6 +103,9 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     # Packed variable-length prefill of 16 Qwen3-shaped prompts (256..4096 tokens).
     Workload("varlen_qwen3_16seqs", B=16, Hq=16, Hkv=8, L=_VARLEN16_MAX, S=_VARLEN16_MAX, D=128,
              seqlens=tuple((n, n) for n in _VARLEN16)),
+    # The backward pass on the Llama chunk (gradients of q, k, v).
+    Workload("llama_gqa_chunk_2048x8192_backward", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
+             backward=True),
     # Short queries (1 <= L <= 8): token-by-token decoding over a long cache,
     # batched Qwen3-shaped decoding, and an 8-row chunk (e.g. draft verification).
     Workload("llama_gqa_decode_1x32768", B=1, Hq=56, Hkv=8, L=1, S=32768, D=128),
@@ -154,7 +162,16 @@ def _draw(w: Workload, seed: int):
     sinks = None
     if w.sink_scale is not None:
         sinks = w.sink_scale * torch.randn(w.Hq, generator=g, dtype=torch.float32)
-    return q.bfloat16(), k.bfloat16(), v.bfloat16(), key_mask, sinks
+    dout = None
+    if w.backward:
+        dout = torch.randn(*q_shape, generator=g, dtype=torch.float32).bfloat16()
+    return q.bfloat16(), k.bfloat16(), v.bfloat16(), key_mask, sinks, dout
+
+
+def make_dout(w: Workload, seed: int = 0):
+    """bf16 upstream gradient of the output (shape of q) of a backward workload,
+    drawn after q, k, v, the key mask and the sinks from the same generator."""
+    return _draw(w, seed)[5]
 
 
 def shaped(B, Hq, Hkv, L, S, D, *, causal=True, window=0, key_mask_keep=None, k_scale=1.0,
