@@ -85,6 +85,13 @@ def _load():
             lib.oracle_attention_backward_mutant.argtypes = [P] * 7 + [i32] * 6 + [f64, i32, i32, P,
                                                                                  i32]
             lib.oracle_attention_backward_mutant.restype = i32
+            lib.oracle_attention_backward_dq_rows.argtypes = [P] * 5 + [i32] * 6 + [f64, i32, i32, P,
+                                                                                  P, i64, i32]
+            lib.oracle_attention_backward_dq_rows.restype = i32
+            lib.oracle_attention_backward_kv_rows.argtypes = [P] * 6 + [i32] * 6 + [f64, i32, i32, P,
+                                                                                  i32, i32, P, i64,
+                                                                                  i32]
+            lib.oracle_attention_backward_kv_rows.restype = i32
             lib.oracle_attention_mutant.restype = i32
             lib.oracle_softmax_weights.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                    i32, i32, P, i32, i32, i32]
@@ -268,6 +275,43 @@ def attention_backward(q, k, v, dout, *, scale, causal, window=0, key_mask=None,
     if rc:
         raise ValueError(f"oracle_attention_backward rejected its arguments (code {rc})")
     return dq, dk, dv
+
+
+def attention_backward_dq_rows(q, k, v, dout, rows, *, scale, causal, window=0, key_mask=None,
+                               threads=0):
+    """dQ (float64, len(rows) x D) of the listed flattened rows (b*Hq+h)*L+i only."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    km = _mask(key_mask)
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    out = np.empty((r.size, D), dtype=np.float64)
+    rc = _load().oracle_attention_backward_dq_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(db), _ptr(out),
+                                                   B, Hq, Hkv, L, S, D, float(scale),
+                                                   int(bool(causal)), int(window), _ptr(km),
+                                                   r.ctypes.data_as(ctypes.c_void_p), r.size,
+                                                   int(threads))
+    if rc:
+        raise ValueError(f"oracle_attention_backward_dq_rows rejected its arguments (code {rc})")
+    return out
+
+
+def attention_backward_kv_rows(q, k, v, dout, *, b, g, keys, scale, causal, window=0,
+                               key_mask=None, threads=0):
+    """(dk, dv) float64 (len(keys) x D each) of the listed keys of KV head g, batch b."""
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    B, Hq, Hkv, L, S, D = _shape(qb, kb)
+    km = _mask(key_mask)
+    kk = np.ascontiguousarray(np.asarray(keys, dtype=np.int64))
+    dk = np.empty((kk.size, D), dtype=np.float64)
+    dv = np.empty((kk.size, D), dtype=np.float64)
+    rc = _load().oracle_attention_backward_kv_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(db), _ptr(dk),
+                                                   _ptr(dv), B, Hq, Hkv, L, S, D, float(scale),
+                                                   int(bool(causal)), int(window), _ptr(km), int(b),
+                                                   int(g), kk.ctypes.data_as(ctypes.c_void_p),
+                                                   kk.size, int(threads))
+    if rc:
+        raise ValueError(f"oracle_attention_backward_kv_rows rejected its arguments (code {rc})")
+    return dk, dv
 
 
 def attention_blockwise(q, k, v, *, scale, causal, window=0, key_mask=None, bq=128, bk=128,

@@ -564,6 +564,182 @@ static int backward_impl(const uint16_t *q, const uint16_t *k, const uint16_t *v
     return failed ? 5 : 0;
 }
 
+/* dQ of the listed rows only (row = (b*Hq + h)*L + i; dq holds nrows x D):
+ * the same per-row arithmetic as backward_impl, which a row's dQ needs alone
+ * (its softmax weights, dP and row term), so it scales to any size. */
+int oracle_attention_backward_dq_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                      const uint16_t *dout, double *dq, int B, int Hq, int Hkv,
+                                      int L, int S, int D, double scale, int causal, int window,
+                                      const float *key_mask, const int64_t *rows, int64_t nrows,
+                                      int nthreads)
+{
+    int rc = check_args(q, k, v, dq, B, Hq, Hkv, L, S, D);
+    if (rc) return rc;
+    if (!dout || !rows) return 1;
+    for (int64_t r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= (int64_t)B * Hq * L) return 4;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)S);
+        double *dP = (double *)malloc(sizeof(double) * (size_t)S);
+        if (!P || !dP) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < nrows; ++r) {
+            if (!P || !dP) continue;
+            const long row = (long)rows[r];
+            const long i = row % L;
+            const long bh = row / L;
+            const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+            const int g = kv_head_impl(h, Hq, Hkv, MUT_NONE);
+            const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+            const uint16_t *kb = k + ((size_t)b * Hkv + g) * (size_t)S * D;
+            const uint16_t *vb = v + ((size_t)b * Hkv + g) * (size_t)S * D;
+            const uint16_t *qr = q + (size_t)row * D, *dor = dout + (size_t)row * D;
+            double *out = dq + (size_t)r * D;
+            for (int d = 0; d < D; ++d) out[d] = 0.0;
+            double m = -INFINITY;
+            for (long j = 0; j < S; ++j) {
+                P[j] = -INFINITY;
+                if (!allowed_impl(L, S, i, j, causal, window, mrow, MUT_NONE)) continue;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d)
+                    acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kb[(size_t)j * D + d]);
+                P[j] = scale * acc;
+                if (P[j] > m) m = P[j];
+            }
+            if (m == -INFINITY) continue;
+            double denom = 0.0;
+            for (long j = 0; j < S; ++j) {
+                P[j] = (P[j] == -INFINITY) ? 0.0 : exp(P[j] - m);
+                denom += P[j];
+            }
+            double delta = 0.0;
+            for (long j = 0; j < S; ++j) {
+                P[j] /= denom;
+                dP[j] = 0.0;
+                if (P[j] == 0.0) continue;
+                for (int d = 0; d < D; ++d)
+                    dP[j] += bf16_bits_to_f64(dor[d]) * bf16_bits_to_f64(vb[(size_t)j * D + d]);
+                delta += P[j] * dP[j];
+            }
+            for (long j = 0; j < S; ++j) {
+                if (P[j] == 0.0) continue;
+                const double ds = P[j] * (dP[j] - delta);
+                for (int d = 0; d < D; ++d) out[d] += scale * ds * bf16_bits_to_f64(kb[(size_t)j * D + d]);
+            }
+        }
+        free(P);
+        free(dP);
+    }
+    return failed ? 5 : 0;
+}
+
+/* dK and dV of the listed keys of KV head g of batch b only (dk, dv hold
+ * nkeys x D each): every query row of the group's heads still needs its full
+ * softmax normalisation and row term, but only the listed keys' products are
+ * accumulated.  Same arithmetic as backward_impl; parallel over query rows
+ * with per-thread accumulators reduced at the end. */
+int oracle_attention_backward_kv_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                      const uint16_t *dout, double *dk, double *dv, int B, int Hq,
+                                      int Hkv, int L, int S, int D, double scale, int causal,
+                                      int window, const float *key_mask, int b, int g,
+                                      const int64_t *keys, int64_t nkeys, int nthreads)
+{
+    int rc = check_args(q, k, v, dk, B, Hq, Hkv, L, S, D);
+    if (rc) return rc;
+    if (!dout || !dv || !keys) return 1;
+    if (b < 0 || b >= B || g < 0 || g >= Hkv) return 4;
+    for (int64_t t = 0; t < nkeys; ++t)
+        if (keys[t] < 0 || keys[t] >= S) return 4;
+    const int G = Hq / Hkv;
+    memset(dk, 0, sizeof(double) * (size_t)nkeys * D);
+    memset(dv, 0, sizeof(double) * (size_t)nkeys * D);
+    const float *mrow = key_mask ? key_mask + (size_t)b * S : NULL;
+    const uint16_t *kb = k + ((size_t)b * Hkv + g) * (size_t)S * D;
+    const uint16_t *vb = v + ((size_t)b * Hkv + g) * (size_t)S * D;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *P = (double *)malloc(sizeof(double) * (size_t)S);
+        double *dP = (double *)malloc(sizeof(double) * (size_t)S);
+        double *ak = (double *)calloc((size_t)nkeys * D, sizeof(double));
+        double *av = (double *)calloc((size_t)nkeys * D, sizeof(double));
+        if (!P || !dP || !ak || !av) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 8)
+        for (long hi = 0; hi < (long)G * L; ++hi) {
+            if (!P || !dP || !ak || !av) continue;
+            const int h = g * G + (int)(hi / L);
+            const long i = hi % L;
+            const size_t row = (((size_t)b * Hq + h) * L + i) * D;
+            const uint16_t *qr = q + row, *dor = dout + row;
+            double m = -INFINITY;
+            for (long j = 0; j < S; ++j) {
+                P[j] = -INFINITY;
+                if (!allowed_impl(L, S, i, j, causal, window, mrow, MUT_NONE)) continue;
+                double acc = 0.0;
+                for (int d = 0; d < D; ++d)
+                    acc += bf16_bits_to_f64(qr[d]) * bf16_bits_to_f64(kb[(size_t)j * D + d]);
+                P[j] = scale * acc;
+                if (P[j] > m) m = P[j];
+            }
+            if (m == -INFINITY) continue;
+            double denom = 0.0;
+            for (long j = 0; j < S; ++j) {
+                P[j] = (P[j] == -INFINITY) ? 0.0 : exp(P[j] - m);
+                denom += P[j];
+            }
+            double delta = 0.0;
+            for (long j = 0; j < S; ++j) {
+                P[j] /= denom;
+                dP[j] = 0.0;
+                if (P[j] == 0.0) continue;
+                for (int d = 0; d < D; ++d)
+                    dP[j] += bf16_bits_to_f64(dor[d]) * bf16_bits_to_f64(vb[(size_t)j * D + d]);
+                delta += P[j] * dP[j];
+            }
+            for (int64_t t = 0; t < nkeys; ++t) {
+                const long j = (long)keys[t];
+                if (P[j] == 0.0) continue;
+                const double ds = P[j] * (dP[j] - delta);
+                for (int d = 0; d < D; ++d) {
+                    av[(size_t)t * D + d] += P[j] * bf16_bits_to_f64(dor[d]);
+                    ak[(size_t)t * D + d] += scale * ds * bf16_bits_to_f64(qr[d]);
+                }
+            }
+        }
+#pragma omp critical
+        {
+            if (ak && av)
+                for (size_t e = 0; e < (size_t)nkeys * D; ++e) {
+                    dk[e] += ak[e];
+                    dv[e] += av[e];
+                }
+        }
+        free(P);
+        free(dP);
+        free(ak);
+        free(av);
+    }
+    return failed ? 5 : 0;
+}
+
 int oracle_attention_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                               const uint16_t *dout, double *dq, double *dk, double *dv, int B,
                               int Hq, int Hkv, int L, int S, int D, double scale, int causal,

@@ -18,7 +18,7 @@ import torch
 
 import oracle
 from sliding_window_gqa_tfa_b200 import binding as tb
-from sliding_window_gqa_tfa_b200.inputs import make_inputs, shaped
+from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_dout, make_inputs, shaped
 
 pytestmark = pytest.mark.gpu
 
@@ -119,3 +119,64 @@ def test_backward_keys_no_row_sees_are_zero():
     _check(dq, rq, bq, "dq")
     _check(dk, rk, bk, "dk")
     _check(dv, rv, bv, "dv")
+
+
+def _row_softmax(scores, allowed):
+    s = np.where(allowed, scores, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    m = np.where(np.isfinite(m), m, 0.0)
+    e = np.where(allowed, np.exp(s - m), 0.0)
+    d = e.sum(axis=-1, keepdims=True)
+    return e / np.where(d > 0, d, 1.0)
+
+
+def test_backward_full_size_sampled():
+    """The benchmark's backward workload, launched as the benchmark launches it:
+    dQ on sampled rows and dK/dV on sampled keys of one KV group against the
+    oracle's row entries, with the per-element bound of the small cases."""
+    w = WORKLOADS["llama_gqa_chunk_2048x8192_backward"]
+    q, k, v, km = make_inputs(w, seed=0)
+    do = make_dout(w, seed=0)
+    dq, dk, dv = tb.backward(q.cuda(), k.cuda(), v.cuda(), do.cuda(), scale=w.softmax_scale,
+                             causal=w.causal, window=w.window)
+    tb.check_status()
+    s, G, P0 = w.softmax_scale, w.Hq // w.Hkv, w.S - w.L
+    Q, K, V, dO = (t.double().numpy() for t in (q, k, v, do))
+    keys_all = np.arange(w.S)
+    # dQ rows
+    rng = np.random.default_rng(3)
+    rows = np.unique(np.concatenate([[0, w.L - 1, 127, 128, 1023, 2047],
+                                     rng.integers(0, w.Hq * w.L, 58)]))
+    ref = oracle.attention_backward_dq_rows(q, k, v, do, rows, scale=s, causal=True)
+    O = oracle.attention(q, k, v, scale=s, causal=True, rows=rows)
+    got = dq.reshape(-1, w.D)[torch.as_tensor(rows, device=dq.device)]
+    bound = np.zeros_like(ref)
+    for n, row in enumerate(rows):
+        h, i = divmod(int(row), w.L)
+        g = h // G
+        allowed = keys_all <= P0 + i
+        Prow = _row_softmax(s * (K[0, g] @ Q[0, h, i]), allowed)
+        dP = V[0, g] @ dO[0, h, i]
+        dS = Prow * (dP - (Prow * dP).sum())
+        e = np.abs(dO[0, h, i] * O[n]).sum()
+        bound[n] = EPS * s * (np.abs(dS) @ np.abs(K[0, g]) + e * (Prow @ np.abs(K[0, g])))
+    ratio = _check(got, ref, bound, "full-size dq rows")
+    # dK / dV of sampled keys of the last KV group
+    g = w.Hkv - 1
+    keys = np.unique(np.concatenate([[0, 127, 128, 6143, 6144, 8191], rng.integers(0, w.S, 18)]))
+    rk, rv = oracle.attention_backward_kv_rows(q, k, v, do, b=0, g=g, keys=keys, scale=s, causal=True)
+    bk = np.zeros_like(rk)
+    bv = np.zeros_like(rv)
+    allowed = keys_all[None, :] <= P0 + np.arange(w.L)[:, None]
+    for h in range(g * G, (g + 1) * G):
+        Ph = _row_softmax(s * (Q[0, h] @ K[0, g].T), allowed)
+        dPh = dO[0, h] @ V[0, g].T
+        dSh = Ph * (dPh - (Ph * dPh).sum(axis=1, keepdims=True))
+        Oh = Ph @ V[0, g]
+        eh = np.abs(dO[0, h] * Oh).sum(axis=1)
+        bv += EPS * (Ph[:, keys].T @ np.abs(dO[0, h]))
+        bk += EPS * s * (np.abs(dSh[:, keys]).T @ np.abs(Q[0, h]) + (Ph[:, keys] * eh[:, None]).T @ np.abs(Q[0, h]))
+    kk = torch.as_tensor(keys, device=dk.device)
+    rk_ratio = _check(dk[0, g][kk], rk, bk, "full-size dk rows")
+    rv_ratio = _check(dv[0, g][kk], rv, bv, "full-size dv rows")
+    print("full size worst error / bound", f"{ratio:.3g} {rk_ratio:.3g} {rv_ratio:.3g}")

@@ -132,3 +132,33 @@ def test_backward_planted_mistake_fails_a_pin(mutation):
         except AssertionError:
             caught.append(pin.__name__)
     assert caught, f"mutation {mutation} passed every pin"
+
+
+def test_dq_rows_equal_the_full_backward():
+    """The per-row dQ entry (used at sizes the full oracle cannot reach) against
+    the full oracle backward (itself pinned above)."""
+    w = shaped(2, 6, 2, 40, 90, 32, key_mask_keep=0.8)
+    q, k, v, km = make_inputs(w, seed=81)
+    do = _dout(q.shape, 82)
+    for causal, window in [(True, 0), (True, 9), (False, 0)]:
+        dq, _, _ = oracle.attention_backward(q, k, v, do, scale=0.3, causal=causal, window=window,
+                                             key_mask=km)
+        rows = np.array([0, 5, 39, 40, 41, 150, 479], dtype=np.int64)
+        got = oracle.attention_backward_dq_rows(q, k, v, do, rows, scale=0.3, causal=causal,
+                                                window=window, key_mask=km)
+        assert np.array_equal(got, dq.reshape(-1, w.D)[rows])
+
+
+def test_kv_rows_equal_the_full_backward():
+    w = shaped(2, 6, 2, 40, 90, 32, key_mask_keep=0.8)
+    q, k, v, km = make_inputs(w, seed=83)
+    do = _dout(q.shape, 84)
+    for causal, window in [(True, 0), (True, 9), (False, 0)]:
+        _, dk, dv = oracle.attention_backward(q, k, v, do, scale=0.3, causal=causal, window=window,
+                                              key_mask=km)
+        keys = [0, 3, 49, 50, 88, 89]
+        for b, g in [(0, 0), (1, 1)]:
+            gk, gv = oracle.attention_backward_kv_rows(q, k, v, do, b=b, g=g, keys=keys, scale=0.3,
+                                                       causal=causal, window=window, key_mask=km)
+            assert np.allclose(gk, dk[b, g, keys], atol=1e-13, rtol=1e-12)
+            assert np.allclose(gv, dv[b, g, keys], atol=1e-13, rtol=1e-12)
