@@ -35,6 +35,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sliding_window_gqa_tfa_b200 import binding as tb  # noqa: E402
+from sliding_window_gqa_tfa_b200.dist import (barrier, max_over_ranks, setup,  # noqa: E402
+                                              teardown, weak_scaling_rate)
 from sliding_window_gqa_tfa_b200.flops import workload_bytes, workload_flops  # noqa: E402
 from sliding_window_gqa_tfa_b200.inputs import (HEADLINE, WORKLOADS, make_dout,  # noqa: E402
                                                 make_inputs, make_sinks, varlen_cu)
@@ -130,38 +132,6 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
                 "reasons": sorted(reasons), "samples": len(sm)}
-
-
-def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.barrier()
-
-
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
 
 
 def cpu_threads():
@@ -316,7 +286,7 @@ def main():
     if args.impl == "reference":
         return run_reference(args, w)
 
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = setup("nccl")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     tb.lib()  # fail loudly if the library is missing
@@ -382,7 +352,7 @@ def main():
     per = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
     mean_ms = sum(per) / len(per)
     mean_ms = max_over_ranks(mean_ms, world)
-    value = flops * world / (mean_ms * 1e-3) / 1e12
+    value = weak_scaling_rate(flops, world, mean_ms * 1e-3) / 1e12
     per_sorted = sorted(per)
 
     # end to end through the C ABI with host buffers (copies inside the timed region)
@@ -472,10 +442,7 @@ def main():
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.destroy_process_group()
+    teardown(world)
     return 0
 
 
