@@ -42,11 +42,13 @@ struct BwdScratch {
     size_t rows = 0, o_bytes = 0;
 };
 
+constexpr int kVariantsPerD = 10;  // forward kernel variants per head dim (variant_index)
+
 struct DeviceState {
     bool init = false;
     int sm_count = 0;
     unsigned *status = nullptr;  // device status word (TFA_DEVICE_TIMEOUT bits)
-    bool smem_attr[8] = {};  // per kernel variant: D, key mask, softcap
+    bool smem_attr[2 * kVariantsPerD] = {};  // per kernel variant: D, layout, key mask, score mode
     std::unordered_map<cudaStream_t, SplitScratch> split;
     std::unordered_map<cudaStream_t, BwdScratch> bwd;
     bool bwd_attr[4] = {};  // backward kernels prepared, per (D, key mask)
@@ -83,17 +85,22 @@ int get_encode_fn() {
     return TFA_OK;
 }
 
+// Kernel variants per head dim: dense (key mask x score mode: 6), then ring
+// and varlen (plain or softcap: 2 each; neither takes a key mask or writes LSE).
+constexpr int variant_index(int D, bool km, int mode, int layout) {
+    return (D == 128 ? kVariantsPerD : 0) +
+           (layout == tfa::kLayoutDense ? 2 * mode + (km ? 1 : 0) : 4 + 2 * layout + (mode == tfa::kModeSoftcap));
+}
+
 // Shared-memory opt-in and the register check for one kernel variant, done
 // once per device at first use (never lazily, so a captured call needs neither).
-constexpr int variant_index(int D, bool km, bool sc) { return (D == 128 ? 4 : 0) + (sc ? 2 : 0) + (km ? 1 : 0); }
-
-template <int D, bool KM, bool SC>
+template <int D, bool KM, int MODE, int LY>
 int prepare_kernel(DeviceState &st) {
     using C = tfa::Cfg<D>;
-    auto kern = tfa::tfa_prefill_kernel<D, KM, SC>;
+    auto kern = tfa::tfa_prefill_kernel<D, KM, MODE, LY>;
     // the largest launch of this variant: with a key mask, or a varlen table
     const int smem = KM ? C::kSmemBytesKeyMask : C::kSmemBytesVarlen;
-    const int which = variant_index(D, KM, SC);
+    const int which = variant_index(D, KM, MODE, LY);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
     cudaFuncAttributes fa;
@@ -122,15 +129,25 @@ int prepare_bwd_kernels(DeviceState &st) {
     return TFA_OK;
 }
 
+template <int D>
+int prepare_forward_kernels(DeviceState &st) {
+    using namespace tfa;
+    int rc = prepare_kernel<D, false, kModePlain, kLayoutDense>(st);
+    if (!rc) rc = prepare_kernel<D, true, kModePlain, kLayoutDense>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutDense>(st);
+    if (!rc) rc = prepare_kernel<D, true, kModeSoftcap, kLayoutDense>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeLse, kLayoutDense>(st);
+    if (!rc) rc = prepare_kernel<D, true, kModeLse, kLayoutDense>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModePlain, kLayoutRing>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutRing>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModePlain, kLayoutVarlen>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutVarlen>(st);
+    return rc;
+}
+
 int prepare_all_kernels(DeviceState &st) {
-    int rc = prepare_kernel<64, false, false>(st);
-    if (!rc) rc = prepare_kernel<64, true, false>(st);
-    if (!rc) rc = prepare_kernel<64, false, true>(st);
-    if (!rc) rc = prepare_kernel<64, true, true>(st);
-    if (!rc) rc = prepare_kernel<128, false, false>(st);
-    if (!rc) rc = prepare_kernel<128, true, false>(st);
-    if (!rc) rc = prepare_kernel<128, false, true>(st);
-    if (!rc) rc = prepare_kernel<128, true, true>(st);
+    int rc = prepare_forward_kernels<64>(st);
+    if (!rc) rc = prepare_forward_kernels<128>(st);
     if (!rc) rc = prepare_bwd_kernels<64, false>(st);
     if (!rc) rc = prepare_bwd_kernels<64, true>(st);
     if (!rc) rc = prepare_bwd_kernels<128, false>(st);
@@ -304,13 +321,27 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
              encode_map(&mk, k, S, B * Hkv, D) || encode_map(&mv, v, S, B * Hkv, D);
     if (rc) return TFA_ERR_CUDA;
     // separate instantiations with and without a key mask (the mask costs an
-    // extra MMA per score tile and extra shared memory) and a softcap (extra
-    // work per score); plain calls carry neither
+    // extra MMA per score tile and extra shared memory), a softcap (extra work
+    // per score) and the log-sum-exp output; plain calls carry none of them
     const bool sc = softcap > 0.f;
-    auto kern = key_mask ? (sc ? tfa::tfa_prefill_kernel<D, true, true> : tfa::tfa_prefill_kernel<D, true, false>)
-                         : (sc ? tfa::tfa_prefill_kernel<D, false, true> : tfa::tfa_prefill_kernel<D, false, false>);
+    if (sc && ad.lse) return TFA_ERR_SOFTCAP;  // no variant computes both (the backward has no softcap)
+    const int mode = ad.lse ? tfa::kModeLse : sc ? tfa::kModeSoftcap : tfa::kModePlain;
+    const int layout = varlen ? tfa::kLayoutVarlen : ad.ring_rows ? tfa::kLayoutRing : tfa::kLayoutDense;
+    if (layout != tfa::kLayoutDense && (key_mask || ad.lse)) return TFA_ERR_RING;  // not instantiated
+    using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const tfa::Params);
+    using namespace tfa;
+    static const Kern dense[3][2] = {  // [mode][key mask]
+        {tfa_prefill_kernel<D, false, kModePlain, kLayoutDense>, tfa_prefill_kernel<D, true, kModePlain, kLayoutDense>},
+        {tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutDense>,
+         tfa_prefill_kernel<D, true, kModeSoftcap, kLayoutDense>},
+        {tfa_prefill_kernel<D, false, kModeLse, kLayoutDense>, tfa_prefill_kernel<D, true, kModeLse, kLayoutDense>}};
+    static const Kern other[2][2] = {  // [ring, varlen][plain, softcap]
+        {tfa_prefill_kernel<D, false, kModePlain, kLayoutRing>, tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutRing>},
+        {tfa_prefill_kernel<D, false, kModePlain, kLayoutVarlen>,
+         tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutVarlen>}};
+    const Kern kern = layout == kLayoutDense ? dense[mode][key_mask ? 1 : 0] : other[layout - 1][sc ? 1 : 0];
     const int smem = key_mask ? C::kSmemBytesKeyMask : varlen ? C::kSmemBytesVarlen : C::kSmemBytes;
-    const int which = variant_index(D, key_mask != nullptr, sc);
+    const int which = variant_index(D, key_mask != nullptr, mode, layout);
     if (!st.smem_attr[which]) return drv_fail("kernel not prepared", which);
     tfa::Params p;
     p.o = static_cast<__nv_bfloat16 *>(o);
@@ -332,7 +363,6 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.softcap_u = sc ? scale / softcap : 0.f;
     p.sinks = sinks;
     p.ring_rows = ad.ring_rows;
-    p.varlen = varlen ? 1 : 0;
     p.total_q = ad.total_q;
     p.total_k = ad.total_k;
     p.cu_q = ad.cu_q;

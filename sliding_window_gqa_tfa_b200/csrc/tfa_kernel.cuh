@@ -144,10 +144,10 @@ struct Params {
     // rotating cache: K/V hold ring_rows rows and key position j sits in row
     // j mod ring_rows (0: K/V hold all S keys in order)
     int ring_rows;
-    // packed variable-length batch: q/o [total_q, Hq, D], k/v [total_k, Hkv, D],
-    // sequence b = rows [cu_q[b], cu_q[b+1]) / [cu_k[b], cu_k[b+1]); shape.L is
-    // the longest query (max_seqlen_q)
-    int varlen, total_q, total_k;
+    // packed variable-length batch (the varlen layout): q/o [total_q, Hq, D],
+    // k/v [total_k, Hkv, D], sequence b = rows [cu_q[b], cu_q[b+1]) /
+    // [cu_k[b], cu_k[b+1]); shape.L is the longest query (max_seqlen_q)
+    int total_q, total_k;
     const int *cu_q, *cu_k;
     // optional per-row log-sum-exp in base 2 of the scaled scores,
     // log2(sum_j 2^(s_j * scale_log2)) (+inf for a row with no allowed key),
@@ -208,12 +208,17 @@ __device__ __forceinline__ uint8_t *smem_base() {
     return smem_raw + (((raw + 1023u) & ~1023u) - raw);
 }
 
+// Where K and V rows live, fixed at compile time so that a dense call carries
+// no code for the others: [B*H][rows][D] planes, a rotating cache of ring_rows
+// rows per plane, or packed variable-length sequences [total][H][D].
+enum Layout : int { kLayoutDense = 0, kLayoutRing = 1, kLayoutVarlen = 2 };
+
 // Start the CTA's piece iterator (with the validated sequence table for a
 // packed variable-length call).
-template <int D>
+template <int D, int LY>
 __device__ __forceinline__ void iter_init(SegIter &it, const Params &p) {
     it.init(p.shape, p.W, blockIdx.x);
-    if (p.varlen) {
+    if constexpr (LY == kLayoutVarlen) {
         const int *tab = reinterpret_cast<const int *>(smem_base() + Cfg<D>::kTableOff);
         it.seq.q_start = tab;
         it.seq.q_len = tab + kMaxVarlenSeqs;
@@ -274,7 +279,7 @@ struct Bars {
 };
 
 // ------------------------------------------------------------------ producer
-template <int D, bool KM>
+template <int D, bool KM, int LY>
 __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                           const CUtensorMap *tm_v, uint32_t sbase, uint8_t *gbase, const Bars &bar,
                           volatile int *abort_flag) {
@@ -288,7 +293,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
     uint32_t kv_prod = 0;
     uint32_t q_use[2] = {0, 0};
     SegIter it;
-    iter_init<D>(it, p);
+    iter_init<D, LY>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
         const ItemPlan ip = plan_piece(p, seg);
@@ -307,7 +312,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                                     tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0);
                 } else {  // dense: plane b*Hq + h; varlen: packed rows, plane h
                     mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
-                    const int plane = p.varlen ? ip.h : ip.b * p.Hq + ip.h;
+                    const int plane = LY == kLayoutVarlen ? ip.h : ip.b * p.Hq + ip.h;
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
                                     tm_q, bar.q_full(t), cb * 64, ip.q_row0 + ip.q0[t], plane);
@@ -339,7 +344,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                 if (lane == 0) {
                     mbar_arrive_expect_tx(bar.kv_full(s), C::kTileBytes);
                     const uint32_t dst = sbase + C::kKVOff + s * C::kTileBytes;
-                    if (p.ring_rows) {
+                    if constexpr (LY == kLayoutRing) {
                         // rotating cache: two 64-row boxes, each contiguous in
                         // the ring (ring_rows is a multiple of 64)
                         for (int hf = 0; hf < 2; ++hf) {
@@ -349,7 +354,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                                             bar.kv_full(s), cb * 64, row, ip.b * p.Hkv + ip.g);
                         }
                     } else {
-                        const int plane = p.varlen ? ip.g : ip.b * p.Hkv + ip.g;
+                        const int plane = LY == kLayoutVarlen ? ip.g : ip.b * p.Hkv + ip.g;
                         for (int cb = 0; cb < C::kColBlocks; ++cb)
                             tma_load_3d(dst + cb * C::kColBlockBytes, which ? tm_v : tm_k, bar.kv_full(s),
                                         cb * 64, ip.k_row0 + j * kBlockK, plane);
@@ -373,7 +378,7 @@ out:
 }
 
 // ------------------------------------------------------------ tensor cores
-template <int D, bool KM>
+template <int D, bool KM, int LY>
 __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const Bars &bar,
                          volatile int *abort_flag) {
     using C = Cfg<D>;
@@ -428,7 +433,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     int trace_step = 0;
     (void)trace_step;
     SegIter it;
-    iter_init<D>(it, p);
+    iter_init<D, LY>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
         const ItemPlan ip = plan_piece(p, seg);
@@ -514,10 +519,16 @@ __device__ __forceinline__ float add_sink(const Params &p, float l, float m, flo
     return l + ex2(fmaf(__ldg(p.sinks + head), kLog2e, -m * c));
 }
 
-template <int D, bool KM, bool SC>
+// Epilogue / score variants of the kernel, fixed at compile time so that a
+// plain call carries no code for the others: a softcap on the scores, or the
+// per-row log-sum-exp written beside the output (for a backward pass).
+enum ScoreMode : int { kModePlain = 0, kModeSoftcap = 1, kModeLse = 2 };
+
+template <int D, bool KM, int MODE, int LY>
 __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint32_t tmem,
                                           const Bars &bar, volatile int *abort_flag) {
     using C = Cfg<D>;
+    constexpr bool SC = MODE == kModeSoftcap;
     const int r = threadIdx.x - t * 128;  // row inside the query tile
     const uint32_t lane_base = (static_cast<uint32_t>((threadIdx.x >> 5) & 3) * 32u) << 16;
     const uint32_t tS = tmem + C::kTmemS + t * 128 + lane_base;
@@ -531,7 +542,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     (void)trace_step;
 
     SegIter it;
-    iter_init<D>(it, p);
+    iter_init<D, LY>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
         const ItemSpan sp = seg_span(p.shape, seg);
@@ -775,13 +786,13 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         // l == 0 and is written as zeros).
         if (!warp_live) continue;
         if (row_live) l = add_sink(p, l, m_star, c, out_head);  // m_star == m_ref for a whole tile
-        if (p.lse && row_valid)
+        if (MODE == kModeLse && row_valid)
             p.lse[static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row] =
                 l > 0.f ? fmaf(m_star, c, __log2f(l)) : CUDART_INF_F;
         const float inv = l > 0.f ? 1.f / l : 0.f;
         __nv_bfloat16 *orow = nullptr;
         if (row_valid)  // dense [B,Hq,L,D]; varlen packed [total_q, Hq, D]
-            orow = p.o + (p.varlen ? static_cast<size_t>(seg.q_base + row) * p.Hq + out_head
+            orow = p.o + (LY == kLayoutVarlen ? static_cast<size_t>(seg.q_base + row) * p.Hq + out_head
                                    : static_cast<size_t>(seg.b * p.Hq + out_head) * p.L + row) *
                              static_cast<size_t>(D);
 #pragma unroll
@@ -825,7 +836,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, bool KM, bool SC>
+template <int D, bool KM, int MODE, int LY>
 __global__ void __launch_bounds__(kThreads, 1)
     tfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -876,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<uint16_t *>(gbase + C::kOnesOff + bias_offset(n, 0)) = 0x3F80u;
         fence_proxy_async_smem();
     }
-    if (p.varlen && warp < 8) {
+    if (LY == kLayoutVarlen && warp < 8) {
         // validated copy of cu_seqlens; a bad sequence is skipped and reported
         int *tab = reinterpret_cast<int *>(gbase + C::kTableOff);
         for (int b = threadIdx.x; b < p.B; b += 256) {
@@ -906,12 +917,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         reg_alloc<kRegsSoftmax>();
-        softmax_role<D, KM, SC>(p, warp >> 2, tmem, bar, abort_flag);
+        softmax_role<D, KM, MODE, LY>(p, warp >> 2, tmem, bar, abort_flag);
     } else {
         reg_dealloc<kRegsOther>();
         if (warp == 8 && (lane == 0 || KM))
-            load_role<D, KM>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
-        if (warp == 9 && lane == 0) mma_role<D, KM>(p, sbase, tmem, bar, abort_flag);
+            load_role<D, KM, LY>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
+        if (warp == 9 && lane == 0) mma_role<D, KM, LY>(p, sbase, tmem, bar, abort_flag);
     }
 
     tc_fence_before();

@@ -159,7 +159,7 @@ def test_varlen_empty_and_rejected_calls():
     assert e.value.code == tb.TFA_ERR_WINDOW
 
 
-@pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items() if w.kind != "dense"])
+@pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items() if w.kind in ("ring", "varlen")])
 def test_full_size_workloads_sampled(name):
     """The benchmark's rotating-cache and variable-length workloads, launched as
     the benchmark launches them, on rows the oracle computes one by one."""
