@@ -42,7 +42,7 @@ struct BwdScratch {
     size_t rows = 0, o_bytes = 0;
 };
 
-constexpr int kVariantsPerD = 10;  // forward kernel variants per head dim (variant_index)
+constexpr int kVariantsPerD = 18;  // forward kernel variants per head dim (variant_index)
 
 struct DeviceState {
     bool init = false;
@@ -85,22 +85,26 @@ int get_encode_fn() {
     return TFA_OK;
 }
 
-// Kernel variants per head dim: dense (key mask x score mode: 6), then ring
-// and varlen (plain or softcap: 2 each; neither takes a key mask or writes LSE).
-constexpr int variant_index(int D, bool km, int mode, int layout) {
-    return (D == 128 ? kVariantsPerD : 0) +
-           (layout == tfa::kLayoutDense ? 2 * mode + (km ? 1 : 0) : 4 + 2 * layout + (mode == tfa::kModeSoftcap));
+// Kernel variants per head dim: dense (packed x key mask x score mode: 12),
+// ring (packed x plain/softcap: 4) and varlen (plain/softcap: 2); ring and
+// varlen take no key mask and write no LSE, varlen is never packed.
+constexpr int variant_index(int D, bool km, int mode, int layout, bool pk) {
+    const int sc = mode == tfa::kModeSoftcap ? 1 : 0;
+    const int v = layout == tfa::kLayoutDense ? (pk ? 6 : 0) + 2 * mode + (km ? 1 : 0)
+                  : layout == tfa::kLayoutRing ? 12 + (pk ? 2 : 0) + sc
+                                               : 16 + sc;
+    return (D == 128 ? kVariantsPerD : 0) + v;
 }
 
 // Shared-memory opt-in and the register check for one kernel variant, done
 // once per device at first use (never lazily, so a captured call needs neither).
-template <int D, bool KM, int MODE, int LY>
+template <int D, bool KM, int MODE, int LY, bool PK>
 int prepare_kernel(DeviceState &st) {
     using C = tfa::Cfg<D>;
-    auto kern = tfa::tfa_prefill_kernel<D, KM, MODE, LY>;
+    auto kern = tfa::tfa_prefill_kernel<D, KM, MODE, LY, PK>;
     // the largest launch of this variant: with a key mask, or a varlen table
     const int smem = KM ? C::kSmemBytesKeyMask : C::kSmemBytesVarlen;
-    const int which = variant_index(D, KM, MODE, LY);
+    const int which = variant_index(D, KM, MODE, LY, PK);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(max dynamic smem)", e);
     cudaFuncAttributes fa;
@@ -129,19 +133,27 @@ int prepare_bwd_kernels(DeviceState &st) {
     return TFA_OK;
 }
 
+template <int D, bool PK>
+int prepare_dense_kernels(DeviceState &st) {
+    using namespace tfa;
+    int rc = prepare_kernel<D, false, kModePlain, kLayoutDense, PK>(st);
+    if (!rc) rc = prepare_kernel<D, true, kModePlain, kLayoutDense, PK>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutDense, PK>(st);
+    if (!rc) rc = prepare_kernel<D, true, kModeSoftcap, kLayoutDense, PK>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeLse, kLayoutDense, PK>(st);
+    if (!rc) rc = prepare_kernel<D, true, kModeLse, kLayoutDense, PK>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModePlain, kLayoutRing, PK>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutRing, PK>(st);
+    return rc;
+}
+
 template <int D>
 int prepare_forward_kernels(DeviceState &st) {
     using namespace tfa;
-    int rc = prepare_kernel<D, false, kModePlain, kLayoutDense>(st);
-    if (!rc) rc = prepare_kernel<D, true, kModePlain, kLayoutDense>(st);
-    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutDense>(st);
-    if (!rc) rc = prepare_kernel<D, true, kModeSoftcap, kLayoutDense>(st);
-    if (!rc) rc = prepare_kernel<D, false, kModeLse, kLayoutDense>(st);
-    if (!rc) rc = prepare_kernel<D, true, kModeLse, kLayoutDense>(st);
-    if (!rc) rc = prepare_kernel<D, false, kModePlain, kLayoutRing>(st);
-    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutRing>(st);
-    if (!rc) rc = prepare_kernel<D, false, kModePlain, kLayoutVarlen>(st);
-    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutVarlen>(st);
+    int rc = prepare_dense_kernels<D, false>(st);
+    if (!rc) rc = prepare_dense_kernels<D, true>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModePlain, kLayoutVarlen, false>(st);
+    if (!rc) rc = prepare_kernel<D, false, kModeSoftcap, kLayoutVarlen, false>(st);
     return rc;
 }
 
@@ -328,20 +340,29 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     const int mode = ad.lse ? tfa::kModeLse : sc ? tfa::kModeSoftcap : tfa::kModePlain;
     const int layout = varlen ? tfa::kLayoutVarlen : ad.ring_rows ? tfa::kLayoutRing : tfa::kLayoutDense;
     if (layout != tfa::kLayoutDense && (key_mask || ad.lse)) return TFA_ERR_RING;  // not instantiated
+    if (varlen && packed) return TFA_ERR_RING;  // not instantiated
     using Kern = void (*)(const CUtensorMap, const CUtensorMap, const CUtensorMap, const tfa::Params);
     using namespace tfa;
-    static const Kern dense[3][2] = {  // [mode][key mask]
-        {tfa_prefill_kernel<D, false, kModePlain, kLayoutDense>, tfa_prefill_kernel<D, true, kModePlain, kLayoutDense>},
-        {tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutDense>,
-         tfa_prefill_kernel<D, true, kModeSoftcap, kLayoutDense>},
-        {tfa_prefill_kernel<D, false, kModeLse, kLayoutDense>, tfa_prefill_kernel<D, true, kModeLse, kLayoutDense>}};
-    static const Kern other[2][2] = {  // [ring, varlen][plain, softcap]
-        {tfa_prefill_kernel<D, false, kModePlain, kLayoutRing>, tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutRing>},
-        {tfa_prefill_kernel<D, false, kModePlain, kLayoutVarlen>,
-         tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutVarlen>}};
-    const Kern kern = layout == kLayoutDense ? dense[mode][key_mask ? 1 : 0] : other[layout - 1][sc ? 1 : 0];
+#define TFA_DENSE(PK)                                                                               \
+    {{tfa_prefill_kernel<D, false, kModePlain, kLayoutDense, PK>,                                   \
+      tfa_prefill_kernel<D, true, kModePlain, kLayoutDense, PK>},                                   \
+     {tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutDense, PK>,                                 \
+      tfa_prefill_kernel<D, true, kModeSoftcap, kLayoutDense, PK>},                                 \
+     {tfa_prefill_kernel<D, false, kModeLse, kLayoutDense, PK>, tfa_prefill_kernel<D, true, kModeLse, kLayoutDense, PK>}}
+    static const Kern dense[2][3][2] = {TFA_DENSE(false), TFA_DENSE(true)};  // [packed][mode][key mask]
+#undef TFA_DENSE
+    static const Kern ring[2][2] = {  // [packed][plain, softcap]
+        {tfa_prefill_kernel<D, false, kModePlain, kLayoutRing, false>,
+         tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutRing, false>},
+        {tfa_prefill_kernel<D, false, kModePlain, kLayoutRing, true>,
+         tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutRing, true>}};
+    static const Kern vlen[2] = {tfa_prefill_kernel<D, false, kModePlain, kLayoutVarlen, false>,
+                                 tfa_prefill_kernel<D, false, kModeSoftcap, kLayoutVarlen, false>};
+    const Kern kern = layout == kLayoutDense ? dense[packed ? 1 : 0][mode][key_mask ? 1 : 0]
+                      : layout == kLayoutRing ? ring[packed ? 1 : 0][sc ? 1 : 0]
+                                              : vlen[sc ? 1 : 0];
     const int smem = key_mask ? C::kSmemBytesKeyMask : varlen ? C::kSmemBytesVarlen : C::kSmemBytes;
-    const int which = variant_index(D, key_mask != nullptr, mode, layout);
+    const int which = variant_index(D, key_mask != nullptr, mode, layout, packed);
     if (!st.smem_attr[which]) return drv_fail("kernel not prepared", which);
     tfa::Params p;
     p.o = static_cast<__nv_bfloat16 *>(o);

@@ -52,7 +52,7 @@ namespace tfa {
 #ifdef TFA_TRACE
 constexpr int kTraceSlots = 2048;
 __device__ unsigned long long g_tfa_trace[8][kTraceSlots];
-__device__ unsigned long long g_tfa_cta_time[1024][4];  // global-timer ns: start, end, softmax done, spare
+__device__ unsigned long long g_tfa_cta_time[1024][4];  // global-timer ns: start, end, softmax done, packed merge start
 #define TFA_TR(role, step, ev)                                                      \
     do {                                                                            \
         const int _i = 8 * (step) + (ev);                                           \
@@ -166,7 +166,7 @@ struct Params {
     // Short-query (decode) mapping: a query tile holds the rows of pack_heads
     // query heads of one KV group, row m = (head m / L, query row m % L);
     // shape.Hq then counts Hkv * pack_chunks "virtual heads", one per tile.
-    int packed, pack_heads, pack_chunks;
+    int packed, pack_heads, pack_chunks;  // packed: 1 exactly in the PK instantiations
 };
 
 // Rows of one packed tile: first real query head, heads present.
@@ -237,11 +237,15 @@ struct ItemPlan {
 };
 
 // The two query tiles of one piece of work, clipped to the piece's key tiles.
+template <bool PK>
 __device__ __forceinline__ ItemPlan plan_piece(const Params &p, const Segment &seg) {
     ItemPlan ip;
     ip.b = seg.b;
     ip.h = seg.h;
-    ip.g = p.packed ? seg.h / p.pack_chunks : seg.h / p.G;
+    // p.packed is tested at run time here and in the producer's Q load (always
+    // equal to PK): the compile-time form of these two tests measured ~3 %
+    // slower on dense prefill, with identical register and spill counts
+    ip.g = (PK || p.packed) ? seg.h / p.pack_chunks : seg.h / p.G;
     ip.jl = seg.jb;
     ip.jh = seg.je;
     ip.q_row0 = seg.q_base;
@@ -279,7 +283,7 @@ struct Bars {
 };
 
 // ------------------------------------------------------------------ producer
-template <int D, bool KM, int LY>
+template <int D, bool KM, int LY, bool PK>
 __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                           const CUtensorMap *tm_v, uint32_t sbase, uint8_t *gbase, const Bars &bar,
                           volatile int *abort_flag) {
@@ -296,7 +300,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
     iter_init<D, LY>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
-        const ItemPlan ip = plan_piece(p, seg);
+        const ItemPlan ip = plan_piece<PK>(p, seg);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (!ip.present[t]) continue;
@@ -304,7 +308,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                 !__all_sync(lanes, mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status)))
                 goto out;
             if (lane == 0) {
-                if (p.packed) {  // box {64, L, pack_heads}: rows (head, query row) in order
+                if (PK || p.packed) {  // box {64, L, pack_heads}: rows (head, query row) in order
                     const PackedRows pr = packed_rows(p, ip.h);
                     mbar_arrive_expect_tx(bar.q_full(t), C::kColBlocks * 128 * p.L * p.pack_heads);
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
@@ -378,7 +382,7 @@ out:
 }
 
 // ------------------------------------------------------------ tensor cores
-template <int D, bool KM, int LY>
+template <int D, bool KM, int LY, bool PK>
 __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const Bars &bar,
                          volatile int *abort_flag) {
     using C = Cfg<D>;
@@ -436,7 +440,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     iter_init<D, LY>(it, p);
     Segment seg;
     while (it.next(p.shape, seg)) {
-        const ItemPlan ip = plan_piece(p, seg);
+        const ItemPlan ip = plan_piece<PK>(p, seg);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
             if (!ip.present[t]) continue;
@@ -524,7 +528,127 @@ __device__ __forceinline__ float add_sink(const Params &p, float l, float m, flo
 // per-row log-sum-exp written beside the output (for a backward pass).
 enum ScoreMode : int { kModePlain = 0, kModeSoftcap = 1, kModeLse = 2 };
 
-template <int D, bool KM, int MODE, int LY>
+// Finalizer of a cut packed (short-query) tile, run by all 128 threads of
+// the tile's warpgroup once every row has stored its own partial in this
+// CTA's second slot (the first may still hold the partial this CTA published
+// for an earlier tile; a packed piece has no second query tile): the merge of all the tile's partials (tiny-llm Week 2 Day 5,
+// Task 1: m* = max m_k, l* = sum 2^(m_k - m*) l_k, a* = sum 2^(m_k - m*) a_k,
+// O = a* / l*), written straight to the output.  A packed tile has few live
+// rows but one partial per CTA of its key range, so the threads split the
+// flag waits and the (row, 4-column) elements between them instead of one
+// thread walking every partial of its row.  Returns false on an abort.
+template <int D, int MODE>
+__device__ __forceinline__ bool merge_packed(const Params &p, const Segment &seg, const ItemSpan &sp,
+                                          int t, int n_valid, unsigned epoch, volatile int *abort_flag) {
+    using C = Cfg<D>;
+    const int r = threadIdx.x - t * 128;
+    const float c = p.scale_log2;
+    const int c_last = last_contributor(p.W, gridDim.x, blockIdx.x, seg, sp, t);
+#ifdef TFA_TRACE
+    if (r == 0 && blockIdx.x < 1024) g_tfa_cta_time[blockIdx.x][3] = globaltimer_ns();
+#endif
+    bool ok = true;
+    for (int k = blockIdx.x + 1 + r; k <= c_last && ok; k += 128)
+        ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status);
+    // the slot writes of this warpgroup and the flags seen by it are ordered
+    // before every read below; all threads leave together on an abort
+    if (named_barrier_or(1 + t, 128, !ok || *abort_flag)) return false;
+    auto slot_of = [&](int k) {
+        return p.partial +
+               static_cast<size_t>(partial_slot(k, k == static_cast<int>(blockIdx.x) ? 1 : t)) * partial_slot_floats<D>();
+    };
+    // Q tile 1's buffer: a packed piece never loads a second query tile
+    float *ms = reinterpret_cast<float *>(smem_base() + C::kQOff + C::kTileBytes);
+    const PackedRows pr = packed_rows(p, seg.h);
+    if (r < n_valid) {
+        // batches of 8 partials: the loads of a batch are independent and in
+        // flight together, the combine is branch-free
+        constexpr int kBatch = 8;
+        float m = -CUDART_INF_F, l = 0.f;
+        for (int k0 = blockIdx.x; k0 <= c_last; k0 += kBatch) {
+            float mk[kBatch], lk[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const bool in = k0 + u <= c_last;
+                const float *sl = slot_of(in ? k0 + u : k0);
+                mk[u] = in ? __ldcg(sl + 128 * D + r) : -CUDART_INF_F;
+                lk[u] = in ? __ldcg(sl + 128 * D + 128 + r) : 0.f;
+            }
+            float mb = mk[0];
+#pragma unroll
+            for (int u = 1; u < kBatch; ++u) mb = fmaxf(mb, mk[u]);
+            const float mn = fmaxf(m, mb);
+            const float mnc = (mn == -CUDART_INF_F) ? 0.f : mn * c;  // an empty row keeps l = 0
+            float lb = (m == -CUDART_INF_F) ? 0.f : l * ex2(fmaf(m, c, -mnc));
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u)
+                lb = fmaf(lk[u], (mk[u] == -CUDART_INF_F) ? 0.f : ex2(fmaf(mk[u], c, -mnc)), lb);
+            m = mn;
+            l = lb;
+        }
+        const int head = pr.h0 + r / p.L, row = r % p.L;
+        l = add_sink(p, l, m, c, head);
+        if constexpr (MODE == kModeLse)
+            p.lse[static_cast<size_t>(seg.b * p.Hq + head) * p.L + row] =
+                l > 0.f ? fmaf(m, c, __log2f(l)) : CUDART_INF_F;
+        ms[r] = m;
+        ms[128 + r] = l > 0.f ? 1.f / l : 0.f;
+    }
+    named_barrier(1 + t, 128);
+    constexpr int kC4 = D / 4;  // float4 columns per row
+    const int n4 = n_valid * kC4;
+    for (int e0 = r; e0 < n4; e0 += 256) {  // two elements per thread per pass
+        const int e1 = e0 + 128;
+        const bool has1 = e1 < n4;
+        const int row0 = e0 / kC4, row1 = has1 ? e1 / kC4 : row0;
+        const int c40 = e0 - row0 * kC4, c41 = has1 ? e1 - row1 * kC4 : c40;
+        const float m0 = ms[row0], m1 = ms[row1];
+        float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+        // batches of partials, loads predicated (not a remainder loop) so that
+        // a batch's loads are all in flight together however few there are
+        constexpr int kBatch = 8;
+        for (int k0 = blockIdx.x; k0 <= c_last; k0 += kBatch) {
+            float mk0[kBatch], mk1[kBatch];
+            float4 v0[kBatch], v1[kBatch];
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const bool in = k0 + u <= c_last;
+                const float *sl = slot_of(in ? k0 + u : k0);
+                mk0[u] = in ? __ldcg(sl + 128 * D + row0) : -CUDART_INF_F;
+                mk1[u] = in ? __ldcg(sl + 128 * D + row1) : -CUDART_INF_F;
+                v0[u] = __ldcg(reinterpret_cast<const float4 *>(sl + row0 * D) + c40);
+                v1[u] = __ldcg(reinterpret_cast<const float4 *>(sl + row1 * D) + c41);
+            }
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const float f0 = (mk0[u] == -CUDART_INF_F) ? 0.f : ex2((mk0[u] - m0) * c);
+                const float f1 = (mk1[u] == -CUDART_INF_F) ? 0.f : ex2((mk1[u] - m1) * c);
+                a0.x = fmaf(f0, v0[u].x, a0.x), a0.y = fmaf(f0, v0[u].y, a0.y);
+                a0.z = fmaf(f0, v0[u].z, a0.z), a0.w = fmaf(f0, v0[u].w, a0.w);
+                a1.x = fmaf(f1, v1[u].x, a1.x), a1.y = fmaf(f1, v1[u].y, a1.y);
+                a1.z = fmaf(f1, v1[u].z, a1.z), a1.w = fmaf(f1, v1[u].w, a1.w);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (u == 1 && !has1) break;
+            const int rr = u ? row1 : row0, c4 = u ? c41 : c40;
+            const float4 a = u ? a1 : a0;
+            const float inv = ms[128 + rr];
+            const int head = pr.h0 + rr / p.L, row = rr % p.L;
+            __nv_bfloat16 *orow = p.o + (static_cast<size_t>(seg.b * p.Hq + head) * p.L + row) * D;
+            *reinterpret_cast<uint2 *>(orow + 4 * c4) = make_uint2(pack_bf16(a.x * inv, a.y * inv),
+                                                                  pack_bf16(a.z * inv, a.w * inv));
+        }
+    }
+    // the next piece may overwrite the scratch row maxima only after every
+    // thread has read them
+    named_barrier(1 + t, 128);
+    return true;
+}
+
+
+template <int D, bool KM, int MODE, int LY, bool PK>
 __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint32_t tmem,
                                           const Bars &bar, volatile int *abort_flag) {
     using C = Cfg<D>;
@@ -553,7 +677,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         int out_head = seg.h;
         bool row_valid = row < seg.L;
         const int q_tile0 = row - r;  // first row of the tile, for the tile-level mask test
-        if (p.packed) {
+        if constexpr (PK) {
             const PackedRows pr = packed_rows(p, seg.h);
             row = r % p.L;
             out_head = pr.h0 + r / p.L;
@@ -711,14 +835,17 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 
         // Rows of this tile that hold a query row: a packed tile fills
         // heads * L of its 128 rows, a prefill tile ends at row L.
-        const int n_valid = p.packed ? packed_rows(p, seg.h).heads * p.L : imin(kBlockQ, seg.L - q_tile0);
+        const int n_valid = PK ? packed_rows(p, seg.h).heads * p.L : imin(kBlockQ, seg.L - q_tile0);
         const bool warp_live = (r & ~31) < n_valid;  // warp-uniform: tcgen05.ld is warp-collective
         const bool row_live = r < n_valid;
 
-        if (!ip.complete && !ip.finalizer) {
-            // A later piece of a cut tile: publish the partial (unscaled
-            // accumulator, row max, row sum) of the live rows for the finalizer.
-            float *slot = p.partial + static_cast<size_t>(partial_slot(blockIdx.x, t)) * partial_slot_floats<D>();
+        // A later piece of a cut tile publishes its partial (unscaled
+        // accumulator, row max, row sum of the live rows) for the finalizer; a
+        // packed tile's finalizer publishes its own too and then merges them
+        // all with the whole warpgroup (few live rows, many contributors).
+        if (!ip.complete && (PK || !ip.finalizer)) {
+            float *slot = p.partial + static_cast<size_t>(partial_slot(blockIdx.x, (PK && ip.finalizer) ? 1 : t)) *
+                                          partial_slot_floats<D>();
             if (warp_live) {
 #pragma unroll
                 for (int cc = 0; cc < D / 32; ++cc) {
@@ -737,6 +864,10 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
                     __stcg(slot + 128 * D + r, m_ref);
                     __stcg(slot + 128 * D + 128 + r, l);
                 }
+            }
+            if (PK && ip.finalizer) {
+                if (!merge_packed<D, MODE>(p, seg, sp, t, n_valid, epoch, abort_flag)) return;
+                continue;
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.pub(t));
@@ -836,7 +967,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 }
 
 // ------------------------------------------------------------------ kernel
-template <int D, bool KM, int MODE, int LY>
+template <int D, bool KM, int MODE, int LY, bool PK>
 __global__ void __launch_bounds__(kThreads, 1)
     tfa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
@@ -917,12 +1048,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp < 8) {
         reg_alloc<kRegsSoftmax>();
-        softmax_role<D, KM, MODE, LY>(p, warp >> 2, tmem, bar, abort_flag);
+        softmax_role<D, KM, MODE, LY, PK>(p, warp >> 2, tmem, bar, abort_flag);
     } else {
         reg_dealloc<kRegsOther>();
         if (warp == 8 && (lane == 0 || KM))
-            load_role<D, KM, LY>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
-        if (warp == 9 && lane == 0) mma_role<D, KM, LY>(p, sbase, tmem, bar, abort_flag);
+            load_role<D, KM, LY, PK>(p, &tm_q, &tm_k, &tm_v, sbase, gbase, bar, abort_flag);
+        if (warp == 9 && lane == 0) mma_role<D, KM, LY, PK>(p, sbase, tmem, bar, abort_flag);
     }
 
     tc_fence_before();
