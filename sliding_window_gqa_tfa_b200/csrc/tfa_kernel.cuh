@@ -439,72 +439,139 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
     SegIter it;
     iter_init<D, LY>(it, p);
     Segment seg;
-    while (it.next(p.shape, seg)) {
-        const ItemPlan ip = plan_piece<PK>(p, seg);
+    if constexpr (PK) {
+        // Short-query tiles: one query tile (tile 0) whose score tiles
+        // alternate between the two S buffers, so S_{j+1} = Q K_{j+1}^T is
+        // computed while the softmax works on S_j.  P.V products then finish
+        // after the next score tile's: each but the piece's last commits to
+        // o_full(1) (tile 1 never exists here), which the softmax waits on
+        // before it may rescale O.
+        auto qk_to = [&](int buf, uint32_t slot) {
+            const uint64_t dk = dkv0 + slot * kTileStep;
+            const uint32_t d_tmem = tmem + C::kTmemS + buf * 128;
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-            if (!ip.present[t]) continue;
-            if (!mbar_wait(bar.q_full(t), q_use[t] & 1, abort_flag, p.status)) goto out;
-            ++q_use[t];
-        }
-        {
-            const uint32_t s = kv_cons % C::kSlots;
-            if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
-            ++kv_cons;
-            tc_fence_after();
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                if (ip.present[t] && ip.lo[t] <= ip.jl) {
-                    issue_qk(t, s);
-                    umma_commit(bar.s_full(t));
-                    if (ip.hi[t] == ip.jl) umma_commit(bar.q_empty(t));
-                }
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = ((kk >> 2) * C::kColBlockBytes + (kk & 3) * 32) >> 4;
+                umma_ss(d_tmem, dq0 + off, dk + off, kIdescQK, kk > 0 ? 1u : 0u);
             }
-            umma_commit(bar.kv_empty(s));
-        }
-        bool acc[2] = {false, false};
-        for (int j = ip.jl; j <= ip.jh; ++j) {
-            TFA_TR(2, trace_step, 0);
-            const uint32_t sv = kv_cons % C::kSlots;
-            if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
-            ++kv_cons;
-            const bool next = j < ip.jh;
-            uint32_t sk = 0;
-            if (next) {
-                sk = kv_cons % C::kSlots;
-                if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status))
-                    goto out;
+            if constexpr (has_km) umma_ss(d_tmem, d_ones, d_bias0 + slot * (C::kBiasBytes >> 4), kIdescQK, 1u);
+        };
+        auto pv_from = [&](int buf, uint32_t slot, bool accumulate, int kk_begin, int kk_end) {
+            const uint64_t dv = dv0 + slot * kTileStep;
+            const uint32_t a_tmem = tmem + C::kTmemS + buf * 128 + C::kTmemP;
+            for (int kk = kk_begin; kk < kk_end; ++kk)
+                umma_ts(tmem + C::kTmemO, a_tmem + kk * 8, dv + kk * ((16 * 128) >> 4), kIdescPV,
+                        (accumulate || kk > 0) ? 1u : 0u);
+        };
+        while (it.next(p.shape, seg)) {
+            const ItemPlan ip = plan_piece<PK>(p, seg);
+            if (ip.jl > ip.jh) continue;  // no key tile: nothing was loaded
+            if (!mbar_wait(bar.q_full(0), q_use[0] & 1, abort_flag, p.status)) goto out;
+            ++q_use[0];
+            {
+                const uint32_t s = kv_cons % C::kSlots;
+                if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
                 ++kv_cons;
+                tc_fence_after();
+                qk_to(0, s);
+                umma_commit(bar.s_full(0));
+                if (ip.jl == ip.jh) umma_commit(bar.q_empty(0));
+                umma_commit(bar.kv_empty(s));
             }
-            TFA_TR(2, trace_step, 1);
-            tc_fence_after();
+            for (int j = ip.jl; j <= ip.jh; ++j) {
+                const int buf = (j - ip.jl) & 1;
+                const uint32_t sv = kv_cons % C::kSlots;
+                if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                ++kv_cons;
+                if (j < ip.jh) {
+                    const uint32_t sk = kv_cons % C::kSlots;
+                    if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                    ++kv_cons;
+                    tc_fence_after();
+                    qk_to(buf ^ 1, sk);
+                    umma_commit(bar.s_full(buf ^ 1));
+                    if (j + 1 == ip.jh) umma_commit(bar.q_empty(0));
+                    umma_commit(bar.kv_empty(sk));
+                }
+                if (!mbar_wait(bar.p_part(0), p_cnt[0] & 1, abort_flag, p.status)) goto out;
+                tc_fence_after();
+                pv_from(buf, sv, j > ip.jl, 0, kPartKeys / 16);
+                if (!mbar_wait(bar.p_full(0), p_cnt[0] & 1, abort_flag, p.status)) goto out;
+                ++p_cnt[0];
+                tc_fence_after();
+                pv_from(buf, sv, true, kPartKeys / 16, kBlockK / 16);
+                umma_commit(j == ip.jh ? bar.o_full(0) : bar.o_full(1));
+                umma_commit(bar.kv_empty(sv));
+            }
+        }
+    } else {
+        while (it.next(p.shape, seg)) {
+            const ItemPlan ip = plan_piece<PK>(p, seg);
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (!ip.present[t]) continue;
-                if (ip.lo[t] <= j && j <= ip.hi[t]) {
-                    // first part of P_t, then the rest (the tensor core works on
-                    // the first part meanwhile)
-                    if (!mbar_wait(bar.p_part(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
-                    TFA_TR(2, trace_step, 2 + 2 * t);
-                    tc_fence_after();
-                    issue_pv(t, sv, acc[t], 0, kPartKeys / 16);
-                    if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
-                    ++p_cnt[t];
-                    tc_fence_after();
-                    issue_pv(t, sv, true, kPartKeys / 16, kBlockK / 16);
-                    acc[t] = true;
-                    if (j == ip.hi[t]) umma_commit(bar.o_full(t));
-                }
-                if (next && ip.lo[t] <= j + 1 && j + 1 <= ip.hi[t]) {
-                    issue_qk(t, sk);
-                    umma_commit(bar.s_full(t));
-                    if (j + 1 == ip.hi[t]) umma_commit(bar.q_empty(t));
-                }
-                TFA_TR(2, trace_step, 3 + 2 * t);
+                if (!mbar_wait(bar.q_full(t), q_use[t] & 1, abort_flag, p.status)) goto out;
+                ++q_use[t];
             }
-            ++trace_step;
-            umma_commit(bar.kv_empty(sv));
-            if (next) umma_commit(bar.kv_empty(sk));
+            {
+                const uint32_t s = kv_cons % C::kSlots;
+                if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                ++kv_cons;
+                tc_fence_after();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (ip.present[t] && ip.lo[t] <= ip.jl) {
+                        issue_qk(t, s);
+                        umma_commit(bar.s_full(t));
+                        if (ip.hi[t] == ip.jl) umma_commit(bar.q_empty(t));
+                    }
+                }
+                umma_commit(bar.kv_empty(s));
+            }
+            bool acc[2] = {false, false};
+            for (int j = ip.jl; j <= ip.jh; ++j) {
+                TFA_TR(2, trace_step, 0);
+                const uint32_t sv = kv_cons % C::kSlots;
+                if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                ++kv_cons;
+                const bool next = j < ip.jh;
+                uint32_t sk = 0;
+                if (next) {
+                    sk = kv_cons % C::kSlots;
+                    if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status))
+                        goto out;
+                    ++kv_cons;
+                }
+                TFA_TR(2, trace_step, 1);
+                tc_fence_after();
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    if (!ip.present[t]) continue;
+                    if (ip.lo[t] <= j && j <= ip.hi[t]) {
+                        // first part of P_t, then the rest (the tensor core works on
+                        // the first part meanwhile)
+                        if (!mbar_wait(bar.p_part(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                        TFA_TR(2, trace_step, 2 + 2 * t);
+                        tc_fence_after();
+                        issue_pv(t, sv, acc[t], 0, kPartKeys / 16);
+                        if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                        ++p_cnt[t];
+                        tc_fence_after();
+                        issue_pv(t, sv, true, kPartKeys / 16, kBlockK / 16);
+                        acc[t] = true;
+                        if (j == ip.hi[t]) umma_commit(bar.o_full(t));
+                    }
+                    if (next && ip.lo[t] <= j + 1 && j + 1 <= ip.hi[t]) {
+                        issue_qk(t, sk);
+                        umma_commit(bar.s_full(t));
+                        if (j + 1 == ip.hi[t]) umma_commit(bar.q_empty(t));
+                    }
+                    TFA_TR(2, trace_step, 3 + 2 * t);
+                }
+                ++trace_step;
+                umma_commit(bar.kv_empty(sv));
+                if (next) umma_commit(bar.kv_empty(sk));
+            }
         }
     }
 out:
@@ -661,6 +728,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     const float c = p.scale_log2;
     const int lane = threadIdx.x & 31;
     uint32_t s_cnt = 0, o_cnt = 0, pub_cnt = 0, fin_cnt = 0;
+    uint32_t s_cnt0 = 0, s_cnt1 = 0, pv_cnt = 0;  // short-query tiles: per S buffer, P.V done
     const unsigned epoch = p.ctl ? launch_epoch(p.ctl) : 0u;
     int trace_step = 0;
     (void)trace_step;
@@ -692,14 +760,24 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 
         for (int j = ip.lo; j <= ip.hi; ++j) {
             if (r == 0) TFA_TR(t, trace_step, 0);
+            // short-query tiles alternate between the two S buffers
+            uint32_t tSj = tS, tPj = tP, sph;
+            int sb = t;
+            if constexpr (PK) {
+                sb = (j - ip.lo) & 1;
+                tSj = tS + sb * 128;
+                tPj = tP + sb * 128;
+                sph = (sb ? s_cnt1++ : s_cnt0++) & 1;
+            } else {
+                sph = s_cnt++ & 1;
+            }
             // all lanes leave together: the tcgen05 loads below are warp-collective
-            if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(t), s_cnt & 1, abort_flag, p.status)))
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(sb), sph, abort_flag, p.status)))
                 return;
-            ++s_cnt;
             if (r == 0) TFA_TR(t, trace_step, 1);
             tc_fence_after();
             uint32_t s[128];
-            tmem_ld128(tS, s);
+            tmem_ld128(tSj, s);
             if (r == 0) TFA_TR(t, trace_step, 2);
             if constexpr (SC) {
                 // Gemma-2 logit softcap (brotensor flash_attention.h): the scaled
@@ -767,6 +845,15 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
 
             // O_t must be rescaled before any of P_t is published: the P.V
             // product may start as soon as the first part is.
+            if constexpr (PK) {
+                // the previous tile's P.V product may still be accumulating
+                if (j > ip.lo) {
+                    if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(1), pv_cnt & 1, abort_flag, p.status)))
+                        return;
+                    ++pv_cnt;
+                    tc_fence_after();
+                }
+            }
             if (rescale) {  // rare; 8 columns at a time while the scores are live
                 for (int cc = 0; cc < D / 8; ++cc) {
                     uint32_t o[8];
@@ -802,8 +889,8 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             for (int i = 0; i < kPartKeys / 2; ++i) TFA_EXP_PAIR(i);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 3);
 #pragma unroll
-            for (int c32 = 0; c32 < kPartKeys / 64; ++c32) tmem_st32(tP + 32 * c32, pk + 32 * c32);
-            if ((kPartKeys / 2) % 32) tmem_st16(tP + (kPartKeys / 64) * 32, pk + (kPartKeys / 64) * 32);
+            for (int c32 = 0; c32 < kPartKeys / 64; ++c32) tmem_st32(tPj + 32 * c32, pk + 32 * c32);
+            if ((kPartKeys / 2) % 32) tmem_st16(tPj + (kPartKeys / 64) * 32, pk + (kPartKeys / 64) * 32);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -817,7 +904,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             const float2 acc = add2(acc0, acc1);
             l = l * alpha + (acc.x + acc.y);
 #pragma unroll
-            for (int c16 = kPartKeys / 32; c16 < 4; ++c16) tmem_st16(tP + 16 * c16, pk + 16 * c16);
+            for (int c16 = kPartKeys / 32; c16 < 4; ++c16) tmem_st16(tPj + 16 * c16, pk + 16 * c16);
             if (r == 0) TFA_TR(t, trace_step, 3);
             if (t == 0 && lane == 0) TFA_TR(4 + (r >> 5), trace_step, 2);
             tmem_wait_st();
