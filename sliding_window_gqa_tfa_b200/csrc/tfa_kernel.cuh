@@ -479,6 +479,7 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                 umma_commit(bar.kv_empty(s));
             }
             for (int j = ip.jl; j <= ip.jh; ++j) {
+                TFA_TR(2, trace_step, 0);
                 const int buf = (j - ip.jl) & 1;
                 const uint32_t sv = kv_cons % C::kSlots;
                 if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
@@ -488,18 +489,22 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                     if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
                     ++kv_cons;
                     tc_fence_after();
+                    TFA_TR(2, trace_step, 1);
                     qk_to(buf ^ 1, sk);
                     umma_commit(bar.s_full(buf ^ 1));
                     if (j + 1 == ip.jh) umma_commit(bar.q_empty(0));
                     umma_commit(bar.kv_empty(sk));
                 }
                 if (!mbar_wait(bar.p_part(0), p_cnt[0] & 1, abort_flag, p.status)) goto out;
+                TFA_TR(2, trace_step, 2);
                 tc_fence_after();
                 pv_from(buf, sv, j > ip.jl, 0, kPartKeys / 16);
                 if (!mbar_wait(bar.p_full(0), p_cnt[0] & 1, abort_flag, p.status)) goto out;
+                TFA_TR(2, trace_step, 3);
                 ++p_cnt[0];
                 tc_fence_after();
                 pv_from(buf, sv, true, kPartKeys / 16, kBlockK / 16);
+                ++trace_step;
                 umma_commit(j == ip.jh ? bar.o_full(0) : bar.o_full(1));
                 umma_commit(bar.kv_empty(sv));
             }
@@ -628,9 +633,9 @@ __device__ __forceinline__ bool merge_packed(const Params &p, const Segment &seg
     float *ms = reinterpret_cast<float *>(smem_base() + C::kQOff + C::kTileBytes);
     const PackedRows pr = packed_rows(p, seg.h);
     if (r < n_valid) {
-        // batches of 8 partials: the loads of a batch are independent and in
+        // batches of 16 partials: the loads of a batch are independent and in
         // flight together, the combine is branch-free
-        constexpr int kBatch = 8;
+        constexpr int kBatch = 16;
         float m = -CUDART_INF_F, l = 0.f;
         for (int k0 = blockIdx.x; k0 <= c_last; k0 += kBatch) {
             float mk[kBatch], lk[kBatch];
