@@ -101,7 +101,11 @@ typedef enum {
  *   window   > 0 (causal only): additionally j > S-L+i-window; <= 0: no window
  *   key_mask fp32 [B,S] device (4-byte aligned) or NULL; key j of batch b kept iff > 0.5
  *   stream   CUDA stream to enqueue on
- * Returns TFA_OK or a tfa_status code. */
+ * Returns TFA_OK or a tfa_status code.
+ * Queries of at most 128 rows run through the packed tiles described under
+ * tfa_decode (floor(128 / L) query heads of a KV group per tile); longer ones
+ * through pairs of 128-row tiles of one head.  The results are the same
+ * attention either way. */
 int tfa_prefill(const void *q, const void *k, const void *v, void *o,
                 int B, int Hq, int Hkv, int L, int S, int D, float scale,
                 int causal, int window, const float *key_mask, tfa_stream_t stream);
@@ -125,8 +129,8 @@ int tfa_decode(const void *q, const void *k, const void *v, void *o,
                int causal, int window, const float *key_mask, tfa_stream_t stream);
 
 /* tfa_attention_ex -- the same attention with the score variants, for any
- * L >= 1 (L <= TFA_MAX_DECODE_ROWS takes tfa_decode's packed path, longer
- * queries tfa_prefill's).  Arguments, layouts, ownership, asynchrony and
+ * L >= 1 (L <= 128 takes the packed tiles, longer queries pairs of
+ * 128-row tiles).  Arguments, layouts, ownership, asynchrony and
  * errors are those of tfa_prefill/tfa_decode, plus:
  *   softcap  logit soft-capping (brotensor flash_attention.h, Gemma-2
  *            extensions): after the scale and before the masks and the

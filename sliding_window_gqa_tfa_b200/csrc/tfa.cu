@@ -315,10 +315,15 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     using C = tfa::Cfg<D>;
     // Short queries: a tile packs pack_heads query heads of one KV group, all L
     // rows of each (pack_heads * L <= 128), loaded as one {64, L, pack_heads} box.
+    // Any call with L <= 128 has one query tile per item, so it runs packed:
+    // the tile fills with more heads where L <= 64, and the packed schedule
+    // double-buffers the score tile, which a single-tile item cannot use
+    // otherwise.  (Variable-length batches keep per-sequence tiles.)
+    const bool varlen = ad.cu_q != nullptr;
+    if (!varlen && L <= tfa::kBlockQ) packed = true;
     const int G = Hq / Hkv;
     const int pack_heads = packed ? (G < tfa::kBlockQ / L ? G : tfa::kBlockQ / L) : 0;
     const int pack_chunks = packed ? (G + pack_heads - 1) / pack_heads : 0;
-    const bool varlen = ad.cu_q != nullptr;
     CUtensorMap mq, mk, mv;
     int rc = 0;
     if (varlen)  // packed [total, H, D]: rows are tokens, planes are heads

@@ -72,6 +72,15 @@ SMALL = [
     ("d64_ragged", shaped(2, 4, 2, 130, 300, 64)),
     ("d64_window", shaped(1, 4, 2, 300, 700, 64, window=129)),
     ("d64_keymask_bidir", shaped(1, 4, 2, 100, 250, 64, causal=False, key_mask_keep=0.8)),
+    # chunks of at most 128 rows run packed: a 128-row tile holds the rows of
+    # floor(128 / L) query heads of one KV group (the last tile of a group may
+    # hold fewer), and long key ranges are cut over several CTAs whose partials
+    # the first piece merges with its whole warpgroup
+    ("pack3_of4_L40_long", shaped(1, 8, 2, 40, 3000, 128)),
+    ("pack2_L64_window", shaped(2, 8, 2, 64, 2000, 128, window=300)),
+    ("pack5_of6_L24_keymask_d64", shaped(1, 12, 2, 24, 900, 64, key_mask_keep=0.7)),
+    ("pack8_L16_bidir", shaped(1, 16, 2, 16, 700, 128, causal=False)),
+    ("pack1_L128_full_tile", shaped(1, 4, 2, 128, 600, 128)),
 ]
 
 
