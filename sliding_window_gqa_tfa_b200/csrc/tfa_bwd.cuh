@@ -36,7 +36,11 @@
 namespace tfa {
 namespace bwd {
 
-constexpr int kThreads = 192;
+// Warps 0-7: elementwise (warp w holds tensor-memory lanes 32 (w % 4) ..,
+// i.e. 32 rows, and half w / 4 of each tile's 128 columns: two warps per SM
+// sub-partition); warp 8: TMA producer; warp 9: MMA issuer.
+constexpr int kEwWarps = 8;
+constexpr int kThreads = 32 * (kEwWarps + 2);
 
 template <int D>
 struct Cfg {
@@ -52,7 +56,7 @@ struct Cfg {
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // dKV kernel: per elementwise warp, the step's 128 values of -lse and delta
     static constexpr int kStageOff = kMiscOff + 16;
-    static constexpr int kSmemBytes = kStageOff + 4 * 256 * 4 + 1024;  // + slack to align the base
+    static constexpr int kSmemBytes = kStageOff + kEwWarps * 256 * 4 + 1024;  // + slack to align the base
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kTmemA = 0;    // S (dQ kernel) / S^T (dKV kernel), 128 columns
     static constexpr uint32_t kTmemB = 128;  // dP / dP^T, 128 columns
@@ -175,9 +179,9 @@ __device__ __forceinline__ Setup<D> setup(const CUtensorMap *m0, const CUtensorM
             mbar_init(st.bar.ring_empty(s), 1);
         }
         mbar_init(st.bar.mm_full(), 1);
-        mbar_init(st.bar.op_full(), 4);
+        mbar_init(st.bar.op_full(), kEwWarps);
         mbar_init(st.bar.acc_full(), 1);
-        mbar_init(st.bar.acc_empty(), 4);
+        mbar_init(st.bar.acc_empty(), kEwWarps);
         mbar_init(st.bar.done(), 1);
         *st.abort_flag = 0;
         fence_barrier_init();
@@ -186,7 +190,7 @@ __device__ __forceinline__ Setup<D> setup(const CUtensorMap *m0, const CUtensorM
         tmem_alloc(smem_addr(tmem_slot), C::kTmemCols);
         tmem_relinquish();
     }
-    if (warp == 4 && (threadIdx.x & 31) == 0) {
+    if (warp == kEwWarps && (threadIdx.x & 31) == 0) {
         prefetch_tensormap(m0);
         prefetch_tensormap(m1);
         prefetch_tensormap(m2);
@@ -231,6 +235,11 @@ __device__ __forceinline__ void load_tile(uint32_t dst, const CUtensorMap *map, 
         tma_load_3d(dst + cb * C::kColBlockBytes, map, bar, cb * 64, row, plane);
 }
 
+// Tensor-memory column of K-step kk (16 keys or queries, 8 packed bf16x2
+// columns) of an operand the elementwise warps wrote: half h of the 128
+// columns writes its 32 packed columns at 64 h, over columns it has read.
+__device__ __forceinline__ uint32_t packed_col(int kk) { return kk * 8 + (kk >= 4 ? 32 : 0); }
+
 // K-step offset (>> 4) inside a K-major 128-byte-swizzled [128][D] tile.
 template <int D>
 __device__ __forceinline__ uint32_t kstep_off(int kk) {
@@ -249,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTileStep = C::kTileBytes >> 4;
 
-    if (warp == 4) {
+    if (warp == kEwWarps) {
         // ---- producer: Q and dO once per item, then K_j, V_j per key tile
         if (lane == 0) {
             uint32_t prod = 0, fix_use = 0;
@@ -280,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             drain_copies<D>(bar, prod, fix_use);
         }
-    } else if (warp == 5) {
+    } else if (warp == kEwWarps + 1) {
         // ---- MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, kBlockK, 0);  // both operands K-major
@@ -313,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_commit(bar.mm_full());
                     umma_commit(bar.ring_empty(sv));
                     if (j == it.hi) umma_commit(bar.fix_empty());
-                    // dQ += dS K, dS (bf16) in the first 64 columns of the dP region
+                    // dQ += dS K, dS (bf16) over dP columns 0-31 and 64-95
                     if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
                     ++op_cnt;
                     // the previous item's dQ must have been read before it is overwritten
@@ -323,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; ++kk)
-                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemB + kk * 8,
+                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemB + packed_col(kk),
                                 d_ring_mn + sk * kTileStep + kk * ((16 * 128) >> 4), kIdescDQ,
                                 (j > it.lo || kk > 0) ? 1u : 0u);
                     umma_commit(bar.ring_empty(sk));
@@ -336,9 +345,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_drain(bar.done(), 0);
         }
     } else {
-        // ---- elementwise (warps 0-3): P, dS per key tile; dQ epilogue per item
-        const int r = threadIdx.x;  // query row inside the tile = tensor-memory lane
-        const uint32_t lane_base = (static_cast<uint32_t>(warp) * 32u) << 16;
+        // ---- elementwise (warps 0-7): P, dS per key tile; dQ epilogue per item
+        const int r = (warp & 3) * 32 + lane;  // query row inside the tile = tensor-memory lane
+        const int hf = warp >> 2;               // key columns 64 hf .. 64 hf + 63
+        const uint32_t lane_base = (static_cast<uint32_t>(warp & 3) * 32u) << 16;
         const uint32_t tA = st.tmem + C::kTmemA + lane_base;
         const uint32_t tB = st.tmem + C::kTmemB + lane_base;
         const uint32_t tC = st.tmem + C::kTmemC + lane_base;
@@ -363,7 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const bool needs = key_tile_needs_mask(p.L, p.S, p.causal, p.window, KM ? 1 : 0, q0, j, 0u);
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int ch = 2 * hf + c2;
                     uint32_t sv[32], dv[32], w[16];
                     tmem_ld32(tA + 32 * ch, sv);
                     tmem_ld32(tB + 32 * ch, dv);
@@ -381,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         w[e] = pack_bf16(p0 * (__uint_as_float(dv[2 * e]) - dl_r),
                                          p1 * (__uint_as_float(dv[2 * e + 1]) - dl_r));
                     }
-                    tmem_st16(tB + 16 * ch, w);  // over dP columns already read
+                    tmem_st16(tB + 64 * hf + 16 * c2, w);  // over dP columns this warp has read
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -395,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             {
                 __nv_bfloat16 *orow = valid ? p.dq + idx * D : nullptr;
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
+                for (int cc = hf * (D / 64); cc < (hf + 1) * (D / 64); ++cc) {
                     uint32_t o[32];
                     tmem_ld32(tC + 32 * cc, o);
                     uint32_t w[16];
@@ -431,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTileStep = C::kTileBytes >> 4;
 
-    if (warp == 4) {
+    if (warp == kEwWarps) {
         // ---- producer: K and V once per item, then Q_i, dO_i per (head, query tile)
         if (lane == 0) {
             uint32_t prod = 0, fix_use = 0;
@@ -464,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             drain_copies<D>(bar, prod, fix_use);
         }
-    } else if (warp == 5) {
+    } else if (warp == kEwWarps + 1) {
         // ---- MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, kBlockQ, 0);  // both operands K-major
@@ -504,14 +515,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
                         goto mma_out;
                     tc_fence_after();
-                    // dV += P^T dO (P^T in the first 64 columns of the S^T region),
-                    // dK += dS^T Q (dS^T in the first 64 columns of the dP^T region)
+                    // dV += P^T dO (P^T over S^T columns 0-31 and 64-95),
+                    // dK += dS^T Q (dS^T over dP^T columns 0-31 and 64-95)
 #pragma unroll
                     for (int kk = 0; kk < kBlockQ / 16; ++kk) {
-                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemA + kk * 8,
+                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemA + packed_col(kk),
                                 d_ring_mn + sd * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
-                        umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + kk * 8,
+                        umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + packed_col(kk),
                                 d_ring_mn + sq * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
                     }
@@ -526,9 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_drain(bar.done(), 0);
         }
     } else {
-        // ---- elementwise (warps 0-3): P^T, dS^T per step; dK, dV epilogue per item
-        const int r = threadIdx.x;  // key row inside the tile = tensor-memory lane
-        const uint32_t lane_base = (static_cast<uint32_t>(warp) * 32u) << 16;
+        // ---- elementwise (warps 0-7): P^T, dS^T per step; dK, dV epilogue per item
+        const int r = (warp & 3) * 32 + lane;  // key row inside the tile = tensor-memory lane
+        const int hf = warp >> 2;               // query columns 64 hf .. 64 hf + 63
+        const uint32_t lane_base = (static_cast<uint32_t>(warp & 3) * 32u) << 16;
         const uint32_t tA = st.tmem + C::kTmemA + lane_base;
         const uint32_t tB = st.tmem + C::kTmemB + lane_base;
         const uint32_t tC = st.tmem + C::kTmemC + lane_base;
@@ -551,7 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (kvalid) {
                     uint4 *dk4 = reinterpret_cast<uint4 *>(p.dk + oidx);
                     uint4 *dv4 = reinterpret_cast<uint4 *>(p.dv + oidx);
-                    for (int v4 = 0; v4 < D / 8; ++v4) {
+                    for (int v4 = hf * (D / 16); v4 < (hf + 1) * (D / 16); ++v4) {
                         dk4[v4] = make_uint4(0u, 0u, 0u, 0u);
                         dv4[v4] = make_uint4(0u, 0u, 0u, 0u);
                     }
@@ -563,12 +575,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int q0 = (it.qlo + step % it.nq) * kBlockQ;
                 const float *lse_h = p.lse + static_cast<size_t>(it.b * p.Hq + h) * p.L;
                 const float *dl_h = p.delta + static_cast<size_t>(it.b * p.Hq + h) * p.L;
-                // -lse and delta of the tile's 128 query columns, loaded once per
-                // warp (lane e: columns e, 32 + e, ...) into the warp's stage and
+                // -lse and delta of the warp's 64 query columns, loaded once per
+                // warp (lane e: columns 32 ch + e) into the warp's stage and
                 // read back as shared-memory broadcasts
                 __syncwarp();  // every lane is done with the previous step's stage
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int ch = 2 * hf + c2;
                     const int q = q0 + 32 * ch + lane;
                     stage[32 * ch + lane] = q < p.L ? -__ldg(lse_h + q) : -CUDART_INF_F;
                     stage[128 + 32 * ch + lane] = q < p.L ? __ldg(dl_h + q) : 0.f;
@@ -579,7 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++mm_cnt;
                 tc_fence_after();
 #pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int ch = 2 * hf + c2;
                     uint32_t sv[32], dv[32], wp[16], wd[16];
                     tmem_ld32(tA + 32 * ch, sv);
                     tmem_ld32(tB + 32 * ch, dv);
@@ -601,8 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                             dv[e] = __float_as_uint(ds);
                         }
                     }
-                    tmem_st16(tA + 16 * ch, wp);  // over S^T columns already read
-                    tmem_st16(tB + 16 * ch, wd);  // over dP^T columns already read
+                    tmem_st16(tA + 64 * hf + 16 * c2, wp);  // over S^T columns this warp has read
+                    tmem_st16(tB + 64 * hf + 16 * c2, wd);  // over dP^T columns this warp has read
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -618,7 +632,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __nv_bfloat16 *orow = kvalid ? (which ? p.dk : p.dv) + oidx : nullptr;
                 const float f = which ? p.scale : 1.f;
 #pragma unroll
-                for (int cc = 0; cc < D / 32; ++cc) {
+                for (int cc = hf * (D / 64); cc < (hf + 1) * (D / 64); ++cc) {
                     uint32_t o[32];
                     tmem_ld32((which ? tD : tC) + 32 * cc, o);
                     uint32_t w[16];
