@@ -52,7 +52,7 @@ struct Cfg {
     static constexpr int kFixOff = 0;                  // two tiles fixed per item
     static constexpr int kRingOff = 2 * kTileBytes;
     static constexpr int kBarOff = kRingOff + kSlots * kTileBytes;
-    static constexpr int kNumBars = 2 * kSlots + 8;
+    static constexpr int kNumBars = 2 * kSlots + 11;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     // dKV kernel: per elementwise warp, the step's 128 values of -lse and delta
     static constexpr int kStageOff = kMiscOff + 16;
@@ -62,6 +62,7 @@ struct Cfg {
     static constexpr uint32_t kTmemB = 128;  // dP / dP^T, 128 columns
     static constexpr uint32_t kTmemC = 256;  // dQ accumulator / dV accumulator, D columns
     static constexpr uint32_t kTmemD = 256 + D;  // dK accumulator (dKV kernel), D columns
+    static constexpr uint32_t kTmemA2 = 256 + D;  // dQ kernel: second S buffer (odd key tiles), 128 columns
 };
 
 struct BwdParams {
@@ -88,6 +89,14 @@ struct Bars {
     __device__ __forceinline__ uint32_t acc_full() const { return base + 8 * (4 + 2 * slots); }
     __device__ __forceinline__ uint32_t acc_empty() const { return base + 8 * (5 + 2 * slots); }
     __device__ __forceinline__ uint32_t done() const { return base + 8 * (6 + 2 * slots); }
+    // dKV kernel, two phases per step: dP^T ready (mm_full: S^T ready), and
+    // P^T written (op_full: dS^T written)
+    __device__ __forceinline__ uint32_t dp_full() const { return base + 8 * (7 + 2 * slots); }
+    __device__ __forceinline__ uint32_t pt_full() const { return base + 8 * (8 + 2 * slots); }
+    // dQ kernel: S of odd key tiles (its second buffer; mm_full: even ones).
+    // One barrier per buffer: S_{x+2} is issued only after S_x was consumed,
+    // so neither runs two phases ahead of its waiter.
+    __device__ __forceinline__ uint32_t s2_full() const { return base + 8 * (9 + 2 * slots); }
 };
 
 // delta_i = sum_d dO[i,d] O[i,d] (fp32), one warp per row.
@@ -183,6 +192,9 @@ __device__ __forceinline__ Setup<D> setup(const CUtensorMap *m0, const CUtensorM
         mbar_init(st.bar.acc_full(), 1);
         mbar_init(st.bar.acc_empty(), kEwWarps);
         mbar_init(st.bar.done(), 1);
+        mbar_init(st.bar.dp_full(), 1);
+        mbar_init(st.bar.pt_full(), kEwWarps);
+        mbar_init(st.bar.s2_full(), 1);
         *st.abort_flag = 0;
         fence_barrier_init();
     }
@@ -303,39 +315,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const QItem it = q_item(p, item);
                 if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
                 ++fix_use;
-                for (int j = it.lo; j <= it.hi; ++j) {
-                    const uint32_t sk = cons % C::kSlots;
-                    if (!mbar_wait(bar.ring_full(sk), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                // S_j alternates between two buffers and runs two key tiles
+                // ahead of dQ; dP_{j+1} follows dQ += dS_j K_j (dS_j lies over dP_j's
+                // columns).  The elementwise warps compute P_{j+1} from S_{j+1} while
+                // the tensor core finishes step j.
+                const int n = it.hi - it.lo + 1;
+                auto take = [&](uint32_t &slot) -> bool {
+                    slot = cons % C::kSlots;
+                    if (!mbar_wait(bar.ring_full(slot), (cons / C::kSlots) & 1, st.abort_flag, p.status)) return false;
                     ++cons;
-                    const uint32_t sv = cons % C::kSlots;
-                    if (!mbar_wait(bar.ring_full(sv), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
-                    ++cons;
+                    return true;
+                };
+                auto issue_s = [&](int x, uint32_t ks) {
+                    const uint32_t dst = st.tmem + ((x & 1) ? C::kTmemA2 : C::kTmemA);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(dst, d_q + kstep_off<D>(kk), d_ring + ks * kTileStep + kstep_off<D>(kk), kIdescS,
+                                kk > 0 ? 1u : 0u);
+                    umma_commit((x & 1) ? bar.s2_full() : bar.mm_full());
+                };
+                auto issue_dp = [&](uint32_t vs) {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemB, d_do + kstep_off<D>(kk), d_ring + vs * kTileStep + kstep_off<D>(kk),
+                                kIdescS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar.dp_full());
+                    umma_commit(bar.ring_empty(vs));  // V's only use
+                };
+                uint32_t k_cur = 0, k_nxt = 0, v_nxt = 0, v0 = 0;
+                if (!take(k_cur) || !take(v0)) goto mma_out;
+                tc_fence_after();
+                issue_s(0, k_cur);
+                issue_dp(v0);
+                if (n > 1) {
+                    if (!take(k_nxt) || !take(v_nxt)) goto mma_out;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss(st.tmem + C::kTmemA, d_q + kstep_off<D>(kk), d_ring + sk * kTileStep + kstep_off<D>(kk),
-                                kIdescS, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss(st.tmem + C::kTmemB, d_do + kstep_off<D>(kk), d_ring + sv * kTileStep + kstep_off<D>(kk),
-                                kIdescS, kk > 0 ? 1u : 0u);
-                    umma_commit(bar.mm_full());
-                    umma_commit(bar.ring_empty(sv));
-                    if (j == it.hi) umma_commit(bar.fix_empty());
+                    issue_s(1, k_nxt);
+                }
+                if (n == 1) umma_commit(bar.fix_empty());  // Q, dO's last use
+                for (int x = 0; x < n; ++x) {
                     // dQ += dS K, dS (bf16) over dP columns 0-31 and 64-95
                     if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
                     ++op_cnt;
                     // the previous item's dQ must have been read before it is overwritten
-                    if (j == it.lo && acc_use > 0 &&
+                    if (x == 0 && acc_use > 0 &&
                         !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
                         goto mma_out;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBlockK / 16; ++kk)
                         umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemB + packed_col(kk),
-                                d_ring_mn + sk * kTileStep + kk * ((16 * 128) >> 4), kIdescDQ,
-                                (j > it.lo || kk > 0) ? 1u : 0u);
-                    umma_commit(bar.ring_empty(sk));
+                                d_ring_mn + k_cur * kTileStep + kk * ((16 * 128) >> 4), kIdescDQ,
+                                (x > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(bar.ring_empty(k_cur));  // K_j's last use
+                    if (x + 1 < n) {
+                        issue_dp(v_nxt);
+                        if (x + 2 == n) umma_commit(bar.fix_empty());  // Q, dO's last use
+                    }
+                    uint32_t k_nn = 0, v_nn = 0;
+                    if (x + 2 < n) {
+                        if (!take(k_nn) || !take(v_nn)) goto mma_out;
+                        tc_fence_after();
+                        issue_s(x + 2, k_nn);
+                    }
+                    k_cur = k_nxt;
+                    k_nxt = k_nn;
+                    v_nxt = v_nn;
                 }
                 umma_commit(bar.acc_full());
                 ++acc_use;
@@ -350,10 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hf = warp >> 2;               // key columns 64 hf .. 64 hf + 63
         const uint32_t lane_base = (static_cast<uint32_t>(warp & 3) * 32u) << 16;
         const uint32_t tA = st.tmem + C::kTmemA + lane_base;
+        const uint32_t tA2 = st.tmem + C::kTmemA2 + lane_base;
         const uint32_t tB = st.tmem + C::kTmemB + lane_base;
         const uint32_t tC = st.tmem + C::kTmemC + lane_base;
         const float c = p.scale_log2;
-        uint32_t mm_cnt = 0, acc_cnt = 0;
+        uint32_t mm_cnt = 0, acc_cnt = 0;  // mm_cnt: dP tiles seen
+        uint32_t s_even = 0, s_odd = 0;    // S tiles seen per buffer
         for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
             const QItem it = q_item(p, item);
             const int q0 = it.qt * kBlockQ;
@@ -367,31 +414,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int lo_abs = (p.causal && p.window > 0) ? pos - p.window + 1 : 0;
             const float *km_row = KM ? p.key_mask + static_cast<size_t>(it.b) * p.S : nullptr;
             for (int j = it.lo; j <= it.hi; ++j) {
-                if (!__all_sync(0xffffffffu, mbar_wait(bar.mm_full(), mm_cnt & 1, st.abort_flag, p.status)))
+                // phase 1: P = 2^(S c - lse) from S (its buffer alternates per key tile)
+                const bool odd = ((j - it.lo) & 1) != 0;
+                const uint32_t sph = (odd ? s_odd++ : s_even++) & 1;
+                if (!__all_sync(0xffffffffu, mbar_wait(odd ? bar.s2_full() : bar.mm_full(), sph, st.abort_flag, p.status)))
                     goto ew_out;
-                ++mm_cnt;
                 tc_fence_after();
+                const uint32_t tS = odd ? tA2 : tA;
                 const bool needs = key_tile_needs_mask(p.L, p.S, p.causal, p.window, KM ? 1 : 0, q0, j, 0u);
+                float pr[64];
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
                     const int ch = 2 * hf + c2;
-                    uint32_t sv[32], dv[32], w[16];
-                    tmem_ld32(tA + 32 * ch, sv);
+                    uint32_t sv[32];
+                    tmem_ld32(tS + 32 * ch, sv);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        float pe = ex2(fmaf(__uint_as_float(sv[e]), c, -lse_r));
+                        if (needs) {
+                            const int k = j * kBlockK + 32 * ch + e;
+                            const bool al = k >= lo_abs && k <= hi_abs && (!KM || __ldg(km_row + k) > 0.5f);
+                            pe = al ? pe : 0.f;
+                        }
+                        pr[32 * c2 + e] = pe;
+                    }
+                }
+                // phase 2: dS = P (dP - delta) from dP, over dP's columns
+                if (!__all_sync(0xffffffffu, mbar_wait(bar.dp_full(), mm_cnt & 1, st.abort_flag, p.status)))
+                    goto ew_out;
+                ++mm_cnt;
+                tc_fence_after();
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int ch = 2 * hf + c2;
+                    uint32_t dv[32], w[16];
                     tmem_ld32(tB + 32 * ch, dv);
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        float p0 = ex2(fmaf(__uint_as_float(sv[2 * e]), c, -lse_r));
-                        float p1 = ex2(fmaf(__uint_as_float(sv[2 * e + 1]), c, -lse_r));
-                        if (needs) {
-                            const int k = j * kBlockK + 32 * ch + 2 * e;
-                            const bool a0 = k >= lo_abs && k <= hi_abs && (!KM || __ldg(km_row + k) > 0.5f);
-                            const bool a1 = k + 1 >= lo_abs && k + 1 <= hi_abs && (!KM || __ldg(km_row + k + 1) > 0.5f);
-                            p0 = a0 ? p0 : 0.f;
-                            p1 = a1 ? p1 : 0.f;
-                        }
-                        w[e] = pack_bf16(p0 * (__uint_as_float(dv[2 * e]) - dl_r),
-                                         p1 * (__uint_as_float(dv[2 * e + 1]) - dl_r));
-                    }
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16(pr[32 * c2 + 2 * e] * (__uint_as_float(dv[2 * e]) - dl_r),
+                                         pr[32 * c2 + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - dl_r));
                     tmem_st16(tB + 64 * hf + 16 * c2, w);  // over dP columns this warp has read
                 }
                 tmem_wait_st();
@@ -490,44 +551,81 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (it.steps == 0) continue;
                 if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
                 ++fix_use;
+                // Two phases per step i: S^T_i and dP^T_i are in tensor memory;
+                // once P^T_i is written, dV += P^T_i dO_i and S^T_{i+1} (over S^T_i's
+                // columns, after dV read them); once dS^T_i is written, dK += dS^T_i
+                // Q_i and dP^T_{i+1}.  The elementwise warps compute P^T_{i+1} while
+                // the tensor core finishes step i.
+                uint32_t sq = cons % C::kSlots;
+                if (!mbar_wait(bar.ring_full(sq), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                ++cons;
+                uint32_t sd = cons % C::kSlots;
+                if (!mbar_wait(bar.ring_full(sd), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
+                ++cons;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk), d_ring + sq * kTileStep + kstep_off<D>(kk),
+                            kIdescS, kk > 0 ? 1u : 0u);
+                umma_commit(bar.mm_full());
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk), d_ring + sd * kTileStep + kstep_off<D>(kk),
+                            kIdescS, kk > 0 ? 1u : 0u);
+                umma_commit(bar.dp_full());
+                if (it.steps == 1) umma_commit(bar.fix_empty());
                 for (int step = 0; step < it.steps; ++step) {
-                    const uint32_t sq = cons % C::kSlots;
-                    if (!mbar_wait(bar.ring_full(sq), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
-                    ++cons;
-                    const uint32_t sd = cons % C::kSlots;
-                    if (!mbar_wait(bar.ring_full(sd), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
-                    ++cons;
-                    tc_fence_after();
-                    // S^T = K Q^T, dP^T = V dO^T
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk), d_ring + sq * kTileStep + kstep_off<D>(kk),
-                                kIdescS, kk > 0 ? 1u : 0u);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk), d_ring + sd * kTileStep + kstep_off<D>(kk),
-                                kIdescS, kk > 0 ? 1u : 0u);
-                    umma_commit(bar.mm_full());
-                    if (step == it.steps - 1) umma_commit(bar.fix_empty());
-                    if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
-                    ++op_cnt;
+                    const bool more = step + 1 < it.steps;
+                    // the previous item's dK, dV must have been read before they restart
                     if (step == 0 && acc_use > 0 &&
                         !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
                         goto mma_out;
+                    // dV += P^T dO (P^T over S^T columns 0-31 and 64-95)
+                    if (!mbar_wait(bar.pt_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
                     tc_fence_after();
-                    // dV += P^T dO (P^T over S^T columns 0-31 and 64-95),
-                    // dK += dS^T Q (dS^T over dP^T columns 0-31 and 64-95)
 #pragma unroll
-                    for (int kk = 0; kk < kBlockQ / 16; ++kk) {
+                    for (int kk = 0; kk < kBlockQ / 16; ++kk)
                         umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemA + packed_col(kk),
                                 d_ring_mn + sd * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(bar.ring_empty(sd));  // dO_i's last use
+                    uint32_t nq = 0, nd = 0;
+                    if (more) {
+                        nq = cons % C::kSlots;
+                        if (!mbar_wait(bar.ring_full(nq), (cons / C::kSlots) & 1, st.abort_flag, p.status))
+                            goto mma_out;
+                        ++cons;
+                        nd = cons % C::kSlots;
+                        if (!mbar_wait(bar.ring_full(nd), (cons / C::kSlots) & 1, st.abort_flag, p.status))
+                            goto mma_out;
+                        ++cons;
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk),
+                                    d_ring + nq * kTileStep + kstep_off<D>(kk), kIdescS, kk > 0 ? 1u : 0u);
+                        umma_commit(bar.mm_full());
+                    }
+                    // dK += dS^T Q (dS^T over dP^T columns 0-31 and 64-95)
+                    if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++op_cnt;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kBlockQ / 16; ++kk)
                         umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + packed_col(kk),
                                 d_ring_mn + sq * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(bar.ring_empty(sq));  // Q_i's last use
+                    if (more) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk),
+                                    d_ring + nd * kTileStep + kstep_off<D>(kk), kIdescS, kk > 0 ? 1u : 0u);
+                        umma_commit(bar.dp_full());
+                        if (step + 2 == it.steps) umma_commit(bar.fix_empty());  // K, V's last use
+                        sq = nq;
+                        sd = nd;
                     }
-                    umma_commit(bar.ring_empty(sq));
-                    umma_commit(bar.ring_empty(sd));
                 }
                 umma_commit(bar.acc_full());
                 ++acc_use;
@@ -587,35 +685,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                     stage[128 + 32 * ch + lane] = q < p.L ? __ldg(dl_h + q) : 0.f;
                 }
                 __syncwarp();
+                // phase 1: P^T = 2^(S^T c - lse) from S^T (kept in fp32 for dS^T)
                 if (!__all_sync(0xffffffffu, mbar_wait(bar.mm_full(), mm_cnt & 1, st.abort_flag, p.status)))
+                    goto ew_out;
+                tc_fence_after();
+                float pt[64];
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int ch = 2 * hf + c2;
+                    uint32_t sv[32], wp[16];
+                    tmem_ld32(tA + 32 * ch, sv);
+                    const int qc = q0 + 32 * ch;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const bool allowed = (qc + e >= q_lo) & (qc + e <= q_hi);
+                        const float ev = ex2(fmaf(__uint_as_float(sv[e]), c, stage[32 * ch + e]));
+                        pt[32 * c2 + e] = allowed ? ev : 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) wp[e] = pack_bf16(pt[32 * c2 + 2 * e], pt[32 * c2 + 2 * e + 1]);
+                    tmem_st16(tA + 64 * hf + 16 * c2, wp);  // over S^T columns this warp has read
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.pt_full());
+                // phase 2: dS^T = P^T (dP^T - delta) from dP^T
+                if (!__all_sync(0xffffffffu, mbar_wait(bar.dp_full(), mm_cnt & 1, st.abort_flag, p.status)))
                     goto ew_out;
                 ++mm_cnt;
                 tc_fence_after();
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
                     const int ch = 2 * hf + c2;
-                    uint32_t sv[32], dv[32], wp[16], wd[16];
-                    tmem_ld32(tA + 32 * ch, sv);
+                    uint32_t dv[32], wd[16];
                     tmem_ld32(tB + 32 * ch, dv);
-                    const int qc = q0 + 32 * ch;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float nlse_q = stage[32 * ch + e];
-                        const float dl_q = stage[128 + 32 * ch + e];
-                        const bool allowed = (qc + e >= q_lo) & (qc + e <= q_hi);
-                        const float ev = ex2(fmaf(__uint_as_float(sv[e]), c, nlse_q));
-                        const float pv = allowed ? ev : 0.f;
-                        const float ds = pv * (__uint_as_float(dv[e]) - dl_q);
-                        // pack in pairs as they complete
-                        if (e & 1) {
-                            wp[e >> 1] = pack_bf16(__uint_as_float(sv[e - 1]), pv);
-                            wd[e >> 1] = pack_bf16(__uint_as_float(dv[e - 1]), ds);
-                        } else {
-                            sv[e] = __float_as_uint(pv);  // keep the even element until its pair is done
-                            dv[e] = __float_as_uint(ds);
-                        }
+                    for (int e = 0; e < 16; ++e) {
+                        const float d0 = pt[32 * c2 + 2 * e] * (__uint_as_float(dv[2 * e]) - stage[128 + 32 * ch + 2 * e]);
+                        const float d1 =
+                            pt[32 * c2 + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - stage[128 + 32 * ch + 2 * e + 1]);
+                        wd[e] = pack_bf16(d0, d1);
                     }
-                    tmem_st16(tA + 64 * hf + 16 * c2, wp);  // over S^T columns this warp has read
                     tmem_st16(tB + 64 * hf + 16 * c2, wd);  // over dP^T columns this warp has read
                 }
                 tmem_wait_st();

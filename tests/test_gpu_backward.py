@@ -77,6 +77,9 @@ CASES = [
     ("decode_l1", shaped(2, 14, 2, 1, 1000, 128)),
     ("decode_l5_window", shaped(1, 8, 2, 5, 700, 128, window=200)),
     ("long_keys_split", shaped(1, 2, 1, 256, 20000, 128, k_scale=2.0)),
+    # more items than CTAs, each with 1-4 key tiles: a CTA moves to its next
+    # item while the tensor core may have run two score tiles ahead
+    ("multi_item_short_ranges", shaped(2, 32, 4, 512, 512, 128)),
 ]
 
 
