@@ -241,8 +241,14 @@ int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o,
  * read, o written; plain or pinned host memory), for L >= 9 as tfa_prefill and
  * for 1 <= L <= 8 as tfa_decode.  The library copies the
  * inputs to device staging buffers it owns (one set per device, grown on
- * demand and kept until process exit), runs tfa_prefill on `stream`, copies o
- * back and synchronizes the stream before returning.  Not safe to call from
+ * demand and kept until process exit), runs the attention, copies o back and
+ * synchronizes before returning.  The work is pipelined over up to 4 stages
+ * of KV groups (ranges of groups of one batch element, or runs of whole
+ * elements when B > 4): a stage's inputs are copied in on a library-owned
+ * stream while the previous stage computes on `stream` and the one before is
+ * copied out on a second library-owned stream.  With pinned host memory the
+ * transfers overlap the computation; with plain memory the copies are
+ * synchronous to the host and the result is the same.  Not safe to call from
  * two host threads on the same device at once. */
 int tfa_prefill_host(const void *q, const void *k, const void *v, void *o,
                      int B, int Hq, int Hkv, int L, int S, int D, float scale,

@@ -43,6 +43,7 @@ struct BwdScratch {
 };
 
 constexpr int kVariantsPerD = 18;  // forward kernel variants per head dim (variant_index)
+constexpr int kHostStages = 4;     // tfa_prefill_host: most pipeline stages per call (measured best of 4, 8, 16)
 
 struct DeviceState {
     bool init = false;
@@ -52,9 +53,11 @@ struct DeviceState {
     std::unordered_map<cudaStream_t, SplitScratch> split;
     std::unordered_map<cudaStream_t, BwdScratch> bwd;
     bool bwd_attr[4] = {};  // backward kernels prepared, per (D, key mask)
-    // staging buffers of tfa_prefill_host
+    // staging buffers of tfa_prefill_host, and its copy streams and events
     void *h_buf[5] = {nullptr, nullptr, nullptr, nullptr, nullptr};
     size_t h_cap[5] = {0, 0, 0, 0, 0};
+    cudaStream_t h_in = nullptr, h_out = nullptr;
+    cudaEvent_t h_ev[2 * kHostStages + 1] = {};
 };
 
 std::mutex g_mutex;
@@ -685,23 +688,91 @@ extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, voi
         (rc = ensure_capacity(*st, 2, kbytes)) || (rc = ensure_capacity(*st, 3, qbytes)) ||
         (mbytes && (rc = ensure_capacity(*st, 4, mbytes))))
         return rc;
-    if (cudaMemcpyAsync(st->h_buf[0], q, qbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(st->h_buf[1], k, kbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(st->h_buf[2], v, kbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        (mbytes && cudaMemcpyAsync(st->h_buf[4], key_mask, mbytes, cudaMemcpyHostToDevice, s) !=
-                       cudaSuccess))
-        return TFA_ERR_CUDA;
-    const float *dmask = mbytes ? static_cast<const float *>(st->h_buf[4]) : nullptr;
+    if (!st->h_in) {
+        cudaError_t e = cudaStreamCreateWithFlags(&st->h_in, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&st->h_out, cudaStreamNonBlocking);
+        for (int i = 0; i < 2 * kHostStages + 1 && e == cudaSuccess; ++i)
+            e = cudaEventCreateWithFlags(&st->h_ev[i], cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail("tfa_prefill_host stream/event setup", e);
+    }
     SplitScratch *ss = nullptr;
     if ((rc = split_scratch(*st, s, &ss))) return rc;
-    rc = (D == 128) ? launch<128>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
-                                  Hkv, L, S, scale, causal, window, dmask, s, 0u, ss, false, decode)
-                    : launch<64>(*st, st->h_buf[0], st->h_buf[1], st->h_buf[2], st->h_buf[3], B, Hq,
-                                 Hkv, L, S, scale, causal, window, dmask, s, 0u, ss, false, decode);
-    if (rc) return rc;
-    if (cudaMemcpyAsync(o, st->h_buf[3], qbytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    // Pipeline stages over KV groups, which are contiguous in the
+    // [B, H, rows, D] layouts (group g of batch b: query planes b Hq + g G ..,
+    // KV plane b Hkv + g): stage i's inputs are copied in on h_in while stage
+    // i - 1 computes on `stream` and stage i - 2's output is copied out on
+    // h_out.  Up to kHostStages batch elements: ranges of groups inside one element;
+    // beyond: runs of whole elements.
+    const int G = Hq / Hkv;
+    int per_b = 1, gps = Hkv, bps = 1;  // stages per element, groups per stage, elements per stage
+    if (B <= kHostStages) {
+        per_b = kHostStages / B < Hkv ? kHostStages / B : Hkv;
+        gps = (Hkv + per_b - 1) / per_b;
+        per_b = (Hkv + gps - 1) / gps;
+    } else {
+        bps = (B + kHostStages - 1) / kHostStages;
+    }
+    const int n_stages = B <= kHostStages ? B * per_b : (B + bps - 1) / bps;
+    const size_t q_plane = static_cast<size_t>(L) * D * 2, k_plane = static_cast<size_t>(S) * D * 2;
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k),
+               *hv = static_cast<const char *>(v);
+    char *dq = static_cast<char *>(st->h_buf[0]), *dk = static_cast<char *>(st->h_buf[1]),
+         *dv = static_cast<char *>(st->h_buf[2]), *dout = static_cast<char *>(st->h_buf[3]);
+    const float *dmask = mbytes ? static_cast<const float *>(st->h_buf[4]) : nullptr;
+    // the caller's earlier work on `stream` comes first
+    if (cudaEventRecord(st->h_ev[2 * kHostStages], s) != cudaSuccess ||
+        cudaStreamWaitEvent(st->h_in, st->h_ev[2 * kHostStages], 0) != cudaSuccess)
         return TFA_ERR_CUDA;
-    if (cudaStreamSynchronize(s) != cudaSuccess) return TFA_ERR_CUDA;
+    if (mbytes && cudaMemcpyAsync(st->h_buf[4], key_mask, mbytes, cudaMemcpyHostToDevice, st->h_in) != cudaSuccess)
+        return TFA_ERR_CUDA;
+    for (int i = 0; i < n_stages; ++i) {
+        // query planes [qp0, qp0 + nq), KV planes [kp0, kp0 + nk) of this stage; the
+        // kernel sees them as Bs elements of Hs query and Hks KV heads
+        int b0, Bs, Hs, Hks;
+        size_t qp0, kp0;
+        if (B <= kHostStages) {
+            b0 = i / per_b;
+            const int g0 = (i % per_b) * gps;
+            const int ng = Hkv - g0 < gps ? Hkv - g0 : gps;
+            Bs = 1;
+            Hs = ng * G;
+            Hks = ng;
+            qp0 = static_cast<size_t>(b0) * Hq + static_cast<size_t>(g0) * G;
+            kp0 = static_cast<size_t>(b0) * Hkv + g0;
+        } else {
+            b0 = i * bps;
+            Bs = B - b0 < bps ? B - b0 : bps;
+            Hs = Hq;
+            Hks = Hkv;
+            qp0 = static_cast<size_t>(b0) * Hq;
+            kp0 = static_cast<size_t>(b0) * Hkv;
+        }
+        const size_t nq = static_cast<size_t>(Bs) * Hs, nk = static_cast<size_t>(Bs) * Hks;
+        if (cudaMemcpyAsync(dq + qp0 * q_plane, hq + qp0 * q_plane, nq * q_plane, cudaMemcpyHostToDevice, st->h_in) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(dk + kp0 * k_plane, hk + kp0 * k_plane, nk * k_plane, cudaMemcpyHostToDevice, st->h_in) !=
+                cudaSuccess ||
+            cudaMemcpyAsync(dv + kp0 * k_plane, hv + kp0 * k_plane, nk * k_plane, cudaMemcpyHostToDevice, st->h_in) !=
+                cudaSuccess ||
+            cudaEventRecord(st->h_ev[2 * i], st->h_in) != cudaSuccess ||
+            cudaStreamWaitEvent(s, st->h_ev[2 * i], 0) != cudaSuccess)
+            return TFA_ERR_CUDA;
+        const float *smask = dmask ? dmask + static_cast<size_t>(b0) * S : nullptr;
+        rc = (D == 128) ? launch<128>(*st, dq + qp0 * q_plane, dk + kp0 * k_plane, dv + kp0 * k_plane,
+                                      dout + qp0 * q_plane, Bs, Hs, Hks, L, S, scale, causal, window, smask, s, 0u,
+                                      ss, false, decode)
+                        : launch<64>(*st, dq + qp0 * q_plane, dk + kp0 * k_plane, dv + kp0 * k_plane,
+                                     dout + qp0 * q_plane, Bs, Hs, Hks, L, S, scale, causal, window, smask, s, 0u,
+                                     ss, false, decode);
+        if (rc) return rc;
+        if (cudaEventRecord(st->h_ev[2 * i + 1], s) != cudaSuccess ||
+            cudaStreamWaitEvent(st->h_out, st->h_ev[2 * i + 1], 0) != cudaSuccess ||
+            cudaMemcpyAsync(static_cast<char *>(o) + qp0 * q_plane, dout + qp0 * q_plane, nq * q_plane,
+                            cudaMemcpyDeviceToHost, st->h_out) != cudaSuccess)
+            return TFA_ERR_CUDA;
+    }
+    if (cudaStreamSynchronize(st->h_out) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess)
+        return TFA_ERR_CUDA;
     return TFA_OK;
 }
 

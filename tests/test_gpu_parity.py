@@ -168,6 +168,24 @@ def test_host_entry_matches_device_entry():
     assert torch.equal(host, dev.cpu())
 
 
+@pytest.mark.parametrize("name,w,pinned", [
+    # three pipeline stages, one batch element each, with a key mask and D = 64
+    ("b3_element_stages", shaped(3, 8, 4, 64, 300, 64, key_mask_keep=0.7), True),
+    # 20 batch elements: four stages of five whole elements; short rows run packed
+    ("b20_batch_stages", shaped(20, 4, 2, 16, 130, 128), True),
+    # pageable host memory (copies synchronous to the host, same results); two
+    # stages per element over its three KV groups (2 + 1)
+    ("pageable_ragged_groups", shaped(2, 6, 3, 150, 400, 128, window=100), False),
+])
+def test_host_entry_pipelined_stages(name, w, pinned):
+    q, k, v, km = make_inputs(w, seed=11)
+    dev, _ = _run(w, inputs=(q, k, v, km))
+    prep = (lambda t: t.pin_memory()) if pinned else (lambda t: t)
+    host = tb.prefill_host(prep(q), prep(k), prep(v), scale=w.softmax_scale, causal=w.causal,
+                           window=w.window, key_mask=km)
+    assert torch.equal(host, dev.cpu()), name
+
+
 def test_stream_argument_is_respected():
     w = shaped(1, 4, 2, 128, 256, 128)
     q, k, v, _ = make_inputs(w, seed=8)
