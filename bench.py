@@ -355,6 +355,20 @@ def main():
     value = weak_scaling_rate(flops, world, mean_ms * 1e-3) / 1e12
     per_sorted = sorted(per)
 
+    # L2-warm reference (no flush between launches; the inputs of the previous
+    # launch may still be in L2): reported beside the flushed headline, not in it
+    n_warm = min(args.steps, 50)
+    w_starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_warm)]
+    w_ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_warm)]
+    for i in range(n_warm):
+        w_starts[i].record(stream)
+        step()
+        w_ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    tb.check_status(stream)
+    warm_sorted = sorted(s_.elapsed_time(e_) for s_, e_ in zip(w_starts, w_ends))
+    warm_ms = max_over_ranks(warm_sorted[len(warm_sorted) // 2], world)
+
     # end to end through the C ABI with host buffers (copies inside the timed region)
     pinned = [t.pin_memory() if t is not None else None for t in host_inputs]
     hq, hk, hv, hkm = pinned[:4]
@@ -424,6 +438,8 @@ def main():
                        "parallelism": f"weak x{world}" if world > 1 else "single GPU"},
             "ms_p10": per_sorted[len(per) // 10], "ms_p50": per_sorted[len(per) // 2],
             "ms_p90": per_sorted[(9 * len(per)) // 10],
+            "l2_warm": {"ms_p50": warm_ms, "value": weak_scaling_rate(flops, world, warm_ms * 1e-3) / 1e12,
+                        "unit": UNIT, "launches": n_warm},
             "pct_of_peak": 100.0 * achieved / peak,
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                          "unit": roof_unit, "frac": achieved / peak,
