@@ -105,7 +105,12 @@ struct SegIter {
     long long pos, end;   // split: current / end global step
     long long gstart;     // split: first global step of group r
     int r, gsteps, bh;    // split: current group, steps per item in it, items per group
-    int item, stride, n_items;  // whole-item schedule
+    // whole-item schedule: CTA c visits items c, 2G - 1 - c, 2G + c, 4G - 1 - c,
+    // ... (G CTAs): the step alternates between 2G - 1 - 2c and 2c + 1, which sum
+    // to 2G.  Items come largest first (causal tile pairs in decreasing order),
+    // so alternating the direction pairs a CTA's large items with small ones.
+    // Once a CTA's item is past the end, so are all its later ones.
+    int item, stride, n_items;
     SeqTable seq;  // varlen batches (whole-item schedule only); q_start == nullptr otherwise
 
     TFA_HD void init(const Shape &s, long long W, int c) {
@@ -113,7 +118,7 @@ struct SegIter {
         bh = s.B * s.Hq;
         n_items = s.n_qp * bh;
         item = c;
-        stride = s.grid;
+        stride = 2 * s.grid - 1 - 2 * c;
         pos = cta_begin(W, s.grid, c);
         end = cta_begin(W, s.grid, c + 1);
         r = 0;
@@ -138,6 +143,7 @@ struct SegIter {
                 seg.b = rem / s.Hq;
                 seg.h = rem - seg.b * s.Hq;
                 item += stride;
+                stride = 2 * s.grid - stride;
                 seg.L = s.L;
                 seg.S = s.S;
                 seg.q_base = 0;
