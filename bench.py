@@ -301,6 +301,12 @@ def main():
         extra = ()
     host_inputs = [q, k, v, km, sinks, *extra]  # what one call reads (None: absent)
     dev_inputs = [t.to(dev) if t is not None else None for t in host_inputs]
+    if w.saved_stats:  # the forward's output and log-sum-exp, made once before any timing
+        o_saved, lse_saved = tb.prefill_lse(*dev_inputs[:3], scale=w.softmax_scale, causal=w.causal,
+                                            window=w.window, key_mask=dev_inputs[3])
+        torch.cuda.synchronize(dev)
+        host_inputs += [o_saved.cpu(), lse_saved.cpu()]
+        dev_inputs += [o_saved, lse_saved]
     if w.kind == "backward":  # (dq, dk, dv)
         out = tuple(torch.empty_like(t) for t in dev_inputs[:3])
     else:
@@ -314,7 +320,7 @@ def main():
         dq, dk, dv, dkm, dsinks = ins[:5]
         if w.kind == "backward":
             tb.backward(dq, dk, dv, ins[5], scale=w.softmax_scale, causal=w.causal, window=w.window,
-                        key_mask=dkm, out=o)
+                        key_mask=dkm, out=o, saved=(ins[6], ins[7]) if w.saved_stats else None)
         elif w.kind == "varlen":
             tb.prefill_varlen(dq, dk, dv, ins[5], ins[6], max_seqlen_q=w.L, scale=w.softmax_scale,
                               causal=w.causal, window=w.window, softcap=w.softcap, sinks=dsinks,
@@ -390,7 +396,8 @@ def main():
             for h, d in (zip(hout, eout) if w.kind == "backward" else [(hout, eout)]):
                 h.copy_(d, non_blocking=True)
         entry = {"varlen": "tfa_prefill_varlen", "ring": "tfa_prefill_ring",
-                 "backward": "tfa_prefill_backward"}.get(w.kind, "tfa_attention_ex")
+                 "backward": "tfa_prefill_backward_saved" if w.saved_stats else "tfa_prefill_backward"
+                 }.get(w.kind, "tfa_attention_ex")
         e2e_api = f"{entry} (pinned host buffers, copies on the stream)"
     else:
         def e2e_step():
@@ -450,8 +457,8 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "api": e2e_api},
             # kernels per step: one, or four for the backward (forward recompute,
-            # delta, dQ, dK/dV)
-            "gpu_launches": args.steps * (4 if w.kind == "backward" else 1),
+            # delta, dQ, dK/dV), three when it starts from the saved statistics
+            "gpu_launches": args.steps * ((3 if w.saved_stats else 4) if w.kind == "backward" else 1),
             "clocks": clocks,
             "wall_s_timed_region": t_wall,
         }

@@ -218,6 +218,30 @@ int tfa_prefill_backward(const void *q, const void *k, const void *v, const void
                          int D, float scale, int causal, int window, const float *key_mask,
                          tfa_stream_t stream);
 
+/* tfa_prefill_lse -- tfa_prefill (any L >= 1) that also writes each query
+ * row's base-2 log-sum-exp of its scaled scores,
+ *   lse[b, h, i] = log2( sum over allowed j of 2^(scale * log2(e) * q.k_j) )
+ * (+inf for a row with no allowed key), fp32 [B, Hq, L], caller-owned device
+ * memory, 4-byte aligned (TFA_ERR_NULL if NULL, TFA_ERR_ALIGN if not).  Other
+ * arguments, layouts, errors and asynchrony are tfa_prefill's.  The output
+ * and lse are what tfa_prefill_backward_saved takes. */
+int tfa_prefill_lse(const void *q, const void *k, const void *v, void *o, float *lse,
+                    int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                    int causal, int window, const float *key_mask, tfa_stream_t stream);
+
+/* tfa_prefill_backward_saved -- tfa_prefill_backward given the forward's
+ * output o (bf16 [B, Hq, L, D], 16-byte aligned) and lse (fp32 [B, Hq, L],
+ * 4-byte aligned) as tfa_prefill_lse wrote them for the same q, k, v, mask,
+ * scale, causal and window: the forward is not re-run (the usual training
+ * order, the forward's statistics saved for the backward).  Gradients,
+ * layouts, workspace, errors and asynchrony as for tfa_prefill_backward;
+ * NULL o or lse returns TFA_ERR_NULL.  With o and lse from tfa_prefill_lse
+ * the gradients are bit-identical to tfa_prefill_backward's. */
+int tfa_prefill_backward_saved(const void *q, const void *k, const void *v, const void *o,
+                               const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                               int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                               int causal, int window, const float *key_mask, tfa_stream_t stream);
+
 /* Debug flags for tfa_prefill_debug. */
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
 #define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */

@@ -84,6 +84,10 @@ def lib():
             L.tfa_attention_ex.restype = i32
             L.tfa_prefill_backward.argtypes = [P] * 7 + [i32] * 6 + [f32, i32, i32, P, P]
             L.tfa_prefill_backward.restype = i32
+            L.tfa_prefill_lse.argtypes = [P] * 5 + [i32] * 6 + [f32, i32, i32, P, P]
+            L.tfa_prefill_lse.restype = i32
+            L.tfa_prefill_backward_saved.argtypes = [P] * 9 + [i32] * 6 + [f32, i32, i32, P, P]
+            L.tfa_prefill_backward_saved.restype = i32
             L.tfa_prefill_ring.argtypes = [P, P, P, P] + [i32] * 7 + [f32, i32, f32, P, P]
             L.tfa_prefill_ring.restype = i32
             L.tfa_prefill_varlen.argtypes = [P] * 6 + [i32] * 7 + [f32, i32, i32, f32, P, P]
@@ -293,10 +297,38 @@ def tfa_prefill_backward(q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, D, scale, 
                                       window, key_mask, stream)
 
 
+def prefill_lse(q, k, v, *, scale=None, causal=True, window=0, key_mask=None, out=None, lse=None,
+                stream=None):
+    """(o, lse): the forward of any L >= 1 and each row's base-2 log-sum-exp of
+    its scaled scores, fp32 [B,Hq,L] (+inf for a row with no allowed key)."""
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, Hq, L, D = q.shape
+    Bk, Hkv, S, Dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or Dk != D:
+        raise ValueError("q, k and v disagree")
+    if key_mask is not None:
+        _check(key_mask, "key_mask", torch.float32, 2)
+    scale = 1.0 / math.sqrt(D) if scale is None else scale
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(out, "out", torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    rc = lib().tfa_prefill_lse(*(ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, out, lse)),
+                               B, Hq, Hkv, L, S, D, float(scale), int(bool(causal)), int(window),
+                               _ptr_or_none(key_mask), _stream_handle(stream))
+    if rc != TFA_OK:
+        raise TfaError(rc, "tfa_prefill_lse")
+    return out, lse
+
+
 def backward(q, k, v, dout, *, scale=None, causal=True, window=0, key_mask=None, out=None,
-             stream=None):
+             saved=None, stream=None):
     """(dq, dk, dv) bf16 of the attention core for the upstream gradient dout
-    [B,Hq,L,D] (recompute-based: the forward is re-run inside)."""
+    [B,Hq,L,D]: recompute-based (the forward is re-run inside), or, given
+    saved=(o, lse) from prefill_lse on the same inputs, from those."""
     import torch
 
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (dout, "dout")):
@@ -315,6 +347,19 @@ def backward(q, k, v, dout, *, scale=None, causal=True, window=0, key_mask=None,
         _check(t, n, torch.bfloat16, 4)
         if tuple(t.shape) != tuple(ref.shape):
             raise ValueError(f"{n} has the wrong shape")
+    if saved is not None:
+        o, lse = saved
+        _check(o, "o", torch.bfloat16, 4)
+        _check(lse, "lse", torch.float32, 3)
+        if tuple(o.shape) != tuple(q.shape) or tuple(lse.shape) != (B, Hq, L):
+            raise ValueError("saved (o, lse) have the wrong shape")
+        rc = lib().tfa_prefill_backward_saved(
+            *(ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, o, lse, dout, dq, dk, dv)),
+            B, Hq, Hkv, L, S, D, float(scale), int(bool(causal)), int(window), _ptr_or_none(key_mask),
+            _stream_handle(stream))
+        if rc != TFA_OK:
+            raise TfaError(rc, "tfa_prefill_backward_saved")
+        return dq, dk, dv
     rc = tfa_prefill_backward(*(ctypes.c_void_p(t.data_ptr()) for t in (q, k, v, dout, dq, dk, dv)),
                               B, Hq, Hkv, L, S, D, float(scale), int(bool(causal)), int(window),
                               _ptr_or_none(key_mask), _stream_handle(stream))

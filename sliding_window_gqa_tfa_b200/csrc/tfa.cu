@@ -579,22 +579,30 @@ extern "C" int tfa_prefill_varlen(const void *q, const void *k, const void *v, v
 namespace {
 // Backward: a forward recompute (output and log-sum-exp into the workspace),
 // delta = rowsum(dO o O), then the dQ and the dK/dV kernels, all on `stream`.
+// o_saved / lse_saved: the forward's output and per-row log-sum-exp (as
+// tfa_prefill_lse writes them), or nullptr to recompute both into the workspace.
 template <int D>
 int backward_impl(DeviceState &st, SplitScratch *ss, BwdScratch &bs, const void *q, const void *k,
                   const void *v, const void *dout, void *dq, void *dk, void *dv, int B, int Hq,
                   int Hkv, int L, int S, float scale, int causal, int window, const float *key_mask,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, const void *o_saved = nullptr, const float *lse_saved = nullptr) {
     namespace bw = tfa::bwd;
-    const bool decode = L <= TFA_MAX_DECODE_ROWS;
-    Addressing ad;
-    ad.lse = bs.lse;
-    int rc = launch<D>(st, q, k, v, bs.o, B, Hq, Hkv, L, S, scale, causal, window, key_mask, stream, 0u,
-                       ss, false, decode, 0.f, nullptr, ad);
-    if (rc) return rc;
+    const void *o = o_saved;
+    const float *lse = lse_saved;
+    if (!o) {
+        const bool decode = L <= TFA_MAX_DECODE_ROWS;
+        Addressing ad;
+        ad.lse = bs.lse;
+        const int rc = launch<D>(st, q, k, v, bs.o, B, Hq, Hkv, L, S, scale, causal, window, key_mask, stream,
+                                 0u, ss, false, decode, 0.f, nullptr, ad);
+        if (rc) return rc;
+        o = bs.o;
+        lse = bs.lse;
+    }
     const long long rows = static_cast<long long>(B) * Hq * L;
     const long long threads = rows * 32;
     bw::delta_kernel<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16 *>(bs.o), static_cast<const __nv_bfloat16 *>(dout), bs.delta, rows);
+        static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), bs.delta, rows);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("delta kernel launch", e);
     CUtensorMap mq, mdo, mk, mv;
@@ -606,7 +614,7 @@ int backward_impl(DeviceState &st, SplitScratch *ss, BwdScratch &bs, const void 
     p.dq = static_cast<__nv_bfloat16 *>(dq);
     p.dk = static_cast<__nv_bfloat16 *>(dk);
     p.dv = static_cast<__nv_bfloat16 *>(dv);
-    p.lse = bs.lse;
+    p.lse = lse;
     p.delta = bs.delta;
     p.key_mask = key_mask;
     p.status = st.status;
@@ -659,6 +667,50 @@ extern "C" int tfa_prefill_backward(const void *q, const void *k, const void *v,
                                            causal, window, key_mask, s)
                       : backward_impl<64>(*st, ss, *bs, q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, scale,
                                           causal, window, key_mask, s);
+}
+
+extern "C" int tfa_prefill_lse(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                               int Hq, int Hkv, int L, int S, int D, float scale, int causal, int window,
+                               const float *key_mask, tfa_stream_t stream) {
+    const bool decode = L >= 1 && L <= TFA_MAX_DECODE_ROWS;
+    int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true, decode);
+    if (rc) return rc;
+    if (!lse) return TFA_ERR_NULL;
+    if (reinterpret_cast<uintptr_t>(lse) & 3u) return TFA_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    SplitScratch *ss = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st)) || (rc = split_scratch(*st, s, &ss))) return rc;
+    Addressing ad;
+    ad.lse = lse;
+    return (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window, key_mask, s, 0u,
+                                    ss, false, decode, 0.f, nullptr, ad)
+                      : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window, key_mask, s, 0u,
+                                   ss, false, decode, 0.f, nullptr, ad);
+}
+
+extern "C" int tfa_prefill_backward_saved(const void *q, const void *k, const void *v, const void *o,
+                                          const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                                          int B, int Hq, int Hkv, int L, int S, int D, float scale,
+                                          int causal, int window, const float *key_mask, tfa_stream_t stream) {
+    const bool decode = L >= 1 && L <= TFA_MAX_DECODE_ROWS;
+    int rc = validate(q, k, v, dout, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true, decode);
+    if (rc) return rc;
+    if (!o || !lse || !dq || !dk || !dv) return TFA_ERR_NULL;
+    auto mis16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; };
+    if (mis16(o) || mis16(dq) || mis16(dk) || mis16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return TFA_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    DeviceState *st = nullptr;
+    BwdScratch *bs = nullptr;
+    std::lock_guard<std::mutex> lk(g_mutex);
+    if ((rc = device_state(s, &st)) || (rc = bwd_scratch(*st, s, static_cast<size_t>(B) * Hq * L, D, &bs)))
+        return rc;
+    return (D == 128) ? backward_impl<128>(*st, nullptr, *bs, q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, scale,
+                                           causal, window, key_mask, s, o, lse)
+                      : backward_impl<64>(*st, nullptr, *bs, q, k, v, dout, dq, dk, dv, B, Hq, Hkv, L, S, scale,
+                                          causal, window, key_mask, s, o, lse);
 }
 
 extern "C" int tfa_prefill_debug(const void *q, const void *k, const void *v, void *o, int B,

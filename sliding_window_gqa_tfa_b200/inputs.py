@@ -49,6 +49,9 @@ class Workload:
     seqlens: tuple | None = None
     # the backward pass (gradients of q, k, v for an upstream gradient of the output)
     backward: bool = False
+    # backward given the forward's output and per-row log-sum-exp (computed once,
+    # before any timing, as a training step's forward would leave them)
+    saved_stats: bool = False
 
     @property
     def kind(self) -> str:
@@ -106,6 +109,9 @@ WORKLOADS: dict[str, Workload] = {w.name: w for w in [
     # The backward pass on the Llama chunk (gradients of q, k, v).
     Workload("llama_gqa_chunk_2048x8192_backward", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
              backward=True),
+    # The same backward from the forward's saved output and log-sum-exp.
+    Workload("llama_gqa_chunk_2048x8192_backward_saved", B=1, Hq=56, Hkv=8, L=2048, S=8192, D=128,
+             backward=True, saved_stats=True),
     # Short queries (1 <= L <= 8): token-by-token decoding over a long cache,
     # batched Qwen3-shaped decoding, and an 8-row chunk (e.g. draft verification).
     Workload("llama_gqa_decode_1x32768", B=1, Hq=56, Hkv=8, L=1, S=32768, D=128),

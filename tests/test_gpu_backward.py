@@ -183,3 +183,80 @@ def test_backward_full_size_sampled():
     rk_ratio = _check(dk[0, g][kk], rk, bk, "full-size dk rows")
     rv_ratio = _check(dv[0, g][kk], rv, bv, "full-size dv rows")
     print("full size worst error / bound", f"{ratio:.3g} {rk_ratio:.3g} {rv_ratio:.3g}")
+
+
+SAVED_CASES = [
+    ("causal_130x300", shaped(2, 4, 2, 130, 300, 128)),
+    ("d64_window_mask", shaped(1, 6, 3, 260, 900, 64, window=300, key_mask_keep=0.8)),
+    ("decode_l1", shaped(2, 14, 2, 1, 1000, 128)),
+    ("bidirectional", shaped(1, 4, 2, 190, 333, 128, causal=False, k_scale=3.0)),
+    ("fully_masked_batch", shaped(2, 4, 2, 150, 300, 128, key_mask_keep=0.7)),
+]
+
+
+def _saved_inputs(name, w):
+    q, k, v, km = make_inputs(w, seed=71)
+    if name == "fully_masked_batch":
+        km[1] = 0.0
+    do = _dout(q.shape, 72)
+    return q, k, v, km, do
+
+
+@pytest.mark.parametrize("name,w", SAVED_CASES, ids=[n for n, _ in SAVED_CASES])
+def test_saved_backward_is_the_recompute_backward(name, w):
+    """tfa_prefill_backward_saved on tfa_prefill_lse's (o, lse) gives the
+    recompute-based backward's gradients bit for bit (same kernels, same
+    statistics)."""
+    q, k, v, km, do = _saved_inputs(name, w)
+    Q, K, V, DO = (t.cuda() for t in (q, k, v, do))
+    KM = km.cuda() if km is not None else None
+    kw = dict(scale=w.softmax_scale, causal=w.causal, window=w.window, key_mask=KM)
+    o, lse = tb.prefill_lse(Q, K, V, **kw)
+    saved = tb.backward(Q, K, V, DO, saved=(o, lse), **kw)
+    recomputed = tb.backward(Q, K, V, DO, **kw)
+    tb.check_status()
+    for a, b, n in zip(saved, recomputed, ("dq", "dk", "dv")):
+        assert torch.equal(a, b), f"{name}: {n} differs"
+
+
+@pytest.mark.parametrize("name,w", SAVED_CASES, ids=[n for n, _ in SAVED_CASES])
+def test_lse_is_the_log_sum_exp(name, w):
+    """lse[b,h,i] = log2 sum_j exp(scale q.k_j) over the allowed keys, +inf for
+    a row with none.  Bound: the fp32 score sum (D products of bf16 values)
+    errs by at most D 2^-24 sum|q k| per score, and exp2.approx by ~2^-22
+    relative; both stay far below the 1e-3 (log2 units) asserted here.  The
+    output is checked against the oracle at the usual 0.02."""
+    q, k, v, km, _ = _saved_inputs(name, w)
+    Q, K, V = (t.cuda() for t in (q, k, v))
+    KM = km.cuda() if km is not None else None
+    o, lse = tb.prefill_lse(Q, K, V, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                            key_mask=KM)
+    tb.check_status()
+    ref_o = oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                             key_mask=km)
+    got_o = o.float().cpu().double().numpy()
+    assert np.allclose(got_o, ref_o, atol=0.02, rtol=0.02)
+    G = w.Hq // w.Hkv
+    P0 = w.S - w.L
+    i = np.arange(w.L)[:, None]
+    j = np.arange(w.S)[None, :]
+    allowed = np.ones((w.L, w.S), dtype=bool)
+    if w.causal:
+        allowed &= j <= P0 + i
+        if w.window > 0:
+            allowed &= j > P0 + i - w.window
+    got = lse.cpu().double().numpy()
+    Qd, Kd = q.double().numpy(), k.double().numpy()
+    for b in range(w.B):
+        al = allowed if km is None else allowed & (km[b].numpy() > 0.5)[None, :]
+        for h in range(w.Hq):
+            s = w.softmax_scale * (Qd[b, h] @ Kd[b, h // G].T)
+            s = np.where(al, s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            empty = ~al.any(axis=1)
+            mm = np.where(np.isfinite(m), m, 0.0)
+            ref = (mm[:, 0] + np.log(np.exp(s - mm).sum(axis=1))) / np.log(2.0)
+            g = got[b, h]
+            assert np.all(np.isposinf(g[empty])), f"{name}: empty rows must be +inf"
+            assert np.all(np.abs(g[~empty] - ref[~empty]) <= 1e-3), \
+                f"{name}: worst {np.abs(g[~empty] - ref[~empty]).max():.3g}"

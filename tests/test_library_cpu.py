@@ -248,3 +248,26 @@ def test_key_tile_enumeration_is_exact(case):
             assert hi < lo
         else:
             assert (lo, hi) == (qts[0], qts[-1]), (kt, lo, hi, qts[0], qts[-1])
+
+
+def test_lse_and_saved_backward_reject_before_launch():
+    L_ = tb.lib()
+    i = (1, 8, 2, 64, 200, 128)
+    # forward with log-sum-exp: NULL or misaligned lse, then tfa_prefill's own checks
+    assert L_.tfa_prefill_lse(A16, A16, A16, A16, None, *i, 0.1, 1, 0, None, None) == tb.TFA_ERR_NULL
+    assert L_.tfa_prefill_lse(A16, A16, A16, A16, ctypes.c_void_p(0x10002), *i, 0.1, 1, 0, None,
+                              None) == tb.TFA_ERR_ALIGN
+    assert L_.tfa_prefill_lse(A16, A16, A16, A16, A16, 1, 8, 3, 64, 200, 128, 0.1, 1, 0, None,
+                              None) == tb.TFA_ERR_HEADS
+    # backward from saved statistics: NULL o / lse / gradient, misaligned o or lse
+    args = [A16] * 9
+    for n, code in ((3, tb.TFA_ERR_NULL), (4, tb.TFA_ERR_NULL), (8, tb.TFA_ERR_NULL)):
+        bad = list(args)
+        bad[n] = None
+        assert L_.tfa_prefill_backward_saved(*bad, *i, 0.1, 1, 0, None, None) == code
+    for n, p in ((3, MIS), (4, ctypes.c_void_p(0x10002))):
+        bad = list(args)
+        bad[n] = p
+        assert L_.tfa_prefill_backward_saved(*bad, *i, 0.1, 1, 0, None, None) == tb.TFA_ERR_ALIGN
+    assert L_.tfa_prefill_backward_saved(*args, 1, 8, 2, 64, 200, 96, 0.1, 1, 0, None,
+                                         None) == tb.TFA_ERR_HEAD_DIM
