@@ -638,9 +638,21 @@ int backward_impl(DeviceState &st, SplitScratch *ss, BwdScratch &bs, const void 
     const long long nk_items = static_cast<long long>(B) * Hkv * ((S + tfa::kBlockK - 1) / tfa::kBlockK);
     p.n_items = static_cast<int>(nk_items);
     auto dkv_kern = key_mask ? bw::dkv_kernel<D, true> : bw::dkv_kernel<D, false>;
-    dkv_kern<<<static_cast<int>(nk_items < st.sm_count ? nk_items : st.sm_count), bw::kThreads, smem, stream>>>(
-        mq, mdo, mk, mv, p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail("dK/dV kernel launch", e);
+    // Programmatic stream serialisation: the dK/dV CTAs start on the SMs the
+    // dQ kernel's CTAs leave (the two kernels are independent; dK/dV waits for
+    // dQ's completion only before it exits).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(nk_items < st.sm_count ? nk_items : st.sm_count));
+    cfg.blockDim = dim3(bw::kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, dkv_kern, mq, mdo, mk, mv, p)) != cudaSuccess)
+        return cuda_fail("dK/dV kernel launch", e);
     return TFA_OK;
 }
 }  // namespace

@@ -23,8 +23,9 @@
 //               dS (bf16) written over dP, then dQ += dS K.
 //   dKV kernel: work item (b, KV head, 128-key tile), walking the query tiles
 //               of every head of the group that see it: S^T = K Q^T and
-//               dP^T = V dO^T, P^T and dS^T (bf16) written over them, then
-//               dV += P^T dO and dK += dS^T Q.
+//               dP^T = V dO^T, P^T and dS^T (bf16) both written over dP^T,
+//               then dV += P^T dO and dK += dS^T Q; S^T of the next query
+//               tile is computed while the exponentials of this one run.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -97,6 +98,8 @@ struct Bars {
     // One barrier per buffer: S_{x+2} is issued only after S_x was consumed,
     // so neither runs two phases ahead of its waiter.
     __device__ __forceinline__ uint32_t s2_full() const { return base + 8 * (9 + 2 * slots); }
+    // dKV kernel: every elementwise warp has read S^T_i (S^T_{i+1} may overwrite it)
+    __device__ __forceinline__ uint32_t s_free() const { return base + 8 * (10 + 2 * slots); }
 };
 
 // delta_i = sum_d dO[i,d] O[i,d] (fp32), one warp per row.
@@ -121,9 +124,22 @@ __global__ void __launch_bounds__(256) delta_kernel(const __nv_bfloat16 *o, cons
     if (lane == 0) delta[row] = acc;
 }
 
-// Item enumeration shared by the roles of one CTA (round-robin over the grid).
-// dQ kernel: item = (qt, b, h), query tiles in descending order when causal
-// (longest key ranges first).  dKV kernel: item = (kt, b, g).
+// Item enumeration shared by the roles of one CTA.  Items are numbered in
+// roughly descending order of work -- dQ kernel: item = (qt, b, h), query tiles
+// in descending order when causal (longest key ranges first); dKV kernel:
+// item = (kt, b, g), key tiles ascending (when causal, later key tiles are
+// seen by fewer query tiles) -- and dealt in snake order: CTA c takes items
+// c, 2G-1-c, 2G+c, 4G-1-c, ... (G CTAs), so one round's largest items go
+// with the next round's smallest and the CTAs' totals even out.
+struct ItemIter {
+    int item, stride;
+    __device__ __forceinline__ ItemIter()
+        : item(static_cast<int>(blockIdx.x)), stride(2 * static_cast<int>(gridDim.x) - 1 - 2 * item) {}
+    __device__ __forceinline__ void next() {
+        item += stride;
+        stride = 2 * static_cast<int>(gridDim.x) - stride;
+    }
+};
 struct QItem {
     int b, h, qt, lo, hi;  // key tiles [lo, hi]
 };
@@ -195,6 +211,7 @@ __device__ __forceinline__ Setup<D> setup(const CUtensorMap *m0, const CUtensorM
         mbar_init(st.bar.dp_full(), 1);
         mbar_init(st.bar.pt_full(), kEwWarps);
         mbar_init(st.bar.s2_full(), 1);
+        mbar_init(st.bar.s_free(), kEwWarps);
         *st.abort_flag = 0;
         fence_barrier_init();
     }
@@ -258,6 +275,22 @@ __device__ __forceinline__ uint32_t kstep_off(int kk) {
     return static_cast<uint32_t>(((kk >> 2) * Cfg<D>::kColBlockBytes + (kk & 3) * 32) >> 4);
 }
 
+// dKV kernel ring: slots in pairs, step n (counted over the CTA's items) uses
+// pair n % kPairs and alternates which of the two holds Q and which dO, so
+// Q_n takes the slot dO_{n - kPairs} left.  dO is released after dV, a phase
+// before Q is released after dK, so Q (needed first: S^T_n is issued while
+// step n-1's elementwise work runs) lands a phase earlier than in a plain
+// ring.  Each slot is used once per kPairs steps: use index n / kPairs.
+template <int D>
+struct KvRing {
+    static constexpr uint32_t kPairs = Cfg<D>::kSlots / 2;
+    __device__ __forceinline__ static uint32_t q_slot(uint32_t n) { return 2 * (n % kPairs) + ((n / kPairs) & 1); }
+    __device__ __forceinline__ static uint32_t do_slot(uint32_t n) {
+        return 2 * (n % kPairs) + (((n / kPairs) & 1) ^ 1);
+    }
+    __device__ __forceinline__ static uint32_t use(uint32_t n) { return n / kPairs; }
+};
+
 // ------------------------------------------------------------------ dQ kernel
 template <int D, bool KM>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -266,6 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               const BwdParams p) {
     using C = Cfg<D>;
     const Setup<D> st = setup<D>(&tm_q, &tm_do, &tm_k, &tm_v);
+    // The dK/dV kernel reads none of this kernel's output: it may take over
+    // each SM as soon as this kernel's CTA there retires.
+    if (threadIdx.x == 0) grid_dep_launch();
     const Bars &bar = st.bar;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTileStep = C::kTileBytes >> 4;
@@ -274,8 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- producer: Q and dO once per item, then K_j, V_j per key tile
         if (lane == 0) {
             uint32_t prod = 0, fix_use = 0;
-            for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-                const QItem it = q_item(p, item);
+            for (ItemIter ii; ii.item < p.n_items; ii.next()) {
+                const QItem it = q_item(p, ii.item);
                 if (fix_use > 0 && !mbar_wait(bar.fix_empty(), (fix_use - 1) & 1, st.abort_flag, p.status))
                     break;
                 mbar_arrive_expect_tx(bar.fix_full(), 2 * C::kTileBytes);
@@ -311,8 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t d_ring = smem_desc_sw128(st.sbase + C::kRingOff, 16, 1024);
             const uint64_t d_ring_mn = smem_desc_sw128(st.sbase + C::kRingOff, C::kColBlockBytes, 1024);
             uint32_t cons = 0, fix_use = 0, op_cnt = 0, acc_use = 0;
-            for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-                const QItem it = q_item(p, item);
+            for (ItemIter ii; ii.item < p.n_items; ii.next()) {
+                const QItem it = q_item(p, ii.item);
                 if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
                 ++fix_use;
                 // S_j alternates between two buffers and runs two key tiles
@@ -401,8 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float c = p.scale_log2;
         uint32_t mm_cnt = 0, acc_cnt = 0;  // mm_cnt: dP tiles seen
         uint32_t s_even = 0, s_odd = 0;    // S tiles seen per buffer
-        for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-            const QItem it = q_item(p, item);
+        for (ItemIter ii; ii.item < p.n_items; ii.next()) {
+            const QItem it = q_item(p, ii.item);
             const int q0 = it.qt * kBlockQ;
             const int row = q0 + r;
             const bool valid = row < p.L;
@@ -506,10 +542,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kEwWarps) {
         // ---- producer: K and V once per item, then Q_i, dO_i per (head, query tile)
         if (lane == 0) {
-            uint32_t prod = 0, fix_use = 0;
+            using R = KvRing<D>;
+            uint32_t n = 0, fix_use = 0;
+            uint32_t used[C::kSlots];
+#pragma unroll
+            for (int s = 0; s < C::kSlots; ++s) used[s] = 0;
             bool stop = false;
-            for (int item = blockIdx.x; item < p.n_items && !stop; item += gridDim.x) {
-                const KItem it = k_item(p, item);
+            for (ItemIter ii; ii.item < p.n_items && !stop; ii.next()) {
+                const KItem it = k_item(p, ii.item);
                 if (it.steps == 0) continue;
                 if (fix_use > 0 && !mbar_wait(bar.fix_empty(), (fix_use - 1) & 1, st.abort_flag, p.status))
                     break;
@@ -518,23 +558,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 load_tile<D>(st.sbase + C::kFixOff + C::kTileBytes, &tm_v, bar.fix_full(), it.kt * kBlockK,
                              it.b * p.Hkv + it.g);
                 ++fix_use;
-                for (int step = 0; step < it.steps && !stop; ++step) {
+                for (int step = 0; step < it.steps && !stop; ++step, ++n) {
                     const int h = it.g * p.G + step / it.nq;
                     const int qt = it.qlo + step % it.nq;
-                    for (int which = 0; which < 2; ++which) {  // Q_i then dO_i
-                        const uint32_t s = prod % C::kSlots, round = prod / C::kSlots;
-                        if (round > 0 && !mbar_wait(bar.ring_empty(s), (round - 1) & 1, st.abort_flag, p.status)) {
+                    const uint32_t u = R::use(n);
+                    for (int which = 0; which < 2; ++which) {  // Q_n then dO_n
+                        const uint32_t s = which ? R::do_slot(n) : R::q_slot(n);
+                        if (u > 0 && !mbar_wait(bar.ring_empty(s), (u - 1) & 1, st.abort_flag, p.status)) {
                             stop = true;
                             break;
                         }
                         mbar_arrive_expect_tx(bar.ring_full(s), C::kTileBytes);
                         load_tile<D>(st.sbase + C::kRingOff + s * C::kTileBytes, which ? &tm_do : &tm_q,
                                      bar.ring_full(s), qt * kBlockQ, it.b * p.Hq + h);
-                        ++prod;
+                        ++used[s];
                     }
                 }
             }
-            drain_copies<D>(bar, prod, fix_use);
+            // every copy started must land before the CTA leaves
+            for (int s = 0; s < C::kSlots; ++s)
+                if (used[s] > 0) mbar_drain(bar.ring_full(s), (used[s] - 1) & 1);
+            if (fix_use > 0) mbar_drain(bar.fix_full(), (fix_use - 1) & 1);
         }
     } else if (warp == kEwWarps + 1) {
         // ---- MMA issuer
@@ -545,90 +589,84 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t d_v = d_k + kTileStep;
             const uint64_t d_ring = smem_desc_sw128(st.sbase + C::kRingOff, 16, 1024);
             const uint64_t d_ring_mn = smem_desc_sw128(st.sbase + C::kRingOff, C::kColBlockBytes, 1024);
-            uint32_t cons = 0, fix_use = 0, op_cnt = 0, acc_use = 0;
-            for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-                const KItem it = k_item(p, item);
+            using R = KvRing<D>;
+            uint32_t n = 0, fix_use = 0, sf_cnt = 0, op_cnt = 0, acc_use = 0;
+            for (ItemIter ii; ii.item < p.n_items; ii.next()) {
+                const KItem it = k_item(p, ii.item);
                 if (it.steps == 0) continue;
                 if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
                 ++fix_use;
-                // Two phases per step i: S^T_i and dP^T_i are in tensor memory;
-                // once P^T_i is written, dV += P^T_i dO_i and S^T_{i+1} (over S^T_i's
-                // columns, after dV read them); once dS^T_i is written, dK += dS^T_i
-                // Q_i and dP^T_{i+1}.  The elementwise warps compute P^T_{i+1} while
-                // the tensor core finishes step i.
-                uint32_t sq = cons % C::kSlots;
-                if (!mbar_wait(bar.ring_full(sq), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
-                ++cons;
-                uint32_t sd = cons % C::kSlots;
-                if (!mbar_wait(bar.ring_full(sd), (cons / C::kSlots) & 1, st.abort_flag, p.status)) goto mma_out;
-                ++cons;
+                // Per step i: S^T_{i+1} as soon as the elementwise warps have read
+                // S^T_i; dV += P^T_i dO_i once P^T_i is written; dK += dS^T_i Q_i
+                // once dS^T_i is written, then dP^T_{i+1}.  P^T_i and dS^T_i (bf16)
+                // lie over dP^T_i's columns (packed columns 0-31 / 64-95 and 32-63 /
+                // 96-127), so S^T's columns are free as soon as they are read and
+                // S^T_{i+1} overlaps the exponentials of step i.
+                auto take = [&](uint32_t slot, uint32_t m) -> bool {
+                    return mbar_wait(bar.ring_full(slot), R::use(m) & 1, st.abort_flag, p.status);
+                };
+                auto issue_st = [&](uint32_t m) {  // S^T = K Q_m^T
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk),
+                                d_ring + R::q_slot(m) * kTileStep + kstep_off<D>(kk), kIdescS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar.mm_full());
+                };
+                auto issue_dpt = [&](uint32_t m) {  // dP^T = V dO_m^T
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk),
+                                d_ring + R::do_slot(m) * kTileStep + kstep_off<D>(kk), kIdescS, kk > 0 ? 1u : 0u);
+                    umma_commit(bar.dp_full());
+                };
+                if (!take(R::q_slot(n), n) || !take(R::do_slot(n), n)) goto mma_out;
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk), d_ring + sq * kTileStep + kstep_off<D>(kk),
-                            kIdescS, kk > 0 ? 1u : 0u);
-                umma_commit(bar.mm_full());
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk), d_ring + sd * kTileStep + kstep_off<D>(kk),
-                            kIdescS, kk > 0 ? 1u : 0u);
-                umma_commit(bar.dp_full());
+                issue_st(n);
+                issue_dpt(n);
                 if (it.steps == 1) umma_commit(bar.fix_empty());
                 for (int step = 0; step < it.steps; ++step) {
+                    const uint32_t cur = n + step;
                     const bool more = step + 1 < it.steps;
+                    if (more) {
+                        if (!mbar_wait(bar.s_free(), sf_cnt & 1, st.abort_flag, p.status)) goto mma_out;
+                        ++sf_cnt;
+                        if (!take(R::q_slot(cur + 1), cur + 1)) goto mma_out;
+                        tc_fence_after();
+                        issue_st(cur + 1);
+                    }
                     // the previous item's dK, dV must have been read before they restart
                     if (step == 0 && acc_use > 0 &&
                         !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
                         goto mma_out;
-                    // dV += P^T dO (P^T over S^T columns 0-31 and 64-95)
+                    // dV += P^T dO
                     if (!mbar_wait(bar.pt_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBlockQ / 16; ++kk)
-                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemA + packed_col(kk),
-                                d_ring_mn + sd * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
+                        umma_ts(st.tmem + C::kTmemC, st.tmem + C::kTmemB + packed_col(kk),
+                                d_ring_mn + R::do_slot(cur) * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(bar.ring_empty(sd));  // dO_i's last use
-                    uint32_t nq = 0, nd = 0;
-                    if (more) {
-                        nq = cons % C::kSlots;
-                        if (!mbar_wait(bar.ring_full(nq), (cons / C::kSlots) & 1, st.abort_flag, p.status))
-                            goto mma_out;
-                        ++cons;
-                        nd = cons % C::kSlots;
-                        if (!mbar_wait(bar.ring_full(nd), (cons / C::kSlots) & 1, st.abort_flag, p.status))
-                            goto mma_out;
-                        ++cons;
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            umma_ss(st.tmem + C::kTmemA, d_k + kstep_off<D>(kk),
-                                    d_ring + nq * kTileStep + kstep_off<D>(kk), kIdescS, kk > 0 ? 1u : 0u);
-                        umma_commit(bar.mm_full());
-                    }
-                    // dK += dS^T Q (dS^T over dP^T columns 0-31 and 64-95)
+                    umma_commit(bar.ring_empty(R::do_slot(cur)));  // dO_i's last use
+                    // dK += dS^T Q
                     if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
                     ++op_cnt;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBlockQ / 16; ++kk)
-                        umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + packed_col(kk),
-                                d_ring_mn + sq * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
+                        umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + 32 + packed_col(kk),
+                                d_ring_mn + R::q_slot(cur) * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(bar.ring_empty(sq));  // Q_i's last use
-                    if (more) {
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            umma_ss(st.tmem + C::kTmemB, d_v + kstep_off<D>(kk),
-                                    d_ring + nd * kTileStep + kstep_off<D>(kk), kIdescS, kk > 0 ? 1u : 0u);
-                        umma_commit(bar.dp_full());
+                    umma_commit(bar.ring_empty(R::q_slot(cur)));  // Q_i's last use
+                    if (more) {  // dP^T_{i+1} over the columns dV, dK have just read
+                        if (!take(R::do_slot(cur + 1), cur + 1)) goto mma_out;
+                        tc_fence_after();
+                        issue_dpt(cur + 1);
                         if (step + 2 == it.steps) umma_commit(bar.fix_empty());  // K, V's last use
-                        sq = nq;
-                        sd = nd;
                     }
                 }
                 umma_commit(bar.acc_full());
                 ++acc_use;
+                n += it.steps;
             }
         mma_out:
             umma_commit(bar.done());
@@ -647,8 +685,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int P = p.S - p.L;
         float *stage = reinterpret_cast<float *>(st.gbase + C::kStageOff) + warp * 256;
         uint32_t mm_cnt = 0, acc_cnt = 0;
-        for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
-            const KItem it = k_item(p, item);
+        for (ItemIter ii; ii.item < p.n_items; ii.next()) {
+            const KItem it = k_item(p, ii.item);
             const int key = it.kt * kBlockK + r;
             const bool kvalid = key < p.S;
             const bool kept = kvalid && (!KM || __ldg(p.key_mask + static_cast<size_t>(it.b) * p.S + key) > 0.5f);
@@ -668,67 +706,91 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 continue;
             }
-            for (int step = 0; step < it.steps; ++step) {
+            // -lse and delta of the warp's 64 query columns of step i (lane e:
+            // columns 32 c2 + e of its half), fetched one step ahead into
+            // registers, written to the warp's stage at the step's start and
+            // read back as shared-memory broadcasts
+            float nxt[4];
+            auto fetch = [&](int step) {
                 const int h = it.g * p.G + step / it.nq;
                 const int q0 = (it.qlo + step % it.nq) * kBlockQ;
                 const float *lse_h = p.lse + static_cast<size_t>(it.b * p.Hq + h) * p.L;
                 const float *dl_h = p.delta + static_cast<size_t>(it.b * p.Hq + h) * p.L;
-                // -lse and delta of the warp's 64 query columns, loaded once per
-                // warp (lane e: columns 32 ch + e) into the warp's stage and
-                // read back as shared-memory broadcasts
+#pragma unroll
+                for (int c2 = 0; c2 < 2; ++c2) {
+                    const int q = q0 + 64 * hf + 32 * c2 + lane;
+                    nxt[2 * c2] = q < p.L ? -__ldg(lse_h + q) : -CUDART_INF_F;
+                    nxt[2 * c2 + 1] = q < p.L ? __ldg(dl_h + q) : 0.f;
+                }
+            };
+            fetch(0);
+            for (int step = 0; step < it.steps; ++step) {
+                const bool more = step + 1 < it.steps;
+                const int q0 = (it.qlo + step % it.nq) * kBlockQ + 64 * hf;  // the warp's first query column
                 __syncwarp();  // every lane is done with the previous step's stage
 #pragma unroll
                 for (int c2 = 0; c2 < 2; ++c2) {
-                    const int ch = 2 * hf + c2;
-                    const int q = q0 + 32 * ch + lane;
-                    stage[32 * ch + lane] = q < p.L ? -__ldg(lse_h + q) : -CUDART_INF_F;
-                    stage[128 + 32 * ch + lane] = q < p.L ? __ldg(dl_h + q) : 0.f;
+                    stage[64 * hf + 32 * c2 + lane] = nxt[2 * c2];
+                    stage[128 + 64 * hf + 32 * c2 + lane] = nxt[2 * c2 + 1];
                 }
                 __syncwarp();
-                // phase 1: P^T = 2^(S^T c - lse) from S^T (kept in fp32 for dS^T)
+                // S^T_i: read it, then free its columns for S^T_{i+1}
                 if (!__all_sync(0xffffffffu, mbar_wait(bar.mm_full(), mm_cnt & 1, st.abort_flag, p.status)))
                     goto ew_out;
                 tc_fence_after();
+                uint32_t sv[64];
+                tmem_ld64(tA + 64 * hf, sv);
+                if (more) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar.s_free());
+                    fetch(step + 1);
+                }
+                // P^T = 2^(S^T c - lse), kept in fp32 for dS^T
                 float pt[64];
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    const int ch = 2 * hf + c2;
-                    uint32_t sv[32], wp[16];
-                    tmem_ld32(tA + 32 * ch, sv);
-                    const int qc = q0 + 32 * ch;
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const bool allowed = (qc + e >= q_lo) & (qc + e <= q_hi);
-                        const float ev = ex2(fmaf(__uint_as_float(sv[e]), c, stage[32 * ch + e]));
-                        pt[32 * c2 + e] = allowed ? ev : 0.f;
-                    }
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) wp[e] = pack_bf16(pt[32 * c2 + 2 * e], pt[32 * c2 + 2 * e + 1]);
-                    tmem_st16(tA + 64 * hf + 16 * c2, wp);  // over S^T columns this warp has read
+                for (int e = 0; e < 64; ++e) {
+                    const bool allowed = (q0 + e >= q_lo) & (q0 + e <= q_hi);
+                    const float ev = ex2(fmaf(__uint_as_float(sv[e]), c, stage[64 * hf + e]));
+                    pt[e] = allowed ? ev : 0.f;
                 }
-                tmem_wait_st();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar.pt_full());
-                // phase 2: dS^T = P^T (dP^T - delta) from dP^T
+                // dP^T_i: its first 32 columns of the half, then P^T (bf16) over them
                 if (!__all_sync(0xffffffffu, mbar_wait(bar.dp_full(), mm_cnt & 1, st.abort_flag, p.status)))
                     goto ew_out;
                 ++mm_cnt;
                 tc_fence_after();
+                uint32_t wd[32];
+                {
+                    uint32_t dv[32];
+                    tmem_ld32(tB + 64 * hf, dv);
 #pragma unroll
-                for (int c2 = 0; c2 < 2; ++c2) {
-                    const int ch = 2 * hf + c2;
-                    uint32_t dv[32], wd[16];
-                    tmem_ld32(tB + 32 * ch, dv);
+                    for (int c2 = 0; c2 < 2; ++c2) {
+                        uint32_t wp[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float d0 = pt[32 * c2 + 2 * e] * (__uint_as_float(dv[2 * e]) - stage[128 + 32 * ch + 2 * e]);
-                        const float d1 =
-                            pt[32 * c2 + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - stage[128 + 32 * ch + 2 * e + 1]);
-                        wd[e] = pack_bf16(d0, d1);
+                        for (int e = 0; e < 16; ++e) wp[e] = pack_bf16(pt[32 * c2 + 2 * e], pt[32 * c2 + 2 * e + 1]);
+                        tmem_st16(tB + 64 * hf + 16 * c2, wp);
                     }
-                    tmem_st16(tB + 64 * hf + 16 * c2, wd);  // over dP^T columns this warp has read
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar.pt_full());
+                    // dS^T = P^T (dP^T - delta)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        wd[e] = pack_bf16(pt[2 * e] * (__uint_as_float(dv[2 * e]) - stage[128 + 64 * hf + 2 * e]),
+                                          pt[2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - stage[128 + 64 * hf + 2 * e + 1]));
                 }
+                {
+                    uint32_t dv[32];
+                    tmem_ld32(tB + 64 * hf + 32, dv);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        wd[16 + e] = pack_bf16(
+                            pt[32 + 2 * e] * (__uint_as_float(dv[2 * e]) - stage[128 + 64 * hf + 32 + 2 * e]),
+                            pt[32 + 2 * e + 1] * (__uint_as_float(dv[2 * e + 1]) - stage[128 + 64 * hf + 32 + 2 * e + 1]));
+                }
+                // dS^T (bf16) over the half's last 32 columns, read just above
+                tmem_st32(tB + 64 * hf + 32, wd);
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
@@ -765,6 +827,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     ew_out:;
     }
     teardown<D>(st);
+    // Started while the dQ kernel may still run: complete only after it, so
+    // that the backward's end on the stream covers dQ as well.
+    if (threadIdx.x == 0) grid_dep_wait();
 }
 
 }  // namespace bwd

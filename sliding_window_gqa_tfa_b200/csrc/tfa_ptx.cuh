@@ -79,6 +79,16 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
     }
 }
 
+// ------------------------------------------------- programmatic launch
+// Let the grid launched after this one (with programmatic stream
+// serialisation) start its CTAs as this grid's CTAs retire.
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the grids this one depends on have completed and their memory
+// is visible (returns at once when there are none).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -165,6 +175,21 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
         "tcgen05.wait::ld.sync.aligned;"
         : TFA_R8(r, 0)
         : "r"(taddr)
+        : "memory");
+}
+// 32 lanes x 64 columns: two x32 loads issued back to back, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%65];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : TFA_R8(r, 0), TFA_R8(r, 8), TFA_R8(r, 16), TFA_R8(r, 24),
+          TFA_R8(r, 32), TFA_R8(r, 40), TFA_R8(r, 48), TFA_R8(r, 56)
+        : "r"(taddr), "r"(taddr + 32)
         : "memory");
 }
 // 32 lanes x 128 columns: four x32 loads issued back to back, one wait.
