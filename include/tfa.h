@@ -246,8 +246,9 @@ int tfa_prefill_backward_saved(const void *q, const void *k, const void *v, cons
 #define TFA_DEBUG_NO_TILE_SKIP  1u /* visit every key tile, even fully masked ones   */
 #define TFA_DEBUG_MASK_ALL      2u /* apply the mask predicate on interior tiles too */
 #define TFA_DEBUG_SYNC          4u /* synchronize the stream and return the device status */
-#define TFA_DEBUG_NO_SPLIT      8u /* deal whole work items round-robin instead of splitting
-                                      key ranges evenly across the CTAs (no partial merges) */
+#define TFA_DEBUG_NO_SPLIT      8u /* deal whole work items (snake order, longest first) instead
+                                      of splitting key ranges evenly across the CTAs (no partial
+                                      merges) */
 #define TFA_DEBUG_FORCE_SPLIT  16u /* always split key ranges evenly across the CTAs (by
                                       default the library picks the schedule it estimates
                                       finishes first) */
@@ -341,7 +342,8 @@ int tfa_plan_ktile(int L, int S, int causal, int window, int ktile, int *qt_lo, 
  * (tfa_prefill's schedule) the concatenated key-tile steps of all such items
  * are cut into `grid` contiguous ranges of almost equal length; a cut item is
  * finished by the piece holding a tile's first key tile, which merges the
- * others' partial softmax statistics.  With split == 0 items go round-robin.
+ * others' partial softmax statistics.  With split == 0 whole items are dealt
+ * in snake order: CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G = grid).
  *   out          10 ints per piece: item, qp, b, h, first key tile, last key
  *                tile, role of tile 0, role of tile 1 (bit 0 active, bit 1
  *                finalizer, bit 2 complete), and for a finalizer that must

@@ -90,6 +90,12 @@ def test_whole_item_schedule_deals_each_item_once(case):
         for p in pieces:
             assert p[6] & 4 and (p[7] & 4 or not p[7] & 1)
         seen += [p[0] for p in pieces]
+        # snake order: c, 2G-1-c, 2G+c, 4G-1-c, ... (each round reverses the last)
+        want, item, stride = [], c, 2 * grid - 1 - 2 * c
+        while item < n_items:
+            want.append(item)
+            item, stride = item + stride, 2 * grid - stride
+        assert [p[0] for p in pieces] == want
     assert sorted(seen) == list(range(n_items))
 
 
