@@ -15,9 +15,9 @@
 //
 // Two kernels share the forward's machinery (TMA tiles with 128-byte swizzle,
 // tcgen05 MMAs with fp32 accumulators in tensor memory, one thread per
-// 128-lane row for the elementwise work), each with 192 threads: warps 0-3 do
-// the elementwise work and the epilogue, warp 4 is the TMA producer, warp 5
-// issues the MMAs.
+// 128-lane row), each with 320 threads: warps 0-7 do the elementwise work and
+// the epilogue (two per SM sub-partition, each on half a tile's columns), warp
+// 8 is the TMA producer, warp 9 issues the MMAs.
 //   dQ kernel:  work item (b, h, 128-row query tile), walking the key tiles
 //               the tile sees: S = Q K^T and dP = dO V^T into tensor memory,
 //               dS (bf16) written over dP, then dQ += dS K.

@@ -19,8 +19,8 @@
 // piece of a later CTA's range, so partials are produced early, and a
 // finalizer only ever waits for CTAs after its own: no cycle is possible.
 //
-// Whole-item schedule (debug flag, and the no-allocation entry point): items
-// are dealt round-robin to the CTAs; nothing is split and nothing is merged.
+// Whole-item schedule (when the estimate favours it, varlen, no-allocation
+// entry, debug flag): items go out in snake order; nothing is split or merged.
 #pragma once
 
 #include "tfa_plan.h"
@@ -39,7 +39,7 @@ struct Shape {
     unsigned flags;
     int n_qp;   // query-tile pairs per head: ceil(L / 256)
     int grid;   // CTAs
-    int split;  // 1: split schedule; 0: whole items round-robin
+    int split;  // 1: split schedule; 0: whole items in snake order
 };
 
 TFA_HD int shape_n_qp(int L) { return (L + 2 * kBlockQ - 1) / (2 * kBlockQ); }
