@@ -212,7 +212,12 @@ int tfa_prefill_varlen(const void *q, const void *k, const void *v, void *o,
  * dk = scale dS^T Q, dv = P^T dout.  The call re-runs the forward (its output
  * and per-row log-sum-exp go to a per-stream workspace of 2 B Hq L (D + 4)
  * bytes, grown on demand; growth during graph capture returns
- * TFA_ERR_CAPTURE), then three kernels, all asynchronous on `stream`. */
+ * TFA_ERR_CAPTURE), then three kernels, all asynchronous on `stream`: a
+ * delta kernel, the dQ kernel, and the dK/dV kernel, launched with
+ * programmatic stream serialisation so that its CTAs start on the SMs the dQ
+ * kernel's CTAs leave (it reads nothing dQ writes).  The dK/dV kernel does
+ * not complete before the dQ kernel has, so work queued on `stream` after
+ * the call sees all three gradients. */
 int tfa_prefill_backward(const void *q, const void *k, const void *v, const void *dout,
                          void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int L, int S,
                          int D, float scale, int causal, int window, const float *key_mask,
