@@ -282,7 +282,7 @@ __device__ __forceinline__ uint32_t kstep_off(int kk) {
 // step n-1's elementwise work runs) lands a phase earlier than in a plain
 // ring.  Each slot is used once per kPairs steps: use index n / kPairs.
 template <int D>
-struct KvRing {
+struct KvRing {  // dQ kernel: q_slot holds K_t, do_slot V_t
     static constexpr uint32_t kPairs = Cfg<D>::kSlots / 2;
     __device__ __forceinline__ static uint32_t q_slot(uint32_t n) { return 2 * (n % kPairs) + ((n / kPairs) & 1); }
     __device__ __forceinline__ static uint32_t do_slot(uint32_t n) {
@@ -309,7 +309,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kEwWarps) {
         // ---- producer: Q and dO once per item, then K_j, V_j per key tile
         if (lane == 0) {
-            uint32_t prod = 0, fix_use = 0;
+            using R = KvRing<D>;
+            uint32_t t = 0, fix_use = 0;
+            uint32_t used[C::kSlots];
+#pragma unroll
+            for (int s = 0; s < C::kSlots; ++s) used[s] = 0;
             for (ItemIter ii; ii.item < p.n_items; ii.next()) {
                 const QItem it = q_item(p, ii.item);
                 if (fix_use > 0 && !mbar_wait(bar.fix_empty(), (fix_use - 1) & 1, st.abort_flag, p.status))
@@ -320,22 +324,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                              it.b * p.Hq + it.h);
                 ++fix_use;
                 bool stop = false;
-                for (int j = it.lo; j <= it.hi && !stop; ++j) {
-                    for (int which = 0; which < 2; ++which) {
-                        const uint32_t s = prod % C::kSlots, round = prod / C::kSlots;
-                        if (round > 0 && !mbar_wait(bar.ring_empty(s), (round - 1) & 1, st.abort_flag, p.status)) {
+                for (int j = it.lo; j <= it.hi && !stop; ++j, ++t) {
+                    const uint32_t u = R::use(t);
+                    for (int which = 0; which < 2; ++which) {  // K_t then V_t
+                        const uint32_t s = which ? R::do_slot(t) : R::q_slot(t);
+                        if (u > 0 && !mbar_wait(bar.ring_empty(s), (u - 1) & 1, st.abort_flag, p.status)) {
                             stop = true;
                             break;
                         }
                         mbar_arrive_expect_tx(bar.ring_full(s), C::kTileBytes);
                         load_tile<D>(st.sbase + C::kRingOff + s * C::kTileBytes, which ? &tm_v : &tm_k,
                                      bar.ring_full(s), j * kBlockK, it.b * p.Hkv + it.h / p.G);
-                        ++prod;
+                        ++used[s];
                     }
                 }
                 if (stop) break;
             }
-            drain_copies<D>(bar, prod, fix_use);
+            for (int s = 0; s < C::kSlots; ++s)
+                if (used[s] > 0) mbar_drain(bar.ring_full(s), (used[s] - 1) & 1);
+            if (fix_use > 0) mbar_drain(bar.fix_full(), (fix_use - 1) & 1);
         }
     } else if (warp == kEwWarps + 1) {
         // ---- MMA issuer
@@ -346,7 +353,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t d_do = d_q + kTileStep;
             const uint64_t d_ring = smem_desc_sw128(st.sbase + C::kRingOff, 16, 1024);
             const uint64_t d_ring_mn = smem_desc_sw128(st.sbase + C::kRingOff, C::kColBlockBytes, 1024);
-            uint32_t cons = 0, fix_use = 0, op_cnt = 0, acc_use = 0;
+            using R = KvRing<D>;
+            uint32_t tb = 0, fix_use = 0, op_cnt = 0, acc_use = 0;
             for (ItemIter ii; ii.item < p.n_items; ii.next()) {
                 const QItem it = q_item(p, ii.item);
                 if (!mbar_wait(bar.fix_full(), fix_use & 1, st.abort_flag, p.status)) goto mma_out;
@@ -356,11 +364,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // columns).  The elementwise warps compute P_{j+1} from S_{j+1} while
                 // the tensor core finishes step j.
                 const int n = it.hi - it.lo + 1;
-                auto take = [&](uint32_t &slot) -> bool {
-                    slot = cons % C::kSlots;
-                    if (!mbar_wait(bar.ring_full(slot), (cons / C::kSlots) & 1, st.abort_flag, p.status)) return false;
-                    ++cons;
-                    return true;
+                // K_t and V_t of the CTA's t-th key tile (counted over its items)
+                auto take = [&](uint32_t &slot, uint32_t t, int which) -> bool {
+                    slot = which ? R::do_slot(t) : R::q_slot(t);
+                    return mbar_wait(bar.ring_full(slot), R::use(t) & 1, st.abort_flag, p.status);
                 };
                 auto issue_s = [&](int x, uint32_t ks) {
                     const uint32_t dst = st.tmem + ((x & 1) ? C::kTmemA2 : C::kTmemA);
@@ -379,12 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_commit(bar.ring_empty(vs));  // V's only use
                 };
                 uint32_t k_cur = 0, k_nxt = 0, v_nxt = 0, v0 = 0;
-                if (!take(k_cur) || !take(v0)) goto mma_out;
+                if (!take(k_cur, tb, 0) || !take(v0, tb, 1)) goto mma_out;
                 tc_fence_after();
                 issue_s(0, k_cur);
                 issue_dp(v0);
                 if (n > 1) {
-                    if (!take(k_nxt) || !take(v_nxt)) goto mma_out;
+                    if (!take(k_nxt, tb + 1, 0) || !take(v_nxt, tb + 1, 1)) goto mma_out;
                     tc_fence_after();
                     issue_s(1, k_nxt);
                 }
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint32_t k_nn = 0, v_nn = 0;
                     if (x + 2 < n) {
-                        if (!take(k_nn) || !take(v_nn)) goto mma_out;
+                        if (!take(k_nn, tb + x + 2, 0) || !take(v_nn, tb + x + 2, 1)) goto mma_out;
                         tc_fence_after();
                         issue_s(x + 2, k_nn);
                     }
@@ -420,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 umma_commit(bar.acc_full());
                 ++acc_use;
+                tb += static_cast<uint32_t>(n);
             }
         mma_out:
             umma_commit(bar.done());
@@ -638,8 +646,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (step == 0 && acc_use > 0 &&
                         !mbar_wait(bar.acc_empty(), (acc_use - 1) & 1, st.abort_flag, p.status))
                         goto mma_out;
-                    // dV += P^T dO
-                    if (!mbar_wait(bar.pt_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
+                    // dV += P^T dO, dK += dS^T Q and dP^T_{i+1} as one run of MMAs once
+                    // both operands are written: every wait of the issuer between
+                    // MMA blocks lets the tensor pipe drain
+                    if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
+                    ++op_cnt;
                     tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBlockQ / 16; ++kk)
@@ -647,10 +658,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 d_ring_mn + R::do_slot(cur) * kTileStep + kk * ((16 * 128) >> 4), kIdescAcc,
                                 (step > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(bar.ring_empty(R::do_slot(cur)));  // dO_i's last use
-                    // dK += dS^T Q
-                    if (!mbar_wait(bar.op_full(), op_cnt & 1, st.abort_flag, p.status)) goto mma_out;
-                    ++op_cnt;
-                    tc_fence_after();
 #pragma unroll
                     for (int kk = 0; kk < kBlockQ / 16; ++kk)
                         umma_ts(st.tmem + C::kTmemD, st.tmem + C::kTmemB + 32 + packed_col(kk),
@@ -770,10 +777,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 16; ++e) wp[e] = pack_bf16(pt[32 * c2 + 2 * e], pt[32 * c2 + 2 * e + 1]);
                         tmem_st16(tB + 64 * hf + 16 * c2, wp);
                     }
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar.pt_full());
                     // dS^T = P^T (dP^T - delta)
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
