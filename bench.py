@@ -11,16 +11,21 @@ the timed region; L2 is flushed (256 MiB memset) between steps, outside each
 step's CUDA events.  Prints one JSON line on rank 0.
 
 Metric: TFLOP/s over allowed (unmasked) pairs, 4*D flops per pair per head.
-With --gpus N > 1 (launched by torch.distributed.run) every rank runs the same
-workload on its own inputs (weak scaling, no data-path collective); the
-reported time is the max over ranks.
+With --gpus N > 1 (launched by torch.distributed.run) the (batch, KV group)
+units of one call are shared by the ranks (sliding_window_gqa_tfa_b200.dist):
+--shard weak (default) makes the call N times the workload's batch, so each
+rank's share is one copy of the workload on its own inputs; --shard strong
+shares the workload's own units.  No data-path collective; the reported time
+is the max over ranks.  At N = 1 the line also carries `per_config`: each of
+the reference configurations timed the same way, with its max-abs / max-rel
+error against the fp64 oracle on the sampled rows the full-size parity test
+checks.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
-import math
 import os
 import re
 import statistics
@@ -35,11 +40,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sliding_window_gqa_tfa_b200 import binding as tb  # noqa: E402
-from sliding_window_gqa_tfa_b200.dist import (barrier, max_over_ranks, setup,  # noqa: E402
-                                              teardown, weak_scaling_rate)
+from sliding_window_gqa_tfa_b200.dist import (barrier, max_over_ranks, rank_runs,  # noqa: E402
+                                              run_slices, setup, teardown)
 from sliding_window_gqa_tfa_b200.flops import workload_bytes, workload_flops  # noqa: E402
 from sliding_window_gqa_tfa_b200.inputs import (HEADLINE, WORKLOADS, make_dout,  # noqa: E402
-                                                make_inputs, make_sinks, varlen_cu)
+                                                make_inputs, make_sinks, sample_rows, varlen_cu)
 
 METRIC = "prefill attention TFLOP/s (unmasked pairs) and % of B200 BF16 tensor peak"
 UNIT = "TFLOP/s"
@@ -81,57 +86,107 @@ def recorded_traffic(workload: str):
     return int(m_bytes.group(1))
 
 
-class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+_NVML_POLLER = """
+import signal, sys, time, pynvml
+stop = []
+signal.signal(signal.SIGTERM, lambda *a: stop.append(1))
+pynvml.nvmlInit()
+key = sys.argv[1]
+h = (pynvml.nvmlDeviceGetHandleByUUID(key) if key.startswith("GPU-")
+     else pynvml.nvmlDeviceGetHandleByIndex(int(key)))
+get = (getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+       or pynvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=True)
+out = []
+t_end = time.time() + 600
+while not stop and time.time() < t_end:
+    out.append("%d %d" % (pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get(h))))
+    time.sleep(0.0005)
+print(chr(10).join(out), flush=True)
+"""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+
+class ClockSampler:
+    """SM clock and throttle reasons sampled during the timed region: NVML
+    polled every ~0.5 ms by a child process (so even a region of a few
+    milliseconds gets samples, whatever the launching thread does), else
+    nvidia-smi at its fastest interval.  Read-only."""
+
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
+        self.source = None
+        self.samples = []  # (sm MHz, reason bits)
+        self.smax = None
+
+    def _device_key(self):
+        try:  # the same GPU as torch's device, whatever CUDA_VISIBLE_DEVICES says
+            uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+            return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            return str(self.idx)
 
     def __enter__(self):
         try:
+            self.proc = subprocess.Popen([sys.executable, "-c", _NVML_POLLER, self._device_key()],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            first = self.proc.stdout.readline().split()  # "max <MHz>": the poller is running
+            if len(first) == 2 and first[0] == "max":
+                self.smax = float(first[1])
+                self.source = "nvml"
+                return self
+            self.proc.kill()
+            self.proc.communicate()
+        except OSError:
+            pass
+        try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", str(self.idx),
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
                  "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
         except OSError:
             self.proc = None
         time.sleep(0.3)
         return self
 
     def __exit__(self, *exc):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
+        if self.proc is None:
+            return
+        time.sleep(0.002)  # a last sample after the region
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in (out or "").splitlines():
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                self.out, _ = self.proc.communicate()
+                if self.source == "nvml":
+                    mhz, bits = line.split()
+                    self.samples.append((float(mhz), int(bits)))
+                else:
+                    parts = [p.strip() for p in line.split(",")]
+                    self.samples.append((float(parts[0]), int(parts[2], 16)))
+                    self.smax = float(parts[1])
+            except (ValueError, IndexError):
+                continue
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in (self.out or "").splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        load = [(mhz, r) for mhz, r in self.samples if not (r & 0x1)]  # not GPU-idle
+        use = load or self.samples
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": self.smax, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = sorted({n for _, r in use for bit, n in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in use), "sm_max_mhz": self.smax,
+                "reasons": reasons, "samples": len(self.samples), "samples_under_load": len(load),
+                "source": self.source}
 
 
 def cpu_threads():
@@ -270,6 +325,91 @@ def run_reference(args, w):
     return 0
 
 
+# The reference configurations timed beside the headline at N = 1 (the workload
+# the metric is quoted on is the headline line itself; its error is reported too).
+PER_CONFIG = ["witness_33x47", "qwen3_prefill_b4_2048", HEADLINE, "llama_gqa_chunk_2048x8192_keymask",
+              "swa_rotating_w1024_2048", "long_chunk_2048x32768", "long_chunk_2048x32768_d64",
+              "bidirectional_4096"]
+
+
+def oracle_errors(w, o, q, k, v, km):
+    """Max-abs / max-rel error of the bf16 output o (on the device) against the
+    fp64 oracle on the rows the full-size parity test samples (every row of a
+    tiny workload), and the worst ratio of the error to the tolerance
+    0.02 + 0.02 |ref| (<= 1 passes).  Relative error over |ref| >= 0.05."""
+    import oracle
+
+    oracle.build()
+    tiny = w.B * w.Hq * w.L <= 4096
+    rows = None if tiny else sample_rows(w, n_per_head=12 if w.S >= 16384 else 24)
+    ref = oracle.attention(q, k, v, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                           key_mask=km, softcap=w.softcap, sinks=make_sinks(w, 0), rows=rows)
+    got = o.reshape(-1, w.D) if rows is not None else o
+    if rows is not None:
+        got = got[torch.as_tensor(rows, device=o.device)]
+    got = got.float().cpu().double().numpy().reshape(ref.shape)
+    err = np.abs(got - ref)
+    big = np.abs(ref) >= 0.05
+    return {"max_abs_err": float(err.max()),
+            "max_rel_err": float((err[big] / np.abs(ref[big])).max()) if big.any() else 0.0,
+            "worst_tol_ratio": float((err / (0.02 + 0.02 * np.abs(ref))).max()),
+            "rows_checked": int(ref.reshape(-1, w.D).shape[0])}
+
+
+def time_launches(step, flush, stream, steps, warmup, dev, world=1):
+    """Per-launch device times (ms) of `steps` launches after `warmup`, L2 flushed
+    before each, CUDA events on the launching stream; clocks sampled meanwhile."""
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    tb.check_status(stream)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_wall = time.perf_counter()
+        for i in range(steps):
+            flush.zero_()
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    tb.check_status(stream)
+    return [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)], clk.summary(), t_wall
+
+
+def per_config(args, dev, flush, stream, peaks):
+    """Each reference configuration: device time (as the headline), throughput,
+    fraction of the measured peak, clocks, and error against the fp64 oracle."""
+    res = {}
+    for name in PER_CONFIG:
+        w = WORKLOADS[name]
+        q, k, v, km = make_inputs(w, seed=0)
+        dq, dk, dv = q.to(dev), k.to(dev), v.to(dev)
+        dkm = km.to(dev) if km is not None else None
+        o = torch.empty_like(dq)
+
+        def step():
+            tb.prefill(dq, dk, dv, scale=w.softmax_scale, causal=w.causal, window=w.window,
+                       key_mask=dkm, out=o)
+
+        per, clocks, _ = time_launches(step, flush, stream, args.steps, args.warmup, dev)
+        per = sorted(per)
+        mean = sum(per) / len(per)
+        fl = workload_flops(w, key_mask=km)
+        tflops = fl / (mean * 1e-3) / 1e12
+        res[name] = {"ms_mean": mean, "ms_p50": per[len(per) // 2], "tflops": tflops,
+                     "frac": tflops / float(peaks["bf16_tflops"]), "useful_gflop": fl / 1e9,
+                     "clock_sm_mhz": clocks["sm_mhz"], "clock_reasons": clocks["reasons"],
+                     **oracle_errors(w, o, q, k, v, km)}
+        del dq, dk, dv, dkm, o
+        torch.cuda.empty_cache()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -277,7 +417,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="tfa", choices=["tfa", "reference"])
+    ap.add_argument("--shard", default="weak", choices=["weak", "strong"],
+                    help="N > 1: one call N times the workload's batch (weak) or the workload "
+                         "itself (strong), its (batch, KV group) units shared by the ranks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
@@ -291,8 +435,12 @@ def main():
     dev = torch.device("cuda", local)
     tb.lib()  # fail loudly if the library is missing
 
-    q, k, v, km = make_inputs(w, seed=rank)
-    sinks = make_sinks(w, seed=rank)
+    # Dense workloads at N > 1 run this rank's share of one call's (batch, KV
+    # group) units; the other kinds run one copy of the workload per rank.
+    strong = world > 1 and args.shard == "strong" and w.kind == "dense"
+    seed = 0 if strong else rank  # a strong-scaling call's inputs are the same on every rank
+    q, k, v, km = make_inputs(w, seed=seed)
+    sinks = make_sinks(w, seed=seed)
     if w.kind == "varlen":
         extra = tuple(torch.from_numpy(c) for c in varlen_cu(w))
     elif w.kind == "backward":
@@ -311,12 +459,26 @@ def main():
         out = tuple(torch.empty_like(t) for t in dev_inputs[:3])
     else:
         out = torch.empty_like(dev_inputs[0])
-    flops = workload_flops(w, key_mask=km)
+    G = w.Hq // w.Hkv
+    if w.kind == "dense":
+        if strong:  # this rank's units of the workload's own call
+            runs = rank_runs(w.B, w.Hkv, world, rank)
+        else:  # a call of world x B elements: this rank's units are its own B elements
+            runs = [r_.__class__(r_.b0 - rank * w.B, r_.nb, r_.g0, r_.ng)
+                    for r_ in rank_runs(world * w.B, w.Hkv, world, rank)]
+        flops = sum(workload_flops(w.with_(B=r_.nb, Hq=r_.ng * G, Hkv=r_.ng),
+                                   key_mask=km[r_.b0:r_.b0 + r_.nb] if km is not None else None)
+                    for r_ in runs)
+    else:
+        runs = None
+        flops = workload_flops(w, key_mask=km)
+    call_flops = workload_flops(w, key_mask=km)  # one copy of the workload
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def call(ins, o):
-        """One launch on the current stream: the entry point the workload needs."""
+        """One step on the current stream: the entry point the workload needs
+        (for a dense workload, one call per run of this rank's units)."""
         dq, dk, dv, dkm, dsinks = ins[:5]
         if w.kind == "backward":
             tb.backward(dq, dk, dv, ins[5], scale=w.softmax_scale, causal=w.causal, window=w.window,
@@ -329,36 +491,22 @@ def main():
             tb.prefill_ring(dq, dk, dv, S=w.S, window=w.window, scale=w.softmax_scale,
                             softcap=w.softcap, sinks=dsinks, out=o)
         else:
-            tb.prefill(dq, dk, dv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                       key_mask=dkm, out=o, softcap=w.softcap, sinks=dsinks)
+            for r_ in runs:
+                (qb, qh), (kb, kh) = run_slices(r_, G)
+                tb.prefill(dq[qb, qh], dk[kb, kh], dv[kb, kh], scale=w.softmax_scale,
+                           causal=w.causal, window=w.window,
+                           key_mask=dkm[qb] if dkm is not None else None, out=o[qb, qh],
+                           softcap=w.softcap, sinks=dsinks[qh] if dsinks is not None else None)
 
     def step():
         call(dev_inputs, out)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-    tb.check_status(stream)
-
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t_wall = time.perf_counter()
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-        torch.cuda.synchronize(dev)
-        t_wall = time.perf_counter() - t_wall
-    barrier(world)
-    tb.check_status(stream)
-    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]  # ms
+    per, clocks, t_wall = time_launches(step, flush, stream, args.steps, args.warmup, dev, world)
     mean_ms = sum(per) / len(per)
     mean_ms = max_over_ranks(mean_ms, world)
-    value = weak_scaling_rate(flops, world, mean_ms * 1e-3) / 1e12
+    # whole-job throughput: every rank's units over the slowest rank's time
+    job_flops = call_flops if strong else flops * world
+    value = job_flops / (mean_ms * 1e-3) / 1e12
     per_sorted = sorted(per)
 
     # L2-warm reference (no flush between launches; the inputs of the previous
@@ -374,6 +522,7 @@ def main():
     tb.check_status(stream)
     warm_sorted = sorted(s_.elapsed_time(e_) for s_, e_ in zip(w_starts, w_ends))
     warm_ms = max_over_ranks(warm_sorted[len(warm_sorted) // 2], world)
+    errors = oracle_errors(w, out, q, k, v, km) if (w.kind == "dense" and world == 1) else None
 
     # end to end through the C ABI with host buffers (copies inside the timed region)
     pinned = [t.pin_memory() if t is not None else None for t in host_inputs]
@@ -399,11 +548,18 @@ def main():
                  "backward": "tfa_prefill_backward_saved" if w.saved_stats else "tfa_prefill_backward"
                  }.get(w.kind, "tfa_attention_ex")
         e2e_api = f"{entry} (pinned host buffers, copies on the stream)"
+        h2d = sum(t.numel() * t.element_size() for t in pinned if t is not None)
     else:
         def e2e_step():
-            tb.prefill_host(hq, hk, hv, scale=w.softmax_scale, causal=w.causal, window=w.window,
-                            key_mask=hkm, out=hout, stream=stream)
+            for r_ in runs:  # this rank's share, from and to host buffers
+                (qb, qh), (kb, kh) = run_slices(r_, G)
+                tb.prefill_host(hq[qb, qh], hk[kb, kh], hv[kb, kh], scale=w.softmax_scale,
+                                causal=w.causal, window=w.window,
+                                key_mask=hkm[qb] if hkm is not None else None, out=hout[qb, qh],
+                                stream=stream)
         e2e_api = "tfa_prefill_host (pinned host buffers)"
+        h2d = sum(hq[run_slices(r_, G)[0]].numel() * 2 + 2 * hk[run_slices(r_, G)[1]].numel() * 2 +
+                  (hkm[r_.b0:r_.b0 + r_.nb].numel() * 4 if hkm is not None else 0) for r_ in runs)
     for _ in range(3):
         e2e_step()
     barrier(world)
@@ -416,8 +572,10 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world)
-    h2d = sum(t.numel() * t.element_size() for t in pinned if t is not None)
-    d2h = sum(t.numel() * 2 for t in hout) if w.kind == "backward" else hout.numel() * 2
+    if runs is not None:
+        d2h = sum(hout[run_slices(r_, G)[0]].numel() * 2 for r_ in runs)
+    else:
+        d2h = sum(t.numel() * 2 for t in hout) if w.kind == "backward" else hout.numel() * 2
 
     peaks, peak_kind = load_peaks()
     alg_bytes = workload_bytes(w)
@@ -425,27 +583,30 @@ def main():
         # short queries read every K/V byte for a few flops: bounded by HBM
         bound, roof_unit = "hbm", "GB/s"
         peak = float(peaks["hbm_gbs"])
-        achieved = alg_bytes / (mean_ms * 1e-3) / 1e9
+        achieved = alg_bytes * flops / call_flops / (mean_ms * 1e-3) / 1e9
         peak_source = f"{peak_kind} hbm_gbs (copy bandwidth)"
     else:
         bound, roof_unit = "tensor", "TFLOP/s"
         peak = float(peaks["bf16_tflops"])
         achieved = flops / (mean_ms * 1e-3) / 1e12  # per GPU, per launch
         peak_source = f"{peak_kind} bf16_tflops (burst; kernel timed alone)"
-    traffic = recorded_traffic(w.name)
-    clocks = clk.summary()
+    traffic = recorded_traffic(w.name) if (world == 1 or not strong) else None
+    n_calls = len(runs) if runs is not None else 1
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "higher_is_better": True, "scaling": "strong" if strong else "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(w), "useful_gflop": flops / 1e9,
+            "config": {**workload_config(w), "useful_gflop": job_flops / 1e9,
                        "l2": "flushed between steps (256 MiB memset outside the step events)",
-                       "parallelism": f"weak x{world}" if world > 1 else "single GPU"},
+                       "parallelism": ("single GPU" if world == 1 else
+                                       f"(batch, KV group) units of one call over {world} GPUs: "
+                                       + ("the workload's own call (strong)" if strong else
+                                          f"a call of {world} x B elements, one copy per GPU (weak)"))},
             "ms_p10": per_sorted[len(per) // 10], "ms_p50": per_sorted[len(per) // 2],
             "ms_p90": per_sorted[(9 * len(per)) // 10],
-            "l2_warm": {"ms_p50": warm_ms, "value": weak_scaling_rate(flops, world, warm_ms * 1e-3) / 1e12,
+            "l2_warm": {"ms_p50": warm_ms, "value": job_flops / (warm_ms * 1e-3) / 1e12,
                         "unit": UNIT, "launches": n_warm},
             "pct_of_peak": 100.0 * achieved / peak,
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
@@ -453,15 +614,19 @@ def main():
                          "peak_source": peak_source,
                          "traffic": traffic,
                          "algorithmic_bytes": alg_bytes},
-            "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
+            "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms, "api": e2e_api},
-            # kernels per step: one, or four for the backward (forward recompute,
-            # delta, dQ, dK/dV), three when it starts from the saved statistics
-            "gpu_launches": args.steps * ((3 if w.saved_stats else 4) if w.kind == "backward" else 1),
+            # kernels per step: one per call, or four for the backward (forward
+            # recompute, delta, dQ, dK/dV), three when it starts from the saved statistics
+            "gpu_launches": args.steps * ((3 if w.saved_stats else 4) if w.kind == "backward" else n_calls),
             "clocks": clocks,
             "wall_s_timed_region": t_wall,
         }
+        if errors is not None:
+            line["error_vs_oracle"] = errors
+        if world == 1 and not args.no_per_config and w.name == HEADLINE:
+            line["per_config"] = per_config(args, dev, flush, stream, peaks)
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

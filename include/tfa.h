@@ -257,6 +257,14 @@ int tfa_prefill_backward_saved(const void *q, const void *k, const void *v, cons
 #define TFA_DEBUG_FORCE_SPLIT  16u /* always split key ranges evenly across the CTAs (by
                                       default the library picks the schedule it estimates
                                       finishes first) */
+#define TFA_DEBUG_SHORT_WAITS  32u /* give up every pipeline wait of the kernel after ~1000 SM
+                                      cycles instead of ~4 s, to exercise the give-up path: the
+                                      waits run out, the kernel drains its copies and tensor-core
+                                      work, the output is invalid and tfa_check_status (or
+                                      TFA_DEBUG_SYNC) returns TFA_ERR_TIMEOUT.  Refused with
+                                      TFA_ERR_FLAGS for L <= 128 (packed tiles, whose merge joins
+                                      a whole warpgroup at a barrier that a warp which gave up
+                                      early would never reach). */
 
 /* tfa_prefill_debug -- tfa_prefill with debug flags (arguments as above).  With
  * NO_TILE_SKIP and/or MASK_ALL the result must be bit-identical to tfa_prefill's
@@ -288,29 +296,36 @@ int tfa_prefill_host(const void *q, const void *k, const void *v, void *o,
  * memory (a caching or arena allocator owns all of it, allocation is not
  * allowed at the point of the call, or the host runtime only hands out its own
  * buffers).  No counterpart on the pages: it exists for those callers.
- * Arguments, layout and results are exactly tfa_prefill's; the caller still
- * passes every input and output.  The difference is the kernel's scratch (its
- * status word): it lives in a fixed 256-byte device array inside the library,
- * which every GPU that loads the library holds until the process exits, and
- * the call makes no cudaMalloc, cudaFree or other allocating call.
+ * Arguments, layout and validation are tfa_prefill's; the caller still passes
+ * every input and output.  The call makes no cudaMalloc, cudaFree or other
+ * allocating call: the kernel's scratch (its status word) lives in a fixed
+ * 256-byte device array inside the library, which every GPU that loads the
+ * library holds until the process exits.
+ *   - It always runs the whole-item schedule (no query tile is cut into key
+ *     ranges; the split schedule's partials would not fit the array), so its
+ *     output is not bit-identical to tfa_prefill's, which may cut tiles and
+ *     merge partial results in another rounding order.  Both match the fp64
+ *     definition within the operator tolerance (|err| <= 0.02 + 0.02 |ref|).
+ *     On large causal calls the whole-item schedule can be slower.
  *   - The first call on a device sets the array up (looks up its address and
- *     clears it with that device current); make that first call before any
- *     stream capture.
+ *     clears it with that device current); a first call made while `stream`
+ *     is being captured is refused with TFA_ERR_CAPTURE.
  *   - Every call shares the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other threads) race on it.
- *   - A call whose scratch would exceed the 256-byte maximum is rejected with
- *     TFA_ERR_SHAPE and a message in tfa_last_error(); today's kernel needs
- *     4 bytes for every size tfa_prefill accepts.
+ *   - The kernel needs 4 bytes of the 256-byte maximum for every size
+ *     tfa_prefill accepts (checked when the library is compiled), so no valid
+ *     call is rejected for its size.
  *   - A timed-out kernel wait is reported by tfa_check_status, as for tfa_prefill. */
 int tfa_prefill_noalloc(const void *q, const void *k, const void *v, void *o,
                         int B, int Hq, int Hkv, int L, int S, int D, float scale,
                         int causal, int window, const float *key_mask, tfa_stream_t stream);
 
 /* tfa_check_status -- synchronizes `stream`, then reads and clears the current
- * device's status words (tfa_prefill's and, once set up, tfa_prefill_noalloc's).
- * Returns TFA_OK, TFA_ERR_TIMEOUT if a kernel launched since the last check
- * recorded a wait that gave up, TFA_ERR_SEQLENS if a tfa_prefill_varlen call
- * met inconsistent cu_seqlens (and no wait gave up), or TFA_ERR_CUDA. */
+ * device's status words (tfa_prefill's and, once set up, tfa_prefill_noalloc's;
+ * both are read and cleared on every call).  Returns TFA_OK, TFA_ERR_TIMEOUT if
+ * a kernel launched since the last check recorded a wait that gave up (in
+ * either word), TFA_ERR_SEQLENS if a tfa_prefill_varlen call met inconsistent
+ * cu_seqlens (and no wait gave up), or TFA_ERR_CUDA. */
 int tfa_check_status(tfa_stream_t stream);
 
 /* tfa_last_error -- for the calling host thread, a description of the last CUDA

@@ -42,6 +42,7 @@ TFA_DEBUG_MASK_ALL = 2
 TFA_DEBUG_SYNC = 4
 TFA_DEBUG_NO_SPLIT = 8
 TFA_DEBUG_FORCE_SPLIT = 16
+TFA_DEBUG_SHORT_WAITS = 32
 
 MIN_QUERY_ROWS = 9
 MAX_DECODE_ROWS = 8

@@ -384,7 +384,8 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     p.G = Hq / Hkv;
     p.causal = causal ? 1 : 0;
     p.window = (causal && window > 0) ? window : 0;
-    p.flags = flags;
+    p.flags = flags & (tfa::kFlagNoTileSkip | tfa::kFlagMaskAll);
+    p.wait_limit = (flags & TFA_DEBUG_SHORT_WAITS) ? tfa::TFA_SHORT_WAIT_CYCLES : tfa::TFA_WAIT_LIMIT_CYCLES;
     p.scale_log2 = scale * 1.4426950408889634f;
     // softcap: y = b (1 - 2 / (2^(a x) + 1)) with a = 2 scale log2(e) / cap, b = cap / scale
     p.softcap_a = sc ? 2.f * scale * 1.4426950408889634f / softcap : 0.f;
@@ -407,7 +408,7 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     sh.S = S;
     sh.causal = p.causal;
     sh.window = p.window;
-    sh.flags = flags;
+    sh.flags = p.flags;
     sh.n_qp = tfa::shape_n_qp(L);
     const long long n_items = static_cast<long long>(B) * sh.Hq * sh.n_qp;
     p.W = varlen ? 0 : tfa::total_steps(sh);  // varlen: per-sequence lengths live on the device
@@ -438,16 +439,18 @@ int prefill_impl(const void *q, const void *k, const void *v, void *o, int B, in
     int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
     if (rc) return rc;
     if (flags & ~(TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL | TFA_DEBUG_SYNC | TFA_DEBUG_NO_SPLIT |
-                  TFA_DEBUG_FORCE_SPLIT) ||
+                  TFA_DEBUG_FORCE_SPLIT | TFA_DEBUG_SHORT_WAITS) ||
         ((flags & TFA_DEBUG_NO_SPLIT) && (flags & TFA_DEBUG_FORCE_SPLIT)))
         return TFA_ERR_FLAGS;
+    // packed tiles (L <= 128) merge at warpgroup barriers that an early give-up could leave waiting
+    if ((flags & TFA_DEBUG_SHORT_WAITS) && L <= tfa::kBlockQ) return TFA_ERR_FLAGS;
     const bool force_split = (flags & TFA_DEBUG_FORCE_SPLIT) != 0;
     DeviceState *st = nullptr;
     SplitScratch *ss = nullptr;
     std::lock_guard<std::mutex> lk(g_mutex);
     if ((rc = device_state(stream, &st))) return rc;
     if (!(flags & TFA_DEBUG_NO_SPLIT) && (rc = split_scratch(*st, stream, &ss))) return rc;
-    const unsigned kflags = flags & (TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL);
+    const unsigned kflags = flags & (TFA_DEBUG_NO_TILE_SKIP | TFA_DEBUG_MASK_ALL | TFA_DEBUG_SHORT_WAITS);
     rc = (D == 128) ? launch<128>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
                                   key_mask, stream, kflags, ss, force_split)
                     : launch<64>(*st, q, k, v, o, B, Hq, Hkv, L, S, scale, causal, window,
@@ -854,7 +857,8 @@ extern "C" int tfa_prefill_host(const void *q, const void *k, const void *v, voi
 // address: its real address is looked up with cudaGetSymbolAddress once per
 // device, with that device current, and passed to the kernel.
 constexpr size_t kNoAllocScratchBytes = 256;            // the stated maximum
-constexpr size_t kKernelScratchBytes = sizeof(unsigned);  // what the kernel needs today
+constexpr size_t kKernelScratchBytes = sizeof(unsigned);  // what the kernel needs, for every size
+static_assert(kKernelScratchBytes <= kNoAllocScratchBytes, "the kernel's scratch must fit the static array");
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
@@ -867,6 +871,9 @@ int noalloc_state(cudaStream_t stream, DeviceState **out) {
     if (dev < 0 || dev >= kMaxDevices) return drv_fail("device index out of range", dev);
     DeviceState &st = g_noalloc_dev[dev];
     if (!st.init) {
+        // the set-up below clears the array with a memset that a capture would
+        // record instead of running
+        if (int rc = refuse_under_capture(stream, "the no-alloc scratch")) return rc;
         void *ptr = nullptr;
         if ((e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch)) != cudaSuccess)
             return cuda_fail("cudaGetSymbolAddress(no-alloc scratch)", e);
@@ -901,12 +908,6 @@ extern "C" int tfa_prefill_noalloc(const void *q, const void *k, const void *v, 
                                    int window, const float *key_mask, tfa_stream_t stream) {
     int rc = validate(q, k, v, o, B, Hq, Hkv, L, S, D, scale, causal, window, key_mask, true);
     if (rc) return rc;
-    if (kKernelScratchBytes > kNoAllocScratchBytes) {
-        snprintf(g_last_error, sizeof g_last_error,
-                 "this call needs %zu bytes of scratch, more than the %zu-byte no-alloc maximum",
-                 kKernelScratchBytes, kNoAllocScratchBytes);
-        return TFA_ERR_SHAPE;
-    }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     DeviceState *st = nullptr;
     std::lock_guard<std::mutex> lk(g_mutex);
@@ -923,10 +924,13 @@ extern "C" int tfa_check_status(tfa_stream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TFA_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mutex);
-    int rc = TFA_OK;
-    if (g_dev[dev].init) rc = take_status_word(g_dev[dev].status);
-    if (rc == TFA_OK && g_noalloc_dev[dev].init) rc = take_status_word(g_noalloc_dev[dev].status);
-    return rc;
+    // read and clear both words every time, so that neither is left set and
+    // blamed on later calls; a timeout in either one wins
+    const int a = g_dev[dev].init ? take_status_word(g_dev[dev].status) : TFA_OK;
+    const int b = g_noalloc_dev[dev].init ? take_status_word(g_noalloc_dev[dev].status) : TFA_OK;
+    if (a == TFA_ERR_CUDA || b == TFA_ERR_CUDA) return TFA_ERR_CUDA;
+    if (a == TFA_ERR_TIMEOUT || b == TFA_ERR_TIMEOUT) return TFA_ERR_TIMEOUT;
+    return a != TFA_OK ? a : b;
 }
 
 extern "C" const char *tfa_last_error(void) { return g_last_error; }

@@ -160,6 +160,7 @@ struct Params {
     int B, Hq, Hkv, L, S, G;
     int causal, window;
     unsigned flags;
+    long long wait_limit;  // SM cycles before a pipeline wait gives up (TFA_WAIT_LIMIT_CYCLES)
     float scale_log2;  // softmax scale * log2(e)
     long long W;       // total key-tile steps (split schedule)
     Shape shape;
@@ -305,7 +306,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
         for (int t = 0; t < 2; ++t) {
             if (!ip.present[t]) continue;
             if (q_use[t] > 0 &&
-                !__all_sync(lanes, mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status)))
+                !__all_sync(lanes, mbar_wait(bar.q_empty(t), (q_use[t] - 1) & 1, abort_flag, p.status, p.wait_limit)))
                 goto out;
             if (lane == 0) {
                 if (PK || p.packed) {  // box {64, L, pack_heads}: rows (head, query row) in order
@@ -329,7 +330,7 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                 const uint32_t s = kv_prod % C::kSlots;
                 const uint32_t round = kv_prod / C::kSlots;
                 if (round > 0 &&
-                    !__all_sync(lanes, mbar_wait(bar.kv_empty(s), (round - 1) & 1, abort_flag, p.status)))
+                    !__all_sync(lanes, mbar_wait(bar.kv_empty(s), (round - 1) & 1, abort_flag, p.status, p.wait_limit)))
                     goto out;
                 if (which == 0 && has_km) {
                     // bias column of this K tile: 0 for kept keys, -inf otherwise
@@ -466,11 +467,11 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
         while (it.next(p.shape, seg)) {
             const ItemPlan ip = plan_piece<PK>(p, seg);
             if (ip.jl > ip.jh) continue;  // no key tile: nothing was loaded
-            if (!mbar_wait(bar.q_full(0), q_use[0] & 1, abort_flag, p.status)) goto out;
+            if (!mbar_wait(bar.q_full(0), q_use[0] & 1, abort_flag, p.status, p.wait_limit)) goto out;
             ++q_use[0];
             {
                 const uint32_t s = kv_cons % C::kSlots;
-                if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 ++kv_cons;
                 tc_fence_after();
                 qk_to(0, s);
@@ -482,11 +483,11 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                 TFA_TR(2, trace_step, 0);
                 const int buf = (j - ip.jl) & 1;
                 const uint32_t sv = kv_cons % C::kSlots;
-                if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 ++kv_cons;
                 if (j < ip.jh) {
                     const uint32_t sk = kv_cons % C::kSlots;
-                    if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                    if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status, p.wait_limit)) goto out;
                     ++kv_cons;
                     tc_fence_after();
                     TFA_TR(2, trace_step, 1);
@@ -495,11 +496,11 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                     if (j + 1 == ip.jh) umma_commit(bar.q_empty(0));
                     umma_commit(bar.kv_empty(sk));
                 }
-                if (!mbar_wait(bar.p_part(0), p_cnt[0] & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.p_part(0), p_cnt[0] & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 TFA_TR(2, trace_step, 2);
                 tc_fence_after();
                 pv_from(buf, sv, j > ip.jl, 0, kPartKeys / 16);
-                if (!mbar_wait(bar.p_full(0), p_cnt[0] & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.p_full(0), p_cnt[0] & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 TFA_TR(2, trace_step, 3);
                 ++p_cnt[0];
                 tc_fence_after();
@@ -515,12 +516,12 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
                 if (!ip.present[t]) continue;
-                if (!mbar_wait(bar.q_full(t), q_use[t] & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.q_full(t), q_use[t] & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 ++q_use[t];
             }
             {
                 const uint32_t s = kv_cons % C::kSlots;
-                if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.kv_full(s), (kv_cons / C::kSlots) & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 ++kv_cons;
                 tc_fence_after();
 #pragma unroll
@@ -537,13 +538,13 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
             for (int j = ip.jl; j <= ip.jh; ++j) {
                 TFA_TR(2, trace_step, 0);
                 const uint32_t sv = kv_cons % C::kSlots;
-                if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status)) goto out;
+                if (!mbar_wait(bar.kv_full(sv), (kv_cons / C::kSlots) & 1, abort_flag, p.status, p.wait_limit)) goto out;
                 ++kv_cons;
                 const bool next = j < ip.jh;
                 uint32_t sk = 0;
                 if (next) {
                     sk = kv_cons % C::kSlots;
-                    if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status))
+                    if (!mbar_wait(bar.kv_full(sk), (kv_cons / C::kSlots) & 1, abort_flag, p.status, p.wait_limit))
                         goto out;
                     ++kv_cons;
                 }
@@ -555,11 +556,11 @@ __device__ void mma_role(const Params &p, uint32_t sbase, uint32_t tmem, const B
                     if (ip.lo[t] <= j && j <= ip.hi[t]) {
                         // first part of P_t, then the rest (the tensor core works on
                         // the first part meanwhile)
-                        if (!mbar_wait(bar.p_part(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                        if (!mbar_wait(bar.p_part(t), p_cnt[t] & 1, abort_flag, p.status, p.wait_limit)) goto out;
                         TFA_TR(2, trace_step, 2 + 2 * t);
                         tc_fence_after();
                         issue_pv(t, sv, acc[t], 0, kPartKeys / 16);
-                        if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status)) goto out;
+                        if (!mbar_wait(bar.p_full(t), p_cnt[t] & 1, abort_flag, p.status, p.wait_limit)) goto out;
                         ++p_cnt[t];
                         tc_fence_after();
                         issue_pv(t, sv, true, kPartKeys / 16, kBlockK / 16);
@@ -621,7 +622,7 @@ __device__ __forceinline__ bool merge_packed(const Params &p, const Segment &seg
 #endif
     bool ok = true;
     for (int k = blockIdx.x + 1 + r; k <= c_last && ok; k += 128)
-        ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status);
+        ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status, p.wait_limit);
     // the slot writes of this warpgroup and the flags seen by it are ordered
     // before every read below; all threads leave together on an abort
     if (named_barrier_or(1 + t, 128, !ok || *abort_flag)) return false;
@@ -777,7 +778,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
                 sph = s_cnt++ & 1;
             }
             // all lanes leave together: the tcgen05 loads below are warp-collective
-            if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(sb), sph, abort_flag, p.status)))
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.s_full(sb), sph, abort_flag, p.status, p.wait_limit)))
                 return;
             if (r == 0) TFA_TR(t, trace_step, 1);
             tc_fence_after();
@@ -853,7 +854,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if constexpr (PK) {
                 // the previous tile's P.V product may still be accumulating
                 if (j > ip.lo) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(1), pv_cnt & 1, abort_flag, p.status)))
+                    if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(1), pv_cnt & 1, abort_flag, p.status, p.wait_limit)))
                         return;
                     ++pv_cnt;
                     tc_fence_after();
@@ -920,7 +921,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             ++trace_step;
         }
 
-        if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(t), o_cnt & 1, abort_flag, p.status)))
+        if (!__all_sync(0xffffffffu, mbar_wait(bar.o_full(t), o_cnt & 1, abort_flag, p.status, p.wait_limit)))
             return;
         ++o_cnt;
         tc_fence_after();
@@ -963,7 +964,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.pub(t));
-            if (r == 0 && mbar_wait(bar.pub(t), pub_cnt & 1, abort_flag, p.status)) {
+            if (r == 0 && mbar_wait(bar.pub(t), pub_cnt & 1, abort_flag, p.status, p.wait_limit)) {
                 __threadfence();
                 st_release_gpu(p.ready + partial_slot(blockIdx.x, t), epoch);
             }
@@ -981,10 +982,10 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
             if (r == 0) {
                 bool ok = true;
                 for (int k = blockIdx.x + 1; k <= c_last && ok; ++k)
-                    ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status);
+                    ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status, p.wait_limit);
                 mbar_arrive(bar.fin(t));  // arrive even on failure; the abort flag tells
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(bar.fin(t), fin_cnt & 1, abort_flag, p.status)))
+            if (!__all_sync(0xffffffffu, mbar_wait(bar.fin(t), fin_cnt & 1, abort_flag, p.status, p.wait_limit)))
                 return;
             ++fin_cnt;
             if (*abort_flag) return;

@@ -13,6 +13,9 @@
 namespace tfa {
 
 constexpr long long TFA_WAIT_LIMIT_CYCLES = 8ll << 30;  // ~4 s at 2 GHz
+// The limit a TFA_DEBUG_SHORT_WAITS launch gives the pipeline waits (the
+// drains on the way out keep their own, normal limit).
+constexpr long long TFA_SHORT_WAIT_CYCLES = 1000;
 constexpr unsigned TFA_DEVICE_TIMEOUT = 1u;
 // A packed variable-length call met a sequence whose cu_seqlens entries are
 // inconsistent (decreasing, past the packed length, longer than max_seqlen_q,
@@ -55,15 +58,16 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 // Wait until the phase with the given parity has completed.  Returns false if
-// the CTA is aborting or the wait ran past its limit (then it starts the abort).
+// the CTA is aborting or the wait ran past `limit` cycles (then it starts the
+// abort).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                          unsigned *status) {
+                                          unsigned *status, long long limit = TFA_WAIT_LIMIT_CYCLES) {
     if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_test(bar, parity)) return true;
         if (*abort_flag) return false;
-        if (clock64() - t0 > TFA_WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             atomicOr(status, TFA_DEVICE_TIMEOUT);
             return false;
@@ -273,11 +277,12 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *addr) {
 }
 // Wait, bounded like mbar_wait, until *flag == value (written by another CTA).
 __device__ __forceinline__ bool flag_wait(const unsigned *flag, unsigned value,
-                                          volatile int *abort_flag, unsigned *status) {
+                                          volatile int *abort_flag, unsigned *status,
+                                          long long limit = TFA_WAIT_LIMIT_CYCLES) {
     const long long t0 = clock64();
     while (ld_acquire_gpu(flag) != value) {
         if (*abort_flag) return false;
-        if (clock64() - t0 > TFA_WAIT_LIMIT_CYCLES) {
+        if (clock64() - t0 > limit) {
             *abort_flag = 1;
             atomicOr(status, TFA_DEVICE_TIMEOUT);
             return false;

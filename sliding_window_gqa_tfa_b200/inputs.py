@@ -180,6 +180,26 @@ def make_dout(w: Workload, seed: int = 0):
     return _draw(w, seed)[5]
 
 
+def sample_rows(w: Workload, n_per_head: int = 24, seed: int = 0):
+    """Flat row indices (b * Hq + h) * L + i of a full-size dense workload to
+    check one by one: the tile edges and tails, the middle row and random rows,
+    n_per_head of them in every head."""
+    import numpy as np
+
+    rng = np.random.default_rng(seed)
+    L = w.L
+    n_per_head = min(n_per_head, L)  # a short query has fewer rows than the sample size
+    fixed = [0, 1, 127, 128, 255, 256, L // 2, L - 129, L - 128, L - 2, L - 1]
+    rows = []
+    for b in range(w.B):
+        for h in range(w.Hq):
+            pick = set(i for i in fixed if 0 <= i < L)
+            while len(pick) < n_per_head:
+                pick.add(int(rng.integers(0, L)))
+            rows += [(b * w.Hq + h) * L + i for i in sorted(pick)]
+    return np.array(rows, dtype=np.int64)
+
+
 def shaped(B, Hq, Hkv, L, S, D, *, causal=True, window=0, key_mask_keep=None, k_scale=1.0,
            softcap=0.0, sink_scale=None, name="custom") -> Workload:
     """A workload of arbitrary shape drawn by the same recipe (for edge-case tests)."""

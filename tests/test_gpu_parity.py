@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from sliding_window_gqa_tfa_b200 import binding as tb
-from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_inputs, make_sinks, shaped
+from sliding_window_gqa_tfa_b200.inputs import WORKLOADS, make_inputs, make_sinks, sample_rows, shaped
 
 pytestmark = pytest.mark.gpu
 
@@ -200,18 +200,7 @@ def test_stream_argument_is_respected():
 
 def _sample_rows(w, n_per_head=24, seed=0):
     """Rows to check at full size: tile edges, tails and random rows, every head."""
-    rng = np.random.default_rng(seed)
-    L = w.L
-    n_per_head = min(n_per_head, L)  # a short query has fewer rows than the sample size
-    fixed = [0, 1, 127, 128, 255, 256, L // 2, L - 129, L - 128, L - 2, L - 1]
-    rows = []
-    for b in range(w.B):
-        for h in range(w.Hq):
-            pick = set(i for i in fixed if 0 <= i < L)
-            while len(pick) < n_per_head:
-                pick.add(int(rng.integers(0, L)))
-            rows += [(b * w.Hq + h) * L + i for i in sorted(pick)]
-    return np.array(rows, dtype=np.int64)
+    return sample_rows(w, n_per_head=n_per_head, seed=seed)
 
 
 @pytest.mark.parametrize("name", [n for n, w in WORKLOADS.items()
