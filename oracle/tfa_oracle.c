@@ -145,8 +145,9 @@ static int check_args(const void *q, const void *k, const void *v, const void *o
 
 /* Where one output row reads its operands: its query vector, and the K and V
  * rows of its KV head -- key j at row slot(j) of kb / vb, rows kv_stride
- * elements apart.  slot(j) = j, or j mod ring for a rotating cache
- * (TensorFold PR 3269: "the ring slot of a key and value row"). */
+ * elements apart.  slot(j) = j, or j mod ring for a rotating cache (the
+ * TensorFold PR 3269 page names a ring-slot position for each cached key and
+ * value row without giving a formula; j mod ring is the reading taken). */
 typedef struct {
     const uint16_t *qr, *kb, *vb;
     size_t kv_stride;
@@ -786,7 +787,8 @@ int64_t oracle_count_pairs(int B, int Hq, int L, int S, int causal, int window,
  * (row, key) pair for ANY row of the block is skipped without reading K/V
  * (the masked-tile skipping of mlx-lm PR "Skip fully masked key tiles in Flint
  * sliding-window prefill").  A tile with no allowed key for one row contributes
- * nothing to that row ("padded score cells contribute no probability mass").
+ * nothing to that row: its masked scores add zero weight to the row sum and to
+ * the accumulator (tiny-llm Week 2 Day 5, Task 1, the merge with masked cells).
  * Exists so tests can show that tiling, merging and skipping leave the plain
  * definition's result unchanged. */
 int oracle_attention_blockwise(const uint16_t *q, const uint16_t *k, const uint16_t *v, double *o,

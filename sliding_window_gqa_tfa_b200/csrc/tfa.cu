@@ -424,11 +424,36 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
         if (force_split || tfa::makespan_estimate(sp, p.W) < tfa::makespan_estimate(sh, p.W)) sh = sp;
     }
     if (!sh.split) ss = nullptr;
-    const int grid = sh.grid;
     p.partial = ss ? ss->partial : nullptr;
     p.ready = ss ? ss->ready : nullptr;
     p.ctl = ss ? ss->ctl : nullptr;
-    kern<<<grid, tfa::kThreads, smem, stream>>>(mq, mk, mv, p);
+    if (sh.split) {
+        // A split-schedule finalizer waits for flags that later CTAs of the grid
+        // set, which needs every CTA resident at once (one per SM).  A cooperative
+        // launch guarantees that or fails at once (an MPS SM limit, a green
+        // context, another kernel holding SMs cannot make it wait forever); the
+        // call then runs the whole-item schedule, which has no waits between CTAs.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sh.grid));
+        cfg.blockDim = dim3(tfa::kThreads);
+        cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
+        if (e == cudaSuccess) return TFA_OK;
+        if (e != cudaErrorCooperativeLaunchTooLarge) return cuda_fail("kernel launch (cooperative)", e);
+        (void)cudaGetLastError();  // not sticky; clear it and deal whole items instead
+        sh.split = 0;
+        sh.grid = n_items < st.sm_count ? static_cast<int>(n_items) : st.sm_count;
+        p.partial = nullptr;
+        p.ready = nullptr;
+        p.ctl = nullptr;
+    }
+    kern<<<sh.grid, tfa::kThreads, smem, stream>>>(mq, mk, mv, p);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? TFA_OK : cuda_fail("kernel launch", e);
 }
