@@ -78,16 +78,6 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunc
 // Lazy rescale: keep the stale row maximum until the true one exceeds it by
 // more than 2^8 in the exp2 domain (P values then stay <= 256).
 constexpr float kRescaleThresholdLog2 = 8.0f;
-// One pair of exponentials in every kPolyPeriod goes to the FMA-pipe polynomial
-// instead of the MUFU unit (0: all on MUFU).  The MUFU unit alone (16/clk/SM)
-// needs as long for a 128 x 128 tile as the tensor core needs for its two MMAs,
-// but with one warp per row block the loop is latency-bound, not MUFU-bound, and
-// measured fastest with every exponential on MUFU; the polynomial path is kept
-// (tested) for configurations where the MUFU unit becomes the limit.
-#ifndef TFA_POLY_PERIOD
-#define TFA_POLY_PERIOD 0
-#endif
-constexpr int kPolyPeriod = TFA_POLY_PERIOD;
 // The softmax publishes P in two parts: keys [0, kPartKeys) first, so the P.V
 // product runs on them while the last keys' exponentials are computed.
 constexpr int kPartKeys = 96;
@@ -878,12 +868,8 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     do {                                                                                   \
         const float2 x = fma2(make_float2(TFA_F(2 * (i)), TFA_F(2 * (i) + 1)), c2, nmc2);  \
         float2 e;                                                                          \
-        if (kPolyPeriod > 0 && ((i) % (kPolyPeriod > 0 ? kPolyPeriod : 1)) == kPolyPeriod - 1) { \
-            e = exp2_poly2(x); /* FMA pipe */                                              \
-        } else {                                                                           \
-            e.x = ex2(x.x); /* MUFU */                                                     \
-            e.y = ex2(x.y);                                                                \
-        }                                                                                  \
+        e.x = ex2(x.x); /* MUFU */                                                         \
+        e.y = ex2(x.y);                                                                    \
         if ((i) & 1)                                                                       \
             acc1 = add2(acc1, e);                                                          \
         else                                                                               \

@@ -337,40 +337,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
         : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
     return *reinterpret_cast<float2 *>(&d);
 }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-    uint64_t d;
-    asm("mul.f32x2 %0, %1, %2;"
-        : "=l"(d)
-        : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
-    return *reinterpret_cast<float2 *>(&d);
-}
-
-// 2^x for a pair, on the FMA/ALU pipes instead of the MUFU unit, so the kernel
-// can split its exponentials between both.  Cody-Waite reduction: n = round(x)
-// by adding 1.5 * 2^23 (the integer lands in the low mantissa bits), f = x - n
-// in [-1/2, 1/2], 2^f by a degree-3 relative-error minimax polynomial fitted
-// with the Remez exchange algorithm (csrc/gen_exp2_poly.py; max relative error
-// 7.5e-5), and 2^n built as a float from n's bits.  x is clamped at -127, where
-// 2^n becomes the bit pattern 0: masked scores (-inf) give exactly 0.
-constexpr float kExp2C0 = 0.9999280571937561f;
-constexpr float kExp2C1 = 0.6932609677314758f;
-constexpr float kExp2C2 = 0.2426111251115799f;
-constexpr float kExp2C3 = 0.0551716685295105f;
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    x.x = fmaxf(x.x, -127.f);
-    x.y = fmaxf(x.y, -127.f);
-    const float2 t = add2(x, make_float2(kRound, kRound));
-    const float2 n = add2(t, make_float2(-kRound, -kRound));
-    const float2 f = fma2(n, make_float2(-1.f, -1.f), x);
-    float2 pf = fma2(make_float2(kExp2C3, kExp2C3), f, make_float2(kExp2C2, kExp2C2));
-    pf = fma2(pf, f, make_float2(kExp2C1, kExp2C1));
-    pf = fma2(pf, f, make_float2(kExp2C0, kExp2C0));
-    // t's low bits hold n (two's complement); (t << 23) + (127 << 23) = bits of 2^n
-    const float2 scale = make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + 0x3F800000u),
-                                     __uint_as_float((__float_as_uint(t.y) << 23) + 0x3F800000u));
-    return mul2(pf, scale);
-}
 
 // Two fp32 -> one bf16x2 word, round to nearest even; `lo` lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
