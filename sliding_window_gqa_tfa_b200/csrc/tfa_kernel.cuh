@@ -79,8 +79,9 @@ static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * kRegsLaunc
 // more than 2^8 in the exp2 domain (P values then stay <= 256).
 constexpr float kRescaleThresholdLog2 = 8.0f;
 // The softmax publishes P in two parts: keys [0, kPartKeys) first, so the P.V
-// product runs on them while the last keys' exponentials are computed.
-constexpr int kPartKeys = 96;
+// product starts on them while the other keys' exponentials are computed.
+// (32 measured 0.5-1.8 % faster than 96 or 64 on the prefill workloads.)
+constexpr int kPartKeys = 32;
 static_assert(kPartKeys % 32 == 0 && kPartKeys % 16 == 0 && kPartKeys < 128, "P split");
 
 constexpr int kMaxVarlenSeqs = 1024;  // sequences per packed variable-length call
