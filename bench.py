@@ -100,17 +100,19 @@ print("max", pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM), flush=Tr
 out = []
 t_end = time.time() + 600
 while not stop and time.time() < t_end:
-    out.append("%d %d" % (pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get(h))))
-    time.sleep(0.0005)
+    t = time.time()
+    out.append("%.6f %d %d" % (t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get(h))))
 print(chr(10).join(out), flush=True)
 """
 
 
 class ClockSampler:
     """SM clock and throttle reasons sampled during the timed region: NVML
-    polled every ~0.5 ms by a child process (so even a region of a few
-    milliseconds gets samples, whatever the launching thread does), else
-    nvidia-smi at its fastest interval.  Read-only."""
+    polled back to back by a child process (so even a region of a few
+    milliseconds gets samples, whatever the launching thread does), each
+    sample time-stamped so that only those inside the region [t0, t1] the
+    caller marks are summarised; else nvidia-smi at its fastest interval.
+    Read-only."""
 
     # NVML clock-event reason bits
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -120,8 +122,9 @@ class ClockSampler:
         self.idx = device_index
         self.proc = None
         self.source = None
-        self.samples = []  # (sm MHz, reason bits)
+        self.samples = []  # (wall time or None, sm MHz, reason bits)
         self.smax = None
+        self.region = None  # (t0, t1) of the timed region, wall clock
 
     def _device_key(self):
         try:  # the same GPU as torch's device, whatever CUDA_VISIBLE_DEVICES says
@@ -168,24 +171,29 @@ class ClockSampler:
         for line in (out or "").splitlines():
             try:
                 if self.source == "nvml":
-                    mhz, bits = line.split()
-                    self.samples.append((float(mhz), int(bits)))
+                    t, mhz, bits = line.split()
+                    self.samples.append((float(t), float(mhz), int(bits)))
                 else:
                     parts = [p.strip() for p in line.split(",")]
-                    self.samples.append((float(parts[0]), int(parts[2], 16)))
+                    self.samples.append((None, float(parts[0]), int(parts[2], 16)))
                     self.smax = float(parts[1])
             except (ValueError, IndexError):
                 continue
 
     def summary(self):
-        load = [(mhz, r) for mhz, r in self.samples if not (r & 0x1)]  # not GPU-idle
-        use = load or self.samples
+        inside = self.samples
+        if self.region is not None and self.source == "nvml":
+            t0, t1 = self.region
+            inside = [s_ for s_ in self.samples if t0 <= s_[0] <= t1]
+        pairs = [(mhz, r) for _, mhz, r in inside]
+        load = [(mhz, r) for mhz, r in pairs if not (r & 0x1)]  # not GPU-idle
+        use = load or pairs
         if not use:
             return {"sm_mhz": None, "sm_max_mhz": self.smax, "reasons": [], "samples": 0,
                     "source": self.source}
         reasons = sorted({n for _, r in use for bit, n in self.REASONS.items() if r & bit})
         return {"sm_mhz": statistics.median(m for m, _ in use), "sm_max_mhz": self.smax,
-                "reasons": reasons, "samples": len(self.samples), "samples_under_load": len(load),
+                "reasons": reasons, "samples": len(pairs), "samples_under_load": len(load),
                 "source": self.source}
 
 
@@ -369,12 +377,14 @@ def time_launches(step, flush, stream, steps, warmup, dev, world=1):
     torch.cuda.synchronize(dev)
     with ClockSampler(torch.cuda.current_device()) as clk:
         t_wall = time.perf_counter()
+        r0 = time.time()
         for i in range(steps):
             flush.zero_()
             starts[i].record(stream)
             step()
             ends[i].record(stream)
         torch.cuda.synchronize(dev)
+        clk.region = (r0, time.time())
         t_wall = time.perf_counter() - t_wall
     barrier(world)
     tb.check_status(stream)

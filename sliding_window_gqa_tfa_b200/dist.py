@@ -132,11 +132,12 @@ def run_slices(run: Run, G: int):
             (slice(run.b0, run.b0 + run.nb), slice(run.g0, run.g0 + run.ng)))
 
 
-def sharded_prefill(q, k, v, out, world: int, rank: int, *, key_mask=None, **kw):
+def sharded_prefill(q, k, v, out, world: int, rank: int, *, key_mask=None, sinks=None, **kw):
     """This rank's share of one attention call: for each of its runs, the
     library's ordinary call on the slices (q, out: [B, Hq, L, D]; k, v:
-    [B, Hkv, S, D]; key_mask [B, S]).  Writes only this rank's rows of `out`.
-    Keyword arguments go to binding.prefill (scale, causal, window, stream, ...)."""
+    [B, Hkv, S, D]; key_mask [B, S]; sinks [Hq]).  Writes only this rank's rows
+    of `out`.  Other keyword arguments go to binding.prefill (scale, causal,
+    window, softcap, stream, ...)."""
     from . import binding
 
     B, Hq = q.shape[0], q.shape[1]
@@ -145,7 +146,8 @@ def sharded_prefill(q, k, v, out, world: int, rank: int, *, key_mask=None, **kw)
     for run in rank_runs(B, Hkv, world, rank):
         (qb, qh), (kb, kh) = run_slices(run, G)
         binding.prefill(q[qb, qh], k[kb, kh], v[kb, kh], out=out[qb, qh],
-                        key_mask=key_mask[qb] if key_mask is not None else None, **kw)
+                        key_mask=key_mask[qb] if key_mask is not None else None,
+                        sinks=sinks[qh] if sinks is not None else None, **kw)
     return out
 
 
