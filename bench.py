@@ -101,14 +101,18 @@ out = []
 t_end = time.time() + 600
 while not stop and time.time() < t_end:
     t = time.time()
-    out.append("%.6f %d %d" % (t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get(h))))
+    try:
+        out.append("%.6f %d %d" % (t, pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM), int(get(h))))
+    except Exception:
+        pass  # a failed query costs one sample, not the record
+    time.sleep(0.0002)
 print(chr(10).join(out), flush=True)
 """
 
 
 class ClockSampler:
     """SM clock and throttle reasons sampled during the timed region: NVML
-    polled back to back by a child process (so even a region of a few
+    polled every ~0.2 ms by a child process (so even a region of a few
     milliseconds gets samples, whatever the launching thread does), each
     sample time-stamped so that only those inside the region [t0, t1] the
     caller marks are summarised; else nvidia-smi at its fastest interval.
