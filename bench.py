@@ -186,9 +186,16 @@ class ClockSampler:
 
     def summary(self):
         inside = self.samples
+        bracketing = False
         if self.region is not None and self.source == "nvml":
             t0, t1 = self.region
             inside = [s_ for s_ in self.samples if t0 <= s_[0] <= t1]
+            if not inside:  # one slow NVML query can span a region of a few ms:
+                # the samples just before and after it stand in, and the line says so
+                before = [s_ for s_ in self.samples if s_[0] < t0]
+                after = [s_ for s_ in self.samples if s_[0] > t1]
+                inside = before[-1:] + after[:1]
+                bracketing = bool(inside)
         pairs = [(mhz, r) for _, mhz, r in inside]
         load = [(mhz, r) for mhz, r in pairs if not (r & 0x1)]  # not GPU-idle
         use = load or pairs
@@ -196,9 +203,12 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": self.smax, "reasons": [], "samples": 0,
                     "source": self.source}
         reasons = sorted({n for _, r in use for bit, n in self.REASONS.items() if r & bit})
-        return {"sm_mhz": statistics.median(m for m, _ in use), "sm_max_mhz": self.smax,
-                "reasons": reasons, "samples": len(pairs), "samples_under_load": len(load),
-                "source": self.source}
+        out = {"sm_mhz": statistics.median(m for m, _ in use), "sm_max_mhz": self.smax,
+               "reasons": reasons, "samples": len(pairs), "samples_under_load": len(load),
+               "source": self.source}
+        if bracketing:
+            out["bracketing_samples"] = True  # none fell inside the timed region itself
+        return out
 
 
 def cpu_threads():

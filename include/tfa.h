@@ -261,10 +261,7 @@ int tfa_prefill_backward_saved(const void *q, const void *k, const void *v, cons
                                       cycles instead of ~4 s, to exercise the give-up path: the
                                       waits run out, the kernel drains its copies and tensor-core
                                       work, the output is invalid and tfa_check_status (or
-                                      TFA_DEBUG_SYNC) returns TFA_ERR_TIMEOUT.  Refused with
-                                      TFA_ERR_FLAGS for L <= 128 (packed tiles, whose merge joins
-                                      a whole warpgroup at a barrier that a warp which gave up
-                                      early would never reach). */
+                                      TFA_DEBUG_SYNC) returns TFA_ERR_TIMEOUT. */
 
 /* tfa_prefill_debug -- tfa_prefill with debug flags (arguments as above).  With
  * NO_TILE_SKIP and/or MASK_ALL the result must be bit-identical to tfa_prefill's

@@ -467,8 +467,6 @@ int prefill_impl(const void *q, const void *k, const void *v, void *o, int B, in
                   TFA_DEBUG_FORCE_SPLIT | TFA_DEBUG_SHORT_WAITS) ||
         ((flags & TFA_DEBUG_NO_SPLIT) && (flags & TFA_DEBUG_FORCE_SPLIT)))
         return TFA_ERR_FLAGS;
-    // packed tiles (L <= 128) merge at warpgroup barriers that an early give-up could leave waiting
-    if ((flags & TFA_DEBUG_SHORT_WAITS) && L <= tfa::kBlockQ) return TFA_ERR_FLAGS;
     const bool force_split = (flags & TFA_DEBUG_FORCE_SPLIT) != 0;
     DeviceState *st = nullptr;
     SplitScratch *ss = nullptr;

@@ -103,7 +103,7 @@ struct Cfg {
     // request that shared memory at all (it would shrink the L1 carve-out).
     static constexpr int kBiasBytes = 128 * 16 * 2;
     static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-    static constexpr int kNumBars = 10 + 2 * kSlots + 1 + 4 + 2;
+    static constexpr int kNumBars = 10 + 2 * kSlots + 1 + 4 + 2 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;
     static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base to 1 KB
     static constexpr int kBiasOff = ((kMiscOff + 16 + 1023) / 1024) * 1024;
@@ -272,6 +272,8 @@ struct Bars {
     // P_t's first kPartKeys key columns are in tensor memory (the P.V product
     // may start on them while the softmax finishes the rest)
     __device__ __forceinline__ uint32_t p_part(int t) const { return base + 8 * (15 + 2 * slots + t); }
+    // packed tiles: one step of a finalizer's merge, the four warps of tile 0 arriving
+    __device__ __forceinline__ uint32_t merge_step() const { return base + 8 * (17 + 2 * slots); }
 };
 
 // ------------------------------------------------------------------ producer
@@ -592,87 +594,64 @@ __device__ __forceinline__ float add_sink(const Params &p, float l, float m, flo
 // per-row log-sum-exp written beside the output (for a backward pass).
 enum ScoreMode : int { kModePlain = 0, kModeSoftcap = 1, kModeLse = 2 };
 
-// Finalizer of a cut packed (short-query) tile, run by all 128 threads of
-// the tile's warpgroup once every row has stored its own partial in this
-// CTA's second slot (the first may still hold the partial this CTA published
-// for an earlier tile; a packed piece has no second query tile): the merge of all the tile's partials (tiny-llm Week 2 Day 5,
-// Task 1: m* = max m_k, l* = sum 2^(m_k - m*) l_k, a* = sum 2^(m_k - m*) a_k,
-// O = a* / l*), written straight to the output.  A packed tile has few live
-// rows but one partial per CTA of its key range, so the threads split the
-// flag waits and the (row, 4-column) elements between them instead of one
-// thread walking every partial of its row.  Returns false on an abort.
+// Finalizer of a cut packed (short-query) tile, run by the 128 threads of
+// tile 0's warpgroup once each has stored its row of the finalizer's own
+// partial in this CTA's second slot (the first may still hold the partial
+// this CTA published for an earlier tile): the merge of all the tile's
+// partials (tiny-llm Week 2 Day 5, Task 1: m* = max m_k,
+// l* = sum 2^(m_k - m*) l_k, a* = sum 2^(m_k - m*) a_k, O = a* / l*),
+// written straight to the output.  A packed tile has few live rows but one
+// partial per CTA of its key range, so the threads split the flag waits and
+// the (row, 4-column) elements between them instead of one thread walking
+// every partial of its row; each thread merges its elements' statistics
+// itself, batch by batch with the same equations (one L2 round trip per
+// batch of partials, no step between statistics and elements).  The threads
+// meet once, after the flag waits, at an mbarrier with bounded waits (never a
+// named barrier: a warp that gave up early must not leave the others
+// waiting).  `steps` counts the merge_step phases this thread has passed.
+// Returns false on an abort.
 template <int D, int MODE>
 __device__ __forceinline__ bool merge_packed(const Params &p, const Segment &seg, const ItemSpan &sp,
-                                          int t, int n_valid, unsigned epoch, volatile int *abort_flag) {
-    using C = Cfg<D>;
-    const int r = threadIdx.x - t * 128;
+                                          int n_valid, unsigned epoch, volatile int *abort_flag,
+                                          const Bars &bar, uint32_t &steps) {
+    constexpr int kN = 128;  // merging threads
+    const int r = threadIdx.x;
+    const int lane = threadIdx.x & 31;
     const float c = p.scale_log2;
-    const int c_last = last_contributor(p.W, gridDim.x, blockIdx.x, seg, sp, t);
+    const int c_last = last_contributor(p.W, gridDim.x, blockIdx.x, seg, sp, 0);
 #ifdef TFA_TRACE
     if (r == 0 && blockIdx.x < 1024) g_tfa_cta_time[blockIdx.x][3] = globaltimer_ns();
 #endif
-    bool ok = true;
-    for (int k = blockIdx.x + 1 + r; k <= c_last && ok; k += 128)
-        ok = flag_wait(p.ready + partial_slot(k, t), epoch, abort_flag, p.status, p.wait_limit);
-    // the slot writes of this warpgroup and the flags seen by it are ordered
-    // before every read below; all threads leave together on an abort
-    if (named_barrier_or(1 + t, 128, !ok || *abort_flag)) return false;
+    for (int k = blockIdx.x + 1 + r; k <= c_last; k += kN)
+        if (!flag_wait(p.ready + partial_slot(k, 0), epoch, abort_flag, p.status, p.wait_limit)) break;
+    // every warp arrives, then every lane waits (bounded): the slot writes of
+    // tile 0's warps and the flags seen here are ordered before every read
+    // below; all threads leave together on an abort, a timed-out wait raising it
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar.merge_step());
+    const bool met = __all_sync(0xffffffffu, mbar_wait(bar.merge_step(), steps & 1, abort_flag, p.status,
+                                                       p.wait_limit));
+    ++steps;
+    if (!met || *abort_flag) return false;
     auto slot_of = [&](int k) {
         return p.partial +
-               static_cast<size_t>(partial_slot(k, k == static_cast<int>(blockIdx.x) ? 1 : t)) * partial_slot_floats<D>();
+               static_cast<size_t>(partial_slot(k, k == static_cast<int>(blockIdx.x) ? 1 : 0)) * partial_slot_floats<D>();
     };
-    // Q tile 1's buffer: a packed piece never loads a second query tile
-    float *ms = reinterpret_cast<float *>(smem_base() + C::kQOff + C::kTileBytes);
     const PackedRows pr = packed_rows(p, seg.h);
-    if (r < n_valid) {
-        // batches of 16 partials: the loads of a batch are independent and in
-        // flight together, the combine is branch-free
-        constexpr int kBatch = 16;
-        float m = -CUDART_INF_F, l = 0.f;
-        for (int k0 = blockIdx.x; k0 <= c_last; k0 += kBatch) {
-            float mk[kBatch], lk[kBatch];
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u) {
-                const bool in = k0 + u <= c_last;
-                const float *sl = slot_of(in ? k0 + u : k0);
-                mk[u] = in ? __ldcg(sl + 128 * D + r) : -CUDART_INF_F;
-                lk[u] = in ? __ldcg(sl + 128 * D + 128 + r) : 0.f;
-            }
-            float mb = mk[0];
-#pragma unroll
-            for (int u = 1; u < kBatch; ++u) mb = fmaxf(mb, mk[u]);
-            const float mn = fmaxf(m, mb);
-            const float mnc = (mn == -CUDART_INF_F) ? 0.f : mn * c;  // an empty row keeps l = 0
-            float lb = (m == -CUDART_INF_F) ? 0.f : l * ex2(fmaf(m, c, -mnc));
-#pragma unroll
-            for (int u = 0; u < kBatch; ++u)
-                lb = fmaf(lk[u], (mk[u] == -CUDART_INF_F) ? 0.f : ex2(fmaf(mk[u], c, -mnc)), lb);
-            m = mn;
-            l = lb;
-        }
-        const int head = pr.h0 + r / p.L, row = r % p.L;
-        l = add_sink(p, l, m, c, head);
-        if constexpr (MODE == kModeLse)
-            p.lse[static_cast<size_t>(seg.b * p.Hq + head) * p.L + row] =
-                l > 0.f ? fmaf(m, c, __log2f(l)) : CUDART_INF_F;
-        ms[r] = m;
-        ms[128 + r] = l > 0.f ? 1.f / l : 0.f;
-    }
-    named_barrier(1 + t, 128);
     constexpr int kC4 = D / 4;  // float4 columns per row
     const int n4 = n_valid * kC4;
-    for (int e0 = r; e0 < n4; e0 += 256) {  // two elements per thread per pass
-        const int e1 = e0 + 128;
+    for (int e0 = r; e0 < n4; e0 += 2 * kN) {  // two elements per thread per pass
+        const int e1 = e0 + kN;
         const bool has1 = e1 < n4;
         const int row0 = e0 / kC4, row1 = has1 ? e1 / kC4 : row0;
         const int c40 = e0 - row0 * kC4, c41 = has1 ? e1 - row1 * kC4 : c40;
-        const float m0 = ms[row0], m1 = ms[row1];
+        float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
         float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
         // batches of partials, loads predicated (not a remainder loop) so that
         // a batch's loads are all in flight together however few there are
         constexpr int kBatch = 8;
         for (int k0 = blockIdx.x; k0 <= c_last; k0 += kBatch) {
-            float mk0[kBatch], mk1[kBatch];
+            float mk0[kBatch], mk1[kBatch], lk0[kBatch], lk1[kBatch];
             float4 v0[kBatch], v1[kBatch];
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
@@ -680,37 +659,52 @@ __device__ __forceinline__ bool merge_packed(const Params &p, const Segment &seg
                 const float *sl = slot_of(in ? k0 + u : k0);
                 mk0[u] = in ? __ldcg(sl + 128 * D + row0) : -CUDART_INF_F;
                 mk1[u] = in ? __ldcg(sl + 128 * D + row1) : -CUDART_INF_F;
+                lk0[u] = in ? __ldcg(sl + 128 * D + 128 + row0) : 0.f;
+                lk1[u] = in ? __ldcg(sl + 128 * D + 128 + row1) : 0.f;
                 v0[u] = __ldcg(reinterpret_cast<const float4 *>(sl + row0 * D) + c40);
                 v1[u] = __ldcg(reinterpret_cast<const float4 *>(sl + row1 * D) + c41);
             }
+            float mb0 = m0, mb1 = m1;
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) mb0 = fmaxf(mb0, mk0[u]), mb1 = fmaxf(mb1, mk1[u]);
+            // an empty row (every m -inf) keeps l = 0 and a = 0
+            const float nb0 = (mb0 == -CUDART_INF_F) ? 0.f : mb0 * c, nb1 = (mb1 == -CUDART_INF_F) ? 0.f : mb1 * c;
+            const float g0 = (m0 == -CUDART_INF_F) ? 0.f : ex2(fmaf(m0, c, -nb0));
+            const float g1 = (m1 == -CUDART_INF_F) ? 0.f : ex2(fmaf(m1, c, -nb1));
+            l0 *= g0, l1 *= g1;
+            a0.x *= g0, a0.y *= g0, a0.z *= g0, a0.w *= g0;
+            a1.x *= g1, a1.y *= g1, a1.z *= g1, a1.w *= g1;
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
-                const float f0 = (mk0[u] == -CUDART_INF_F) ? 0.f : ex2((mk0[u] - m0) * c);
-                const float f1 = (mk1[u] == -CUDART_INF_F) ? 0.f : ex2((mk1[u] - m1) * c);
+                const float f0 = (mk0[u] == -CUDART_INF_F) ? 0.f : ex2(fmaf(mk0[u], c, -nb0));
+                const float f1 = (mk1[u] == -CUDART_INF_F) ? 0.f : ex2(fmaf(mk1[u], c, -nb1));
+                l0 = fmaf(f0, lk0[u], l0), l1 = fmaf(f1, lk1[u], l1);
                 a0.x = fmaf(f0, v0[u].x, a0.x), a0.y = fmaf(f0, v0[u].y, a0.y);
                 a0.z = fmaf(f0, v0[u].z, a0.z), a0.w = fmaf(f0, v0[u].w, a0.w);
                 a1.x = fmaf(f1, v1[u].x, a1.x), a1.y = fmaf(f1, v1[u].y, a1.y);
                 a1.z = fmaf(f1, v1[u].z, a1.z), a1.w = fmaf(f1, v1[u].w, a1.w);
             }
+            m0 = mb0, m1 = mb1;
         }
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
             if (u == 1 && !has1) break;
             const int rr = u ? row1 : row0, c4 = u ? c41 : c40;
             const float4 a = u ? a1 : a0;
-            const float inv = ms[128 + rr];
             const int head = pr.h0 + rr / p.L, row = rr % p.L;
+            const float m = u ? m1 : m0;
+            const float l = add_sink(p, u ? l1 : l0, m, c, head);
+            if (MODE == kModeLse && c4 == 0)
+                p.lse[static_cast<size_t>(seg.b * p.Hq + head) * p.L + row] =
+                    l > 0.f ? fmaf(m, c, __log2f(l)) : CUDART_INF_F;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
             __nv_bfloat16 *orow = p.o + (static_cast<size_t>(seg.b * p.Hq + head) * p.L + row) * D;
             *reinterpret_cast<uint2 *>(orow + 4 * c4) = make_uint2(pack_bf16(a.x * inv, a.y * inv),
                                                                   pack_bf16(a.z * inv, a.w * inv));
         }
     }
-    // the next piece may overwrite the scratch row maxima only after every
-    // thread has read them
-    named_barrier(1 + t, 128);
     return true;
 }
-
 
 template <int D, bool KM, int MODE, int LY, bool PK>
 __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint32_t tmem,
@@ -726,6 +720,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
     const int lane = threadIdx.x & 31;
     uint32_t s_cnt = 0, o_cnt = 0, pub_cnt = 0, fin_cnt = 0;
     uint32_t s_cnt0 = 0, s_cnt1 = 0, pv_cnt = 0;  // short-query tiles: per S buffer, P.V done
+    uint32_t merge_steps = 0;                      // short-query tiles: merge steps passed
     const unsigned epoch = p.ctl ? launch_epoch(p.ctl) : 0u;
     int trace_step = 0;
     (void)trace_step;
@@ -946,7 +941,7 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
                 }
             }
             if (PK && ip.finalizer) {
-                if (!merge_packed<D, MODE>(p, seg, sp, t, n_valid, epoch, abort_flag)) return;
+                if (!merge_packed<D, MODE>(p, seg, sp, n_valid, epoch, abort_flag, bar, merge_steps)) return;
                 continue;
             }
             __syncwarp();
@@ -1081,6 +1076,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar.fin(t), 1);
             mbar_init(bar.p_part(t), 4);
         }
+        mbar_init(bar.merge_step(), 4);
         *abort_flag = 0;
         fence_barrier_init();
     }

@@ -248,24 +248,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
 }
 #undef TFA_W8
 
-// Named barrier `id` (1..15) over `n` threads (a multiple of 32).
-__device__ __forceinline__ void named_barrier(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-// Named barrier that also ORs `pred` over its threads: every thread gets the
-// same answer.
-__device__ __forceinline__ bool named_barrier_or(int id, int n, bool pred) {
-    unsigned out;
-    asm volatile(
-        "{\n\t.reg .pred pi, po;\n\t"
-        "setp.ne.u32 pi, %1, 0;\n\t"
-        "bar.red.or.pred po, %2, %3, pi;\n\t"
-        "selp.u32 %0, 1, 0, po;\n\t}"
-        : "=r"(out)
-        : "r"(pred ? 1u : 0u), "r"(id), "r"(n)
-        : "memory");
-    return out != 0u;
-}
 // GPU-scope publication / observation of a flag in global memory.
 __device__ __forceinline__ void st_release_gpu(unsigned *addr, unsigned v) {
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");

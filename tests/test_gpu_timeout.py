@@ -29,11 +29,15 @@ def _close(got, ref):
     assert np.all(np.abs(got - ref) <= ATOL + RTOL * np.abs(ref))
 
 
-@pytest.mark.parametrize("flags", [0, tb.TFA_DEBUG_FORCE_SPLIT, tb.TFA_DEBUG_NO_SPLIT],
-                         ids=["default", "split", "whole_items"])
-def test_short_waits_give_up_and_the_next_call_is_clean(flags):
-    # L > 128: unpacked query tiles (packed ones refuse the flag)
-    w = shaped(1, 8, 2, 300, 700, 128)
+@pytest.mark.parametrize("L,S,flags", [
+    (300, 700, 0), (300, 700, tb.TFA_DEBUG_FORCE_SPLIT), (300, 700, tb.TFA_DEBUG_NO_SPLIT),
+    (33, 4000, 0), (33, 4000, tb.TFA_DEBUG_FORCE_SPLIT),
+], ids=["default", "split", "whole_items", "packed", "packed_split"])
+def test_short_waits_give_up_and_the_next_call_is_clean(L, S, flags):
+    # L = 300: 128-row query tiles; L = 33: packed tiles (up to three of a KV
+    # group's four query heads per tile), whose split key ranges end in the
+    # merge that both softmax warpgroups share
+    w = shaped(1, 8, 2, L, S, 128)
     q, k, v, _ = make_inputs(w, seed=21)
     dq, dk, dv = q.cuda(), k.cuda(), v.cuda()
     ref = oracle.attention(q, k, v, scale=w.softmax_scale, causal=True)

@@ -117,13 +117,6 @@ def test_varlen_rejections_happen_before_launch():
     assert tb.tfa_prefill_varlen(**{**a, "softcap": float("inf")}) == tb.TFA_ERR_SOFTCAP
 
 
-def test_short_waits_are_refused_for_packed_tiles_before_launch():
-    # L <= 128 runs packed tiles, whose merge a warp that gave up early could stall
-    for L in (9, 33, 128):
-        assert tb.tfa_prefill_debug(A16, A16, A16, A16, 1, 8, 2, L, 300, 128, 0.1, 1, 0, None, None,
-                                    tb.TFA_DEBUG_SHORT_WAITS) == tb.TFA_ERR_FLAGS
-
-
 def test_debug_rejects_unknown_flags_before_launch():
     assert tb.tfa_prefill_debug(A16, A16, A16, A16, 1, 8, 2, 33, 47, 128, 0.1, 1, 0, None, None,
                                 64) == tb.TFA_ERR_FLAGS
