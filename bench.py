@@ -40,8 +40,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from sliding_window_gqa_tfa_b200 import binding as tb  # noqa: E402
-from sliding_window_gqa_tfa_b200.dist import (barrier, max_over_ranks, rank_runs,  # noqa: E402
-                                              run_slices, setup, teardown)
+from sliding_window_gqa_tfa_b200.dist import (Run, barrier, max_over_ranks,  # noqa: E402
+                                              rank_runs, run_slices, setup, teardown)
 from sliding_window_gqa_tfa_b200.flops import workload_bytes, workload_flops  # noqa: E402
 from sliding_window_gqa_tfa_b200.inputs import (HEADLINE, WORKLOADS, make_dout,  # noqa: E402
                                                 make_inputs, make_sinks, sample_rows, varlen_cu)
@@ -434,6 +434,17 @@ def per_config(args, dev, flush, stream, peaks):
     return res
 
 
+def bench_runs(w, world, rank, strong):
+    """The runs (dist.Run, element indices local to this rank's tensors) a rank
+    launches per step.  Strong: its share of the workload's own B x Hkv units
+    (every rank holds the whole call's inputs).  Weak: a call of world x B
+    elements whose share for this rank is exactly its own B elements (its own
+    inputs), so the runs are shifted to local element indices."""
+    if strong:
+        return rank_runs(w.B, w.Hkv, world, rank)
+    return [Run(r_.b0 - rank * w.B, r_.nb, r_.g0, r_.ng) for r_ in rank_runs(world * w.B, w.Hkv, world, rank)]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -485,11 +496,7 @@ def main():
         out = torch.empty_like(dev_inputs[0])
     G = w.Hq // w.Hkv
     if w.kind == "dense":
-        if strong:  # this rank's units of the workload's own call
-            runs = rank_runs(w.B, w.Hkv, world, rank)
-        else:  # a call of world x B elements: this rank's units are its own B elements
-            runs = [r_.__class__(r_.b0 - rank * w.B, r_.nb, r_.g0, r_.ng)
-                    for r_ in rank_runs(world * w.B, w.Hkv, world, rank)]
+        runs = bench_runs(w, world, rank, strong)
         flops = sum(workload_flops(w.with_(B=r_.nb, Hq=r_.ng * G, Hkv=r_.ng),
                                    key_mask=km[r_.b0:r_.b0 + r_.nb] if km is not None else None)
                     for r_ in runs)

@@ -136,3 +136,23 @@ def test_sharded_call_all_gathered_equals_the_whole_call(world, case):
         own_only, err = out[r]
         assert own_only  # before the gather a rank wrote its own planes and nothing else
         assert err == 0.0  # rows are independent: the slices give the whole result bit for bit
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 8])
+def test_bench_runs_weak_and_strong(world):
+    import bench
+
+    for w in (WORKLOADS["llama_gqa_chunk_2048x8192"], WORKLOADS["qwen3_prefill_b4_2048"]):
+        G = w.Hq // w.Hkv
+        strong_units = []
+        for rank in range(world):
+            # weak: every rank runs exactly its own copy of the workload
+            weak = bench.bench_runs(w, world, rank, strong=False)
+            units = [(r_.b0 + i, r_.g0 + j) for r_ in weak for i in range(r_.nb) for j in range(r_.ng)]
+            assert units == [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+            # strong: the ranks share the workload's own units
+            for r_ in bench.bench_runs(w, world, rank, strong=True):
+                (qb, qh), (kb, kh) = tdist.run_slices(r_, G)
+                assert qh.stop - qh.start == G * (kh.stop - kh.start)
+                strong_units += [(r_.b0 + i, r_.g0 + j) for i in range(r_.nb) for j in range(r_.ng)]
+        assert strong_units == [(b, g) for b in range(w.B) for g in range(w.Hkv)]
