@@ -292,6 +292,10 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
     uint32_t q_use[2] = {0, 0};
     SegIter it;
     iter_init<D, LY>(it, p);
+    // K/V tiles are read again by the other CTAs of their KV group (and the
+    // other query tiles); Q tiles are read once.  Marking them evict-last /
+    // evict-first keeps K/V in L2 while Q and O stream through it.
+    const uint64_t pol_kv = make_policy_evict_last(), pol_q = make_policy_evict_first();
     Segment seg;
     while (it.next(p.shape, seg)) {
         const ItemPlan ip = plan_piece<PK>(p, seg);
@@ -306,14 +310,14 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                     const PackedRows pr = packed_rows(p, ip.h);
                     mbar_arrive_expect_tx(bar.q_full(t), C::kColBlocks * 128 * p.L * p.pack_heads);
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
-                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
-                                    tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0);
+                        tma_load_3d_hint(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
+                                         tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0, pol_q);
                 } else {  // dense: plane b*Hq + h; varlen: packed rows, plane h
                     mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
                     const int plane = LY == kLayoutVarlen ? ip.h : ip.b * p.Hq + ip.h;
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
-                        tma_load_3d(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
-                                    tm_q, bar.q_full(t), cb * 64, ip.q_row0 + ip.q0[t], plane);
+                        tma_load_3d_hint(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
+                                         tm_q, bar.q_full(t), cb * 64, ip.q_row0 + ip.q0[t], plane, pol_q);
                 }
             }
             ++q_use[t];
@@ -348,14 +352,14 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                         for (int hf = 0; hf < 2; ++hf) {
                             const int row = (j * kBlockK + 64 * hf) % p.ring_rows;
                             for (int cb = 0; cb < C::kColBlocks; ++cb)
-                                tma_load_3d(dst + cb * C::kColBlockBytes + hf * 64 * 128, which ? tm_v : tm_k,
-                                            bar.kv_full(s), cb * 64, row, ip.b * p.Hkv + ip.g);
+                                tma_load_3d_hint(dst + cb * C::kColBlockBytes + hf * 64 * 128, which ? tm_v : tm_k,
+                                                 bar.kv_full(s), cb * 64, row, ip.b * p.Hkv + ip.g, pol_kv);
                         }
                     } else {
                         const int plane = LY == kLayoutVarlen ? ip.g : ip.b * p.Hkv + ip.g;
                         for (int cb = 0; cb < C::kColBlocks; ++cb)
-                            tma_load_3d(dst + cb * C::kColBlockBytes, which ? tm_v : tm_k, bar.kv_full(s),
-                                        cb * 64, ip.k_row0 + j * kBlockK, plane);
+                            tma_load_3d_hint(dst + cb * C::kColBlockBytes, which ? tm_v : tm_k, bar.kv_full(s),
+                                             cb * 64, ip.k_row0 + j * kBlockK, plane, pol_kv);
                     }
                 }
                 ++kv_prod;
