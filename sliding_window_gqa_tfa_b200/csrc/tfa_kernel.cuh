@@ -113,7 +113,10 @@ struct Cfg {
     // k_len (validated copies of cu_seqlens), in place of the key-mask blocks
     // (the two never meet).
     static constexpr int kTableOff = kBiasOff;
-    static constexpr int kSmemBytesVarlen = kTableOff + 16 * kMaxVarlenSeqs + 1024;
+    // then the sorted sequence order and the group starts of the compact deal
+    static constexpr int kOrderOff = kTableOff + 16 * kMaxVarlenSeqs;
+    static constexpr int kGroupStartOff = kOrderOff + 4 * kMaxVarlenSeqs;
+    static constexpr int kSmemBytesVarlen = kGroupStartOff + 4 * (kMaxVarlenGroups + 1) + 1024;
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kTmemS = 0;                 // S_t at kTmemS + 128 t
     static constexpr uint32_t kTmemO = 256;               // O_t at kTmemO + D t
@@ -216,6 +219,11 @@ __device__ __forceinline__ void iter_init(SegIter &it, const Params &p) {
         it.seq.q_len = tab + kMaxVarlenSeqs;
         it.seq.k_start = tab + 2 * kMaxVarlenSeqs;
         it.seq.k_len = tab + 3 * kMaxVarlenSeqs;
+        if (p.shape.n_qp <= kMaxVarlenGroups) {
+            it.seq.order = reinterpret_cast<const unsigned *>(smem_base() + Cfg<D>::kOrderOff);
+            it.seq.group_start = reinterpret_cast<const int *>(smem_base() + Cfg<D>::kGroupStartOff);
+            it.n_items = it.seq.group_start[p.shape.n_qp];
+        }
     }
 }
 
@@ -1111,6 +1119,70 @@ __global__ void __launch_bounds__(kThreads, 1)
             tab[2 * kMaxVarlenSeqs + b] = k0;
             tab[3 * kMaxVarlenSeqs + b] = k1 - k0;
             if (!ok && blockIdx.x == 0) atomicOr(p.status, TFA_DEVICE_BAD_SEQLENS);
+        }
+    }
+    if (LY == kLayoutVarlen && p.shape.n_qp <= kMaxVarlenGroups) {
+        // The compact deal (the same in every CTA): sequences sorted by their
+        // query-tile pairs, longest first, by a bitonic sort of unique keys
+        // (pairs << 10 | 1023 - b) over all threads, then per group the items
+        // that exist and their prefix sums.  Without it a CTA's share of the
+        // item grid would hold empty slots where short sequences end.
+        __syncthreads();  // the table is complete
+        const int *tab = reinterpret_cast<const int *>(gbase + C::kTableOff);
+        unsigned *order = reinterpret_cast<unsigned *>(gbase + C::kOrderOff);
+        int *gstart = reinterpret_cast<int *>(gbase + C::kGroupStartOff);
+        int n = 1;
+        while (n < p.B) n <<= 1;
+        for (int i = threadIdx.x; i < n; i += kThreads) {
+            const int pairs = i < p.B ? (tab[kMaxVarlenSeqs + i] + 2 * kBlockQ - 1) / (2 * kBlockQ) : 0;
+            order[i] = i < p.B ? (static_cast<unsigned>(pairs) << 10) | static_cast<unsigned>(1023 - i) : 0u;
+        }
+        __syncthreads();
+        for (int k = 2; k <= n; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int i = threadIdx.x; i < n; i += kThreads) {
+                    const int l = i ^ j;
+                    if (l > i) {
+                        const unsigned a = order[i], b = order[l];
+                        if ((i & k) == 0 ? a < b : a > b) {  // decreasing overall
+                            order[i] = b;
+                            order[l] = a;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        const int n_qp = p.shape.n_qp;
+        for (int rr = threadIdx.x; rr < n_qp; rr += kThreads) {
+            // sequences with query-tile pair qp: those with more than qp pairs
+            const unsigned bound = static_cast<unsigned>(group_qp(p.shape, rr) + 1) << 10;
+            int lo = 0, hi = p.B;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (order[mid] >= bound) lo = mid + 1;
+                else hi = mid;
+            }
+            gstart[rr + 1] = lo * p.Hq;
+        }
+        if (threadIdx.x == 0) gstart[0] = 0;
+        __syncthreads();
+        if (warp == 0) {  // prefix sums over the groups, a chunk per lane
+            const int per = (n_qp + 31) / 32;
+            const int a0 = 1 + lane * per, a1 = imin(a0 + per, n_qp + 1);
+            int sum = 0;
+            for (int i = a0; i < a1; ++i) sum += gstart[i];
+            int incl = sum;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            int run = incl - sum;
+            for (int i = a0; i < a1; ++i) {
+                run += gstart[i];
+                gstart[i] = run;
+            }
         }
     }
     if (warp == 8 && lane == 0) {

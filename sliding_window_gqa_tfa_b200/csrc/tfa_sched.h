@@ -30,8 +30,16 @@ namespace tfa {
 // Packed variable-length batches: sequence b has q_len[b] query rows from
 // packed row q_start[b] and k_len[b] keys from packed row k_start[b] (a
 // sequence whose lengths failed validation has q_len 0 and is skipped).
+// With `order` set, only the items that exist are dealt: order[i] low 10 bits
+// = 1023 - b, high bits = b's query-tile pairs, sorted in decreasing order
+// (longest sequences first, then by index), and group_start[rr] = the items
+// of the groups before group rr (the groups' order as for fixed lengths).
+// Group rr holds, for each of its first n sequences of `order`, every head.
+constexpr int kMaxVarlenGroups = 1024;  // query-tile pairs for the compact deal
 struct SeqTable {
     const int *q_start, *q_len, *k_start, *k_len;
+    const unsigned *order;
+    const int *group_start;
 };
 
 struct Shape {
@@ -115,6 +123,8 @@ struct SegIter {
 
     TFA_HD void init(const Shape &s, long long W, int c) {
         seq.q_start = seq.q_len = seq.k_start = seq.k_len = nullptr;
+        seq.order = nullptr;
+        seq.group_start = nullptr;
         bh = s.B * s.Hq;
         n_items = s.n_qp * bh;
         item = c;
@@ -137,11 +147,24 @@ struct SegIter {
         if (!s.split) {
             for (;;) {
                 if (item >= n_items) return false;
-                const int rr = item / bh, rem = item - rr * bh;
+                if (seq.order) {  // varlen, existing items only
+                    int lo = 0, hi = s.n_qp - 1;  // last group starting at or before item
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (seq.group_start[mid] <= item) lo = mid;
+                        else hi = mid - 1;
+                    }
+                    const int idx = item - seq.group_start[lo], bi = idx / s.Hq;
+                    seg.qp = group_qp(s, lo);
+                    seg.b = 1023 - static_cast<int>(seq.order[bi] & 1023u);
+                    seg.h = idx - bi * s.Hq;
+                } else {
+                    const int rr = item / bh, rem = item - rr * bh;
+                    seg.qp = group_qp(s, rr);
+                    seg.b = rem / s.Hq;
+                    seg.h = rem - seg.b * s.Hq;
+                }
                 seg.item = item;
-                seg.qp = group_qp(s, rr);
-                seg.b = rem / s.Hq;
-                seg.h = rem - seg.b * s.Hq;
                 item += stride;
                 stride = 2 * s.grid - stride;
                 seg.L = s.L;

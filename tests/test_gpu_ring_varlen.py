@@ -102,6 +102,13 @@ VARLEN_CASES = [  # name, lengths, (Hq, Hkv, D), causal, window, extras
                         np.random.default_rng(4).integers(0, 300, 64))], (4, 2, 128), True, 0, {}),
     ("softcap_sinks", [(128, 128), (300, 800), (5, 5)], (8, 2, 128), True, 0,
      dict(softcap=10.0, sinks=True)),
+    # the most sequences a call takes: the device-side sort of the compact
+    # item deal runs over all 1024 (lengths 0..299, ties and empty sequences)
+    ("max_seqs", [(int(n), int(n)) for n in np.random.default_rng(5).integers(0, 300, 1024)],
+     (2, 1, 64), True, 0, {}),
+    # a bound beyond the compact deal's group table: the plain item grid
+    ("bound_past_compact_deal", [(300, 300), (1, 40), (700, 900)], (4, 2, 128), True, 0,
+     dict(max_seqlen_q=1024 * 256 + 1)),
 ]
 
 
@@ -114,7 +121,8 @@ def test_varlen_parity(name, lengths, heads, causal, window, extra):
     sinks = torch.linspace(-2.0, 2.0, Hq) if extra.get("sinks") else None
     out = torch.full(q.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
     o = tb.prefill_varlen(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(cq).cuda(),
-                          torch.from_numpy(ck).cuda(), max_seqlen_q=max(L for L, _ in lengths),
+                          torch.from_numpy(ck).cuda(),
+                          max_seqlen_q=extra.get("max_seqlen_q", max(L for L, _ in lengths)),
                           scale=1 / np.sqrt(D), causal=causal, window=window, softcap=softcap,
                           sinks=sinks.cuda() if sinks is not None else None, out=out)
     tb.check_status()
