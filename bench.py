@@ -380,16 +380,20 @@ def oracle_errors(w, o, q, k, v, km):
 
 def time_launches(step, flush, stream, steps, warmup, dev, world=1):
     """Per-launch device times (ms) of `steps` launches after `warmup`, L2 flushed
-    before each, CUDA events on the launching stream; clocks sampled meanwhile."""
-    for _ in range(warmup):
-        flush.zero_()
-        step()
-    tb.check_status(stream)
+    before each, CUDA events on the launching stream; clocks sampled meanwhile.
+    The sampler starts before the warm-up, so that the GPU does not sit idle
+    while it starts between the warm-up and the timed launches (after such a
+    gap the first timed launches ran slower on some boxes); only samples inside
+    the timed region are kept."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
-    barrier(world)
-    torch.cuda.synchronize(dev)
     with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(warmup):
+            flush.zero_()
+            step()
+        tb.check_status(stream)
+        barrier(world)
+        torch.cuda.synchronize(dev)
         t_wall = time.perf_counter()
         r0 = time.time()
         for i in range(steps):
