@@ -104,8 +104,9 @@ typedef enum {
  * Returns TFA_OK or a tfa_status code.
  * Queries of at most 128 rows run through the packed tiles described under
  * tfa_decode (floor(128 / L) query heads of a KV group per tile); longer ones
- * through pairs of 128-row tiles of one head.  The results are the same
- * attention either way. */
+ * through pairs of 128-row tiles of one head, or, for causal calls with short
+ * key ranges and an even number of query heads per KV group, the same
+ * 128-row tile of two heads.  The results are the same attention either way. */
 int tfa_prefill(const void *q, const void *k, const void *v, void *o,
                 int B, int Hq, int Hkv, int L, int S, int D, float scale,
                 int causal, int window, const float *key_mask, tfa_stream_t stream);
@@ -359,9 +360,14 @@ int tfa_plan_ktile(int L, int S, int causal, int window, int ktile, int *qt_lo, 
  * (tfa_prefill's schedule) the concatenated key-tile steps of all such items
  * are cut into `grid` contiguous ranges of almost equal length; a cut item is
  * finished by the piece holding a tile's first key tile, which merges the
- * others' partial softmax statistics.  With split == 0 whole items are dealt
- * in snake order: CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G = grid).
- *   out          10 ints per piece: item, qp, b, h, first key tile, last key
+ * others' partial softmax statistics.  Without bit 0 of split whole items are
+ * dealt in snake order: CTA c takes items c, 2G-1-c, 2G+c, 4G-1-c, ... (G =
+ * grid).  Bit 1 of split (value 2) selects head pairs, as tfa_prefill uses
+ * when Hq / Hkv is even: an item is then one 128-row query tile of query
+ * heads 2h and 2h+1 (h counting pairs, Hq must be even), its two tiles
+ * visiting the same key tiles.
+ *   out          10 ints per piece: item, qp (query-tile pair, or the query
+ *                tile with head pairs), b, h (head, or head pair), first key tile, last key
  *                tile, role of tile 0, role of tile 1 (bit 0 active, bit 1
  *                finalizer, bit 2 complete), and for a finalizer that must
  *                merge, the last CTA contributing to tile 0 / tile 1 (else -1)

@@ -410,8 +410,20 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     sh.window = p.window;
     sh.flags = p.flags;
     sh.n_qp = tfa::shape_n_qp(L);
-    const long long n_items = static_cast<long long>(B) * sh.Hq * sh.n_qp;
     p.W = varlen ? 0 : tfa::total_steps(sh);  // varlen: per-sequence lengths live on the device
+    // Head pairs for causal calls whose items are short (at most 16 key tiles
+    // on average) when a KV group has an even number of query heads: a pair of
+    // consecutive query tiles spends one step on the later tile alone (the
+    // diagonal, or the window's shift), which short items do not amortise;
+    // measured, long items ran slower as head pairs.
+    if (!packed && !varlen && p.causal && (Hq / Hkv) % 2 == 0 &&
+        p.W <= 16LL * B * sh.Hq * sh.n_qp) {
+        sh.hp = 1;
+        sh.Hq = Hq / 2;
+        sh.n_qp = tfa::shape_n_qp(L, 1);
+        p.W = tfa::total_steps(sh);
+    }
+    const long long n_items = static_cast<long long>(B) * sh.Hq * sh.n_qp;
     // whole-item schedule, and the split one when scratch exists and the
     // estimate says it finishes sooner (few, large items per CTA)
     sh.split = 0;
@@ -1038,19 +1050,21 @@ extern "C" int tfa_plan_pieces(int B, int Hq, int L, int S, int causal, int wind
     if (rc) return rc;
     if (!n_pieces || (max_pieces > 0 && !out)) return TFA_ERR_NULL;
     tfa::Shape sh;
+    sh.hp = (split & 2) ? 1 : 0;
+    if (sh.hp && Hq % 2) return TFA_ERR_SHAPE;
     sh.B = B;
-    sh.Hq = Hq;
+    sh.Hq = sh.hp ? Hq / 2 : Hq;
     sh.L = L;
     sh.S = S;
     sh.causal = causal ? 1 : 0;
     sh.window = (causal && window > 0) ? window : 0;
     sh.flags = 0;
-    sh.n_qp = tfa::shape_n_qp(L);
-    sh.split = split ? 1 : 0;
+    sh.n_qp = tfa::shape_n_qp(L, sh.hp);
+    sh.split = (split & 1) ? 1 : 0;
     sh.grid = grid;
     const long long W = tfa::total_steps(sh);
     if (total_steps) *total_steps = W;
-    const long long units = sh.split ? W : static_cast<long long>(B) * Hq * sh.n_qp;
+    const long long units = sh.split ? W : static_cast<long long>(B) * sh.Hq * sh.n_qp;
     if (grid < 1 || grid > units || cta < 0 || cta >= grid) return TFA_ERR_SHAPE;
     tfa::SegIter it;
     it.init(sh, W, cta);

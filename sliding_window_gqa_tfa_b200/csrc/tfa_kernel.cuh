@@ -245,7 +245,7 @@ __device__ __forceinline__ ItemPlan plan_piece(const Params &p, const Segment &s
     // p.packed is tested at run time here and in the producer's Q load (always
     // equal to PK): the compile-time form of these two tests measured ~3 %
     // slower on dense prefill, with identical register and spill counts
-    ip.g = (PK || p.packed) ? seg.h / p.pack_chunks : seg.h / p.G;
+    ip.g = (PK || p.packed) ? seg.h / p.pack_chunks : p.shape.hp ? (2 * seg.h) / p.G : seg.h / p.G;
     ip.jl = seg.jb;
     ip.jh = seg.je;
     ip.q_row0 = seg.q_base;
@@ -254,7 +254,7 @@ __device__ __forceinline__ ItemPlan plan_piece(const Params &p, const Segment &s
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
         const TileRole tr = tile_role(p.shape, seg, sp, t);
-        ip.q0[t] = seg.qp * 2 * kBlockQ + t * kBlockQ;
+        ip.q0[t] = p.shape.hp ? seg.qp * kBlockQ : seg.qp * 2 * kBlockQ + t * kBlockQ;
         ip.present[t] = tr.active;
         ip.lo[t] = tr.lo;
         ip.hi[t] = tr.active ? tr.hi : -1;
@@ -320,9 +320,9 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         tma_load_3d_hint(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
                                          tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0, pol_q);
-                } else {  // dense: plane b*Hq + h; varlen: packed rows, plane h
+                } else {  // dense: plane b*Hq + h (head pairs: 2h + t); varlen: packed rows, plane h
                     mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
-                    const int plane = LY == kLayoutVarlen ? ip.h : ip.b * p.Hq + ip.h;
+                    const int plane = LY == kLayoutVarlen ? ip.h : ip.b * p.Hq + (p.shape.hp ? 2 * ip.h + t : ip.h);
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         tma_load_3d_hint(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
                                          tm_q, bar.q_full(t), cb * 64, ip.q_row0 + ip.q0[t], plane, pol_q);
@@ -745,8 +745,8 @@ __device__ __forceinline__ void softmax_role(const Params &p, const int t, uint3
         const TileRole ip = tile_role(p.shape, seg, sp, t);
         if (!ip.active) continue;
         // query row of this thread (its head too, for a packed tile)
-        int row = seg.qp * 2 * kBlockQ + t * kBlockQ + r;
-        int out_head = seg.h;
+        int row = p.shape.hp ? seg.qp * kBlockQ + r : seg.qp * 2 * kBlockQ + t * kBlockQ + r;
+        int out_head = p.shape.hp ? 2 * seg.h + t : seg.h;
         bool row_valid = row < seg.L;
         const int q_tile0 = row - r;  // first row of the tile, for the tile-level mask test
         if constexpr (PK) {

@@ -45,14 +45,22 @@ struct SeqTable {
 struct Shape {
     int B, Hq, L, S, causal, window;  // varlen: L = longest query, S unused
     unsigned flags;
-    int n_qp;   // query-tile pairs per head: ceil(L / 256)
+    int n_qp;   // query-tile pairs per head: ceil(L / 256); with head pairs, ceil(L / 128)
     int grid;   // CTAs
     int split;  // 1: split schedule; 0: whole items in snake order
+    // Head pairs: an item's two tiles are the same 128-row query tile of two
+    // query heads of one KV group (Hq here counts the pairs), so both visit
+    // the same key tiles; otherwise they are two consecutive query tiles of
+    // one head, whose key ranges differ at the causal diagonal and the window.
+    int hp = 0;
 };
 
-TFA_HD int shape_n_qp(int L) { return (L + 2 * kBlockQ - 1) / (2 * kBlockQ); }
+TFA_HD int shape_n_qp(int L, int hp = 0) {
+    return hp ? (L + kBlockQ - 1) / kBlockQ : (L + 2 * kBlockQ - 1) / (2 * kBlockQ);
+}
 
-// Key-tile ranges of the two query tiles of query-tile pair qp.
+// Key-tile ranges of the two query tiles of item group qp (a query-tile pair,
+// or with head pairs one query tile of both heads).
 struct ItemSpan {
     int jl, jh;     // union range
     int lo[2], hi[2];
@@ -64,7 +72,7 @@ TFA_HD ItemSpan item_span_ls(const Shape &s, int L, int S, int qp) {
     sp.jl = 0x7fffffff;
     sp.jh = -1;
     for (int t = 0; t < 2; ++t) {
-        const int q0 = qp * 2 * kBlockQ + t * kBlockQ;
+        const int q0 = s.hp ? qp * kBlockQ : qp * 2 * kBlockQ + t * kBlockQ;
         sp.present[t] = q0 < L;
         const KeyRange kr = qtile_key_range(L, S, s.causal, s.window, q0, s.flags);
         sp.lo[t] = kr.lo;
