@@ -416,12 +416,14 @@ int launch(DeviceState &st, const void *q, const void *k, const void *v, void *o
     // consecutive query tiles spends one step on the later tile alone (the
     // diagonal, or the window's shift), which short items do not amortise;
     // measured, long items ran slower as head pairs.
-    if (!packed && !varlen && p.causal && (Hq / Hkv) % 2 == 0 &&
-        p.W <= 16LL * B * sh.Hq * sh.n_qp) {
+    // (Variable-length batches: lengths unknown here, so when the longest
+    // sequence has at most 32 query tiles.)
+    if (!packed && p.causal && (Hq / Hkv) % 2 == 0 &&
+        (varlen ? L <= 32 * tfa::kBlockQ : p.W <= 16LL * B * sh.Hq * sh.n_qp)) {
         sh.hp = 1;
         sh.Hq = Hq / 2;
         sh.n_qp = tfa::shape_n_qp(L, 1);
-        p.W = tfa::total_steps(sh);
+        if (!varlen) p.W = tfa::total_steps(sh);
     }
     const long long n_items = static_cast<long long>(B) * sh.Hq * sh.n_qp;
     // whole-item schedule, and the split one when scratch exists and the

@@ -322,7 +322,8 @@ __device__ void load_role(const Params &p, const CUtensorMap *tm_q, const CUtens
                                          tm_q, bar.q_full(t), cb * 64, 0, ip.b * p.Hq + pr.h0, pol_q);
                 } else {  // dense: plane b*Hq + h (head pairs: 2h + t); varlen: packed rows, plane h
                     mbar_arrive_expect_tx(bar.q_full(t), C::kTileBytes);
-                    const int plane = LY == kLayoutVarlen ? ip.h : ip.b * p.Hq + (p.shape.hp ? 2 * ip.h + t : ip.h);
+                    const int head = p.shape.hp ? 2 * ip.h + t : ip.h;
+                    const int plane = LY == kLayoutVarlen ? head : ip.b * p.Hq + head;
                     for (int cb = 0; cb < C::kColBlocks; ++cb)
                         tma_load_3d_hint(sbase + C::kQOff + t * C::kTileBytes + cb * C::kColBlockBytes,
                                          tm_q, bar.q_full(t), cb * 64, ip.q_row0 + ip.q0[t], plane, pol_q);
@@ -1134,7 +1135,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         int n = 1;
         while (n < p.B) n <<= 1;
         for (int i = threadIdx.x; i < n; i += kThreads) {
-            const int pairs = i < p.B ? (tab[kMaxVarlenSeqs + i] + 2 * kBlockQ - 1) / (2 * kBlockQ) : 0;
+            const int rows = p.shape.hp ? kBlockQ : 2 * kBlockQ;  // query rows per item group
+            const int pairs = i < p.B ? (tab[kMaxVarlenSeqs + i] + rows - 1) / rows : 0;
             order[i] = i < p.B ? (static_cast<unsigned>(pairs) << 10) | static_cast<unsigned>(1023 - i) : 0u;
         }
         __syncthreads();
@@ -1163,7 +1165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (order[mid] >= bound) lo = mid + 1;
                 else hi = mid;
             }
-            gstart[rr + 1] = lo * p.Hq;
+            gstart[rr + 1] = lo * p.shape.Hq;  // items per sequence: its (virtual) heads
         }
         if (threadIdx.x == 0) gstart[0] = 0;
         __syncthreads();

@@ -184,7 +184,7 @@ struct SegIter {
                     seg.S = seq.k_len[seg.b];
                     seg.q_base = seq.q_start[seg.b];
                     seg.k_base = seq.k_start[seg.b];
-                    if (seg.qp * 2 * kBlockQ >= seg.L) continue;  // no such tile pair
+                    if (seg.qp * (s.hp ? 1 : 2) * kBlockQ >= seg.L) continue;  // no such tile (pair)
                 }
                 const ItemSpan sp = seg_span(s, seg);
                 seg.jb = sp.jl;
