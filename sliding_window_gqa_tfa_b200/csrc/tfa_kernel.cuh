@@ -1124,10 +1124,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (LY == kLayoutVarlen && p.shape.n_qp <= kMaxVarlenGroups) {
         // The compact deal (the same in every CTA): sequences sorted by their
-        // query-tile pairs, longest first, by a bitonic sort of unique keys
-        // (pairs << 10 | 1023 - b) over all threads, then per group the items
-        // that exist and their prefix sums.  Without it a CTA's share of the
-        // item grid would hold empty slots where short sequences end.
+        // item groups (query-tile pairs; query tiles with head pairs), longest
+        // first, by a bitonic sort of unique keys (groups << 10 | 1023 - b)
+        // over all threads, then per group the items that exist and their
+        // prefix sums.  Without it a CTA's share of the item grid would hold
+        // empty slots where short sequences end.
         __syncthreads();  // the table is complete
         const int *tab = reinterpret_cast<const int *>(gbase + C::kTableOff);
         unsigned *order = reinterpret_cast<unsigned *>(gbase + C::kOrderOff);
@@ -1157,7 +1158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const int n_qp = p.shape.n_qp;
         for (int rr = threadIdx.x; rr < n_qp; rr += kThreads) {
-            // sequences with query-tile pair qp: those with more than qp pairs
+            // sequences with item group qp: those with more than qp groups
             const unsigned bound = static_cast<unsigned>(group_qp(p.shape, rr) + 1) << 10;
             int lo = 0, hi = p.B;
             while (lo < hi) {

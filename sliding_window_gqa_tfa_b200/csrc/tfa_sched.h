@@ -1,10 +1,11 @@
 // tfa_sched.h -- how the persistent grid divides the work (host and device).
 //
-// An *item* is (batch b, query head h, pair qp of 128-row query tiles); its
-// work is the union of the two tiles' key-tile ranges (tfa_plan.h), one *step*
-// per key tile.  Items are ordered by query-tile pair (longest first when
-// causal), then batch, then head, so the heads of one KV group -- which read
-// the same K/V -- sit next to each other.
+// An *item* is (batch b, query head h, pair qp of 128-row query tiles), or with
+// head pairs (batch b, heads 2h and 2h+1, query tile qp); its work is the union
+// of the two tiles' key-tile ranges (tfa_plan.h), one *step* per key tile.
+// Items are ordered by that group qp (longest first when causal), then batch,
+// then head, so the heads of one KV group -- which read the same K/V -- sit
+// next to each other.
 //
 // Split schedule (the default): the concatenated steps of all items are cut
 // into `grid` contiguous ranges of (almost) equal length, one per CTA, so every
@@ -31,11 +32,13 @@ namespace tfa {
 // packed row q_start[b] and k_len[b] keys from packed row k_start[b] (a
 // sequence whose lengths failed validation has q_len 0 and is skipped).
 // With `order` set, only the items that exist are dealt: order[i] low 10 bits
-// = 1023 - b, high bits = b's query-tile pairs, sorted in decreasing order
+// = 1023 - b, high bits = b's item groups (query-tile pairs, or query tiles
+// with head pairs), sorted in decreasing order
 // (longest sequences first, then by index), and group_start[rr] = the items
 // of the groups before group rr (the groups' order as for fixed lengths).
-// Group rr holds, for each of its first n sequences of `order`, every head.
-constexpr int kMaxVarlenGroups = 1024;  // query-tile pairs for the compact deal
+// Group rr holds, for each of its first n sequences of `order`, every head
+// (or head pair).
+constexpr int kMaxVarlenGroups = 1024;  // item groups for the compact deal
 struct SeqTable {
     const int *q_start, *q_len, *k_start, *k_len;
     const unsigned *order;
@@ -87,7 +90,7 @@ TFA_HD ItemSpan item_span_ls(const Shape &s, int L, int S, int qp) {
 
 TFA_HD ItemSpan item_span(const Shape &s, int qp) { return item_span_ls(s, s.L, s.S, qp); }
 
-// Items of group r all have query-tile pair group_qp(r).
+// Items of group r all have query-tile pair (or query tile) group_qp(r).
 TFA_HD int group_qp(const Shape &s, int r) { return s.causal ? s.n_qp - 1 - r : r; }
 
 TFA_HD int item_steps(const Shape &s, int qp) {
@@ -113,7 +116,7 @@ struct Segment {
     int q_base, k_base;  // varlen: first packed query / key row of the sequence
 };
 
-// Key-tile ranges of the segment's query-tile pair, for its own lengths.
+// Key-tile ranges of the segment's two tiles, for its own lengths.
 TFA_HD ItemSpan seg_span(const Shape &s, const Segment &seg) { return item_span_ls(s, seg.L, seg.S, seg.qp); }
 
 // Per-CTA iterator over its pieces, identical on every role of the CTA.
@@ -123,7 +126,7 @@ struct SegIter {
     int r, gsteps, bh;    // split: current group, steps per item in it, items per group
     // whole-item schedule: CTA c visits items c, 2G - 1 - c, 2G + c, 4G - 1 - c,
     // ... (G CTAs): the step alternates between 2G - 1 - 2c and 2c + 1, which sum
-    // to 2G.  Items come largest first (causal tile pairs in decreasing order),
+    // to 2G.  Items come largest first (causal item groups in decreasing order),
     // so alternating the direction pairs a CTA's large items with small ones.
     // Once a CTA's item is past the end, so are all its later ones.
     int item, stride, n_items;
